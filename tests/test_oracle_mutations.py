@@ -1,0 +1,106 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin fails.
+
+Each case swaps one oracle routine for a subtly wrong version (a dropped term,
+a wrong bit order, a transposed operand ...) and runs the pin that should catch
+it.  If a pin passes with the mistake in place, the pin is too weak.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.huffman as H
+import oracle.bf16 as B
+import oracle.palette as P
+import oracle.gemm as G
+import tests.test_oracle_pins as pins
+
+
+def _canonical_desc_within_length(lengths):
+    lengths = [int(l) for l in lengths]
+    codes = np.zeros(len(lengths), np.int64)
+    order = sorted(range(len(lengths)), key=lambda s: (lengths[s], -s))
+    code, prev = 0, 0
+    first = True
+    for s in order:
+        if lengths[s] == 0:
+            continue
+        if first:
+            code, prev, first = 0, lengths[s], False
+        else:
+            code = (code + 1) << (lengths[s] - prev)
+            prev = lengths[s]
+        codes[s] = code
+    return codes
+
+
+def _package_merge_keep_one_more(freqs, max_len=12):
+    lengths = H.package_merge_lengths.__wrapped__(freqs, max_len)  # type: ignore[attr-defined]
+    nz = np.nonzero(lengths)[0]
+    if nz.size > 1:
+        lengths[nz[0]] += 1  # a dropped/extra package
+    return lengths
+
+
+def _split_sign_low(w_bits):
+    b = np.asarray(w_bits, dtype=np.uint16).astype(np.uint32)
+    s = (((b & 0x7F) << 1) | ((b >> 15) & 1)).astype(np.uint8)
+    return s, ((b >> 7) & 0xFF).astype(np.uint8)
+
+
+def _encode_lsb_first(symbols, lengths, codes):
+    words, starts, total = H.encode_bitstream.__wrapped__(symbols, lengths, codes)  # type: ignore
+    rev = np.array([int(f"{int(w):032b}"[::-1], 2) for w in words], dtype=np.uint32)
+    return rev, starts, total
+
+
+def _pack_swapped(idx):
+    idx = np.asarray(idx, dtype=np.uint8)
+    return (idx[:, 1::2] | (idx[:, 0::2] << 4)).astype(np.uint8)
+
+
+def _gemm_no_transpose(x_bits, w_bits):
+    return B.to_float64(x_bits) @ B.to_float64(w_bits)
+
+
+def _palette_ties_descending(hist):
+    hist = np.asarray(hist, dtype=np.int64)
+    present = [v for v in range(256) if hist[v] > 0]
+    ranked = sorted(present, key=lambda v: (-int(hist[v]), -v))[:16]
+    filler = (v for v in range(256) if v not in ranked)
+    while len(ranked) < 16:
+        ranked.append(next(filler))
+    return np.array(ranked, np.uint8)
+
+
+CASES = [
+    ("canonical order", oracle, "canonical_codes", _canonical_desc_within_length,
+     pins.test_canonical_codes_rfc1951_example),
+    ("length off by one", oracle, "package_merge_lengths", _package_merge_keep_one_more,
+     lambda: pins.test_package_merge_matches_brute_force(5, 3)),
+    ("sign in bit 0", oracle, "split_fields", _split_sign_low,
+     pins.test_field_split_definition_values),
+    ("LSB-first stream", oracle, "encode_bitstream", _encode_lsb_first,
+     pins.test_bitstream_hand_example),
+    ("swapped nibbles", oracle, "pack_nibbles", _pack_swapped,
+     pins.test_transcode_and_nibble_order),
+    ("missing transpose", G, "gemm_fp64", _gemm_no_transpose,
+     pins.test_gemm_matches_fsum_triple_loop),
+    ("palette tie order", oracle, "build_palette", _palette_ties_descending,
+     pins.test_palette_order_and_padding),
+]
+
+
+@pytest.mark.parametrize("name,mod,attr,bad,pin", CASES, ids=[c[0] for c in CASES])
+def test_pin_catches_planted_mistake(monkeypatch, name, mod, attr, bad, pin):
+    original = getattr(mod, attr)
+    if not hasattr(original, "__wrapped__"):
+        try:
+            original.__wrapped__ = original  # let a mutant call the real routine
+        except AttributeError:
+            pass
+    monkeypatch.setattr(mod, attr, bad)
+    # the pins call the routine through the ``oracle`` package namespace
+    if mod is not oracle and hasattr(oracle, attr):
+        monkeypatch.setattr(oracle, attr, bad)
+    with pytest.raises((AssertionError, ValueError)):
+        pin()
