@@ -1,0 +1,508 @@
+#!/usr/bin/env python
+"""Benchmark of the compressed-weight hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input on the
+Llama-3.1-8B gate_proj shape (W 14336x4096 BF16 ~ N(0, 0.02), X Mx4096 ~ N(0, 1)):
+for each M in {1, 16, 64}, all four pipelines through the public C ABI
+(uw_gemm):
+
+  full            Huffman decode to BF16 in HBM -> plain tcgen05 GEMM
+  exp             exponent-only decode -> reconstructive GEMM
+  palette_rt      transcode to 4-bit palette indices -> reconstructive GEMM
+  palette_direct  reconstructive GEMM on indices transcoded at load
+
+Four independently drawn weight matrices (seeds 10, 12, 14, 16) are used in
+rotation, one per pipeline run, so every kernel reads weights that are not in
+the 126 MB L2 (each set is ~150 MB compressed + its workspace traffic).
+
+``value`` = algorithmic bytes of the whole step (sum over its kernels of the
+bytes each must move: compressed streams read, preprocessed weights written and
+read back, X read, Y written) / device time of the step, in GB/s, summed over
+ranks.  Per-kernel device times come from the library's own CUDA-event tracing
+(uw_trace_enable) recorded on the launch stream inside the timed region.
+
+Multi-GPU: replicas only (the path does not shard; each rank runs the same
+independent step), timing is the max over ranks.
+
+``--impl reference`` times the CPU oracle (test infrastructure, bit-by-bit
+canonical Huffman decode + FP64 matmul) on a bounded sample of the same
+workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Huffman decode GB/s; fused decompress-GEMM TFLOP/s & µs vs BF16 GEMM, M=1..1024"
+WORKLOAD = "gate_14336x4096"
+MS = (1, 16, 64)
+PIPES = ("full", "exp", "palette_rt", "palette_direct")
+N_SETS = 4
+REF_ROWS = 48             # oracle rows per reference-arm step (~2 s of CPU work)
+CPU_BASELINE_ROWS = 300   # oracle rows for the cpu_baseline leg (~12 s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), valid only while the kernel source is unchanged.
+TRAFFIC = {}
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------- algorithmic bytes --
+
+def _alg_bytes(kind, st, M, N, K, x_frac=1.0):
+    """Bytes a kernel launch must move at minimum: compressed streams read,
+    preprocessed weights written / read back, X read once (x_frac of it when
+    only a slice of W's rows is processed), Y written once."""
+    T = N * K
+    stream = st["bytes_stream"] + st["bytes_offsets"]
+    esc = st["bytes_escape"]
+    xy = x_frac * 2 * M * K + 2 * M * N
+    return {
+        "decode_full": stream + T + 2 * T,
+        "decode_exp": stream + T,
+        "transcode": stream + T // 2,
+        "gemm_bf16": 2 * T + xy,
+        "gemm_exp": 2 * T + xy,
+        "gemm_palette": T + T // 2 + esc + xy,
+        "splitk_fixup": 0,
+    }[kind]
+
+
+def _run_kernels(pipe):
+    pre = {"full": "decode_full", "exp": "decode_exp", "palette_rt": "transcode",
+           "palette_direct": None}[pipe]
+    gemm = {"full": "gemm_bf16", "exp": "gemm_exp"}.get(pipe, "gemm_palette")
+    return pre, gemm
+
+
+# ------------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        busy = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- CPU oracle --
+
+def cpu_oracle_sample(rows=4, ms=MS, target_s=None):
+    """Oracle on a bounded sample of the workload: the first ``rows`` rows of the
+    weight matrix as a matrix of their own, all four pipelines (bit-by-bit
+    decode / transcode, FP64 matmul) for every M.  Returns (GB/s, seconds,
+    description).  Single thread (BLAS limited to 1)."""
+    import numpy as np
+    import oracle
+    import synthdata
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    w = synthdata.workload(WORKLOAD, rows=rows)
+    n, k = w.shape
+    enc = oracle.encode(w, chunk_syms=256)
+    st = {"bytes_stream": (enc.total_bits + 7) // 8, "bytes_offsets": enc.offsets.size * 4,
+          "bytes_escape": enc.esc_exp.size + enc.esc_bits.size * 4 + enc.esc_off.size * 4}
+    xs = {m: synthdata.activation_for(WORKLOAD, m) for m in ms}
+    alg = 0
+    t0 = time.perf_counter()
+    for m in ms:
+        x = xs[m]
+        for pipe in PIPES:
+            if pipe == "full":
+                wd = oracle.decode_full(enc)
+            elif pipe == "exp":
+                wd = oracle.join_fields(enc.sm, oracle.decode_exp(enc))
+            elif pipe == "palette_rt":
+                from oracle.container import rebuild_from_palette
+                wd = rebuild_from_palette(enc, oracle.transcode_from_stream(enc))
+            else:
+                from oracle.container import rebuild_from_palette
+                packed = oracle.pack_nibbles(oracle.transcode(oracle.exponent_bytes(w),
+                                                              enc.palette, enc.esc))
+                wd = rebuild_from_palette(enc, packed)
+            y = oracle.gemm_fp64(x, wd)
+            assert y.shape == (m, n)
+            pre, gemm = _run_kernels(pipe)
+            frac = n / synthdata.WORKLOADS[WORKLOAD]["N"]  # this slice's share of X traffic
+            if pre:
+                alg += _alg_bytes(pre, st, m, n, k, frac)
+            alg += _alg_bytes(gemm, st, m, n, k, frac)
+    dt = time.perf_counter() - t0
+    if limiter is not None:
+        limiter.unregister()
+    desc = (f"first {rows} rows of {WORKLOAD} ({rows * k} weights) encoded on their own; "
+            f"4 pipelines x M in {list(ms)}; oracle bit-by-bit decode + FP64 matmul, 1 thread")
+    return alg / dt / 1e9, dt, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for _ in range(max(args.warmup, 0)):
+        cpu_oracle_sample(rows=REF_ROWS)
+    vals, secs = [], []
+    desc = ""
+    for _ in range(args.steps):
+        v, dt, desc = cpu_oracle_sample(rows=REF_ROWS)
+        vals.append(v)
+        secs.append(dt)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8+f64", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD} sample", "Ms": list(MS), "pipelines": list(PIPES)},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- our arm ----
+
+def _load_build():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("uw_build", os.path.join(ROOT, "decode_gemm_b200",
+                                                                            "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _kernel_src_sha():
+    h = hashlib.sha256()
+    for f in ("decode.cu", "gemm.cu", "gemm_sm100.cuh", "bf16_fields.cuh"):
+        with open(os.path.join(ROOT, "decode_gemm_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    _load_build().build()
+    import decode_gemm_b200 as uw
+    import synthdata
+
+    wl = synthdata.WORKLOADS[args.workload]
+    N, K = wl["N"], wl["K"]
+    Ms = tuple(wl["Ms"]) if args.workload != WORKLOAD else MS
+    stream = torch.cuda.current_stream()
+
+    # weights: N_SETS independent draws of the same shape, encoded and resident
+    handles, stats = [], []
+    for i in range(N_SETS):
+        if wl["kind"] == "normal":
+            w = synthdata.normal(N, K, wl["std"], wl["seed_w"] + 2 * i)
+        else:
+            w = synthdata.student_t(N, K, wl["nu"], wl["std"], wl["seed_w"] + 2 * i)
+        h = uw.uw_encode(w, stream=stream)
+        handles.append(h)
+        stats.append(h.stats())
+        del w
+    need = max(uw.uw_workspace_bytes(handles[0], uw.PIPELINES[p], m) for p in PIPES for m in Ms)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    for h in handles:
+        uw.uw_set_workspace(h, ws)
+    X = {m: torch.from_numpy(synthdata.activations(m, K, wl["seed_x"] + m).view(np.int16))
+         .cuda().view(torch.bfloat16) for m in Ms}
+    Y = {(m, p): torch.empty((m, N), dtype=torch.bfloat16, device="cuda") for m in Ms for p in PIPES}
+    runs = [(m, p) for m in Ms for p in PIPES]
+
+    def step(run0):
+        for j, (m, p) in enumerate(runs):
+            h = handles[(run0 + j) % N_SETS]
+            uw.uw_gemm(h, X[m], Y[(m, p)], m, uw.PIPELINES[p])
+        return run0 + len(runs)
+
+    # algorithmic bytes of one step (depends only on the rotation position)
+    def step_bytes(run0):
+        tot = 0
+        for j, (m, p) in enumerate(runs):
+            st = stats[(run0 + j) % N_SETS]
+            pre, gemm = _run_kernels(p)
+            if pre:
+                tot += _alg_bytes(pre, st, m, N, K)
+            tot += _alg_bytes(gemm, st, m, N, K)
+        return tot
+
+    run0 = 0
+    for _ in range(args.warmup):
+        run0 = step(run0)
+    torch.cuda.synchronize()
+    for h in handles:
+        uw.uw_trace_read(h)  # discard warm-up records
+        uw.uw_trace_enable(h, True)
+
+    # ---- device-resident timed region
+    total_bytes = sum(step_bytes(run0 + s * len(runs)) for s in range(args.steps))
+    run_start = run0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            run0 = step(run0)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    traces = [uw.uw_trace_read(h) for h in handles]
+    for h in handles:
+        uw.uw_trace_enable(h, False)
+    for h in handles:
+        st = uw.uw_last_device_status(h)
+        if st != uw.UW_OK:
+            raise RuntimeError(f"device status {uw.uw_status_str(st)}")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = total_bytes / (elapsed_ms * 1e-3) / 1e9 * world
+
+    # ---- per-kernel attribution from the traces (runs rotate over handles)
+    per_kind = {}
+    per_run = {}
+    cursor = [0] * N_SETS
+    launches = sum(len(t) for t in traces)
+    for s in range(args.steps):
+        for j, (m, p) in enumerate(runs):
+            idx = (run_start + s * len(runs) + j) % N_SETS
+            tr = traces[idx]
+            pre, gemm = _run_kernels(p)
+            st = stats[idx]
+            rec = {}
+            for kind in ([pre] if pre else []) + [gemm, "splitk_fixup"]:
+                c = cursor[idx]
+                if c < len(tr) and tr[c][0] == kind:
+                    rec[kind] = tr[c][1]
+                    cursor[idx] += 1
+                    b = _alg_bytes(kind, st, m, N, K)
+                    agg = per_kind.setdefault(kind, {"ms": 0.0, "n": 0, "bytes": 0, "flops": 0})
+                    agg["ms"] += tr[c][1]
+                    agg["n"] += 1
+                    agg["bytes"] += b
+                    if kind.startswith("gemm"):
+                        agg["flops"] += 2 * m * N * K
+            per_run.setdefault((m, p), []).append(rec)
+    dominant = max(per_kind, key=lambda k: per_kind[k]["ms"])
+    peaks, peak_src = _peaks()
+    d = per_kind[dominant]
+    achieved = d["bytes"] / (d["ms"] * 1e-3) / 1e9
+    traffic = TRAFFIC.get(dominant)
+    if traffic and traffic.get("src_sha") != _kernel_src_sha():
+        traffic = None
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": traffic["bytes_per_launch"] if traffic else None,
+                "algorithmic_bytes_per_launch": d["bytes"] / d["n"],
+                "avg_launch_us": 1e3 * d["ms"] / d["n"], "peak_source": peak_src}
+    kernels = {k: {"launches": v["n"], "total_ms": v["ms"], "share": v["ms"] / elapsed_ms,
+                   "GBps": v["bytes"] / (v["ms"] * 1e-3) / 1e9 if v["ms"] > 0 else None,
+                   "frac_hbm": (v["bytes"] / (v["ms"] * 1e-3) / 1e9) / peaks["hbm_gbs"]
+                   if v["ms"] > 0 else None}
+               for k, v in per_kind.items()}
+    pipelines = {}
+    for (m, p), recs in per_run.items():
+        def med(kind):
+            xs = [r[kind] for r in recs if kind in r]
+            return 1e3 * statistics.median(xs) if xs else None
+        pre, gemm = _run_kernels(p)
+        g = med(gemm) or 0.0
+        fx = med("splitk_fixup") or 0.0
+        pr = med(pre) if pre else 0.0
+        pipelines[f"{p}/M{m}"] = {"preprocess_us": pr, "gemm_us": g + fx, "total_us": pr + g + fx,
+                                  "gemm_tflops": 2 * m * N * K / ((g + fx) * 1e-6) / 1e12
+                                  if g + fx > 0 else None}
+
+    # ---- BF16 torch.matmul on the same box (context only)
+    wbf = []
+    for h in handles:
+        t = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+        uw.uw_decode_full(h, t)
+        wbf.append(t)
+    torch.cuda.synchronize()
+    tm = {}
+    for m in Ms:
+        ts = []
+        for it in range(3 + 12):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            torch.matmul(X[m], wbf[it % N_SETS].t())
+            b.record(stream)
+            b.synchronize()
+            if it >= 3:
+                ts.append(a.elapsed_time(b) * 1e3)
+        tm[f"M{m}"] = statistics.median(ts)
+    del wbf
+
+    # ---- end to end through the public call with host buffers
+    Xh = {m: X[m].cpu().pin_memory() for m in Ms}
+    Yh = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in Y.items()}
+    h2d = sum(x.numel() * 2 for x in Xh.values())
+    d2h = sum(y.numel() * 2 for y in Yh.values())
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    run_e = run0
+    e2e_bytes = 0
+    for _ in range(args.steps):
+        for m in Ms:
+            X[m].copy_(Xh[m], non_blocking=True)
+        e2e_bytes += step_bytes(run_e)
+        run_e = step(run_e)
+        for k in Y:
+            Yh[k].copy_(Y[k], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = e2e_bytes / (e2e_ms * 1e-3) / 1e9 * world
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, desc = cpu_oracle_sample(rows=CPU_BASELINE_ROWS)
+        cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    st0 = stats[0]
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8 (decode) / bf16 x bf16 -> fp32 (gemm)",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "N": N, "K": K, "Ms": list(Ms),
+                   "pipelines": list(PIPES), "weight_sets": N_SETS,
+                   "l2": f"{N_SETS} weight sets rotated per pipeline run, inputs > L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "bits_per_exponent": st0["bits_per_exponent"],
+                   "escape_row_fraction": st0["n_escape_rows"] / st0["n_rows"]},
+        "roofline": roofline,
+        "kernels": kernels,
+        "pipelines": pipelines,
+        "torch_matmul_bf16_us": tm,
+        "gpu_launches": launches,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+        "kernel_src_sha": _kernel_src_sha(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for h in handles:
+        h.free()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,404 @@
+"""Python binding of libunweight (lossless BF16 weight compression fused with the matmul).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library ``libunweight.so`` built in this directory (``python
+decode_gemm_b200/build.py``).  Importing this package fails loudly when the
+library is missing; there is no Python or CPU fallback.
+
+The functions carry the names of the C ABI in ``include/unweight.h``.  Tensors
+are ``torch`` tensors on the GPU (device memory and streams come from torch);
+host arrays are ``numpy`` arrays.  Every call raises :class:`UwError` when the
+library returns a status other than ``UW_OK``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libunweight.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python decode_gemm_b200/build.py` "
+        "(nvcc, sm_100a). There is no fallback implementation.")
+
+lib = C.CDLL(LIB_PATH)
+
+# ----------------------------------------------------------------- constants --
+UW_OK, UW_ERR_ARG, UW_ERR_SHAPE, UW_ERR_FORMAT, UW_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
+UW_ERR_OOM, UW_ERR_CUDA, UW_ERR_DEVICE, UW_ERR_TIMEOUT, UW_ERR_WORKSPACE = 5, 6, 7, 8, 9
+UW_PIPE_AUTO, UW_PIPE_FULL, UW_PIPE_EXP, UW_PIPE_PALETTE_RT, UW_PIPE_PALETTE_DIRECT = 0, 1, 2, 3, 4
+PIPELINES = {"full": UW_PIPE_FULL, "exp": UW_PIPE_EXP, "palette_rt": UW_PIPE_PALETTE_RT,
+             "palette_direct": UW_PIPE_PALETTE_DIRECT}
+
+
+class uw_encode_opts(C.Structure):
+    _fields_ = [("max_code_len", C.c_int32), ("chunk_syms", C.c_int32),
+                ("prepare_direct", C.c_int32), ("reserved", C.c_int32)]
+
+
+class uw_format(C.Structure):
+    _fields_ = [
+        ("N", C.c_int64), ("K", C.c_int64),
+        ("max_code_len", C.c_int32), ("chunk_syms", C.c_int32),
+        ("code_len", C.c_uint8 * 256), ("palette", C.c_uint8 * 16),
+        ("n_words", C.c_int64), ("words", C.POINTER(C.c_uint32)),
+        ("n_chunks", C.c_int64), ("chunk_off", C.POINTER(C.c_uint32)),
+        ("sm", C.POINTER(C.c_uint8)),
+        ("n_esc_words", C.c_int64), ("esc_bits", C.POINTER(C.c_uint32)),
+        ("n_esc_groups", C.c_int64), ("esc_off", C.POINTER(C.c_uint32)),
+        ("n_esc_rows", C.c_int64), ("esc_exp", C.POINTER(C.c_uint8)),
+    ]
+
+
+class uw_stats_t(C.Structure):
+    _fields_ = [
+        ("N", C.c_int64), ("K", C.c_int64),
+        ("bits_per_exponent", C.c_double), ("entropy_bits", C.c_double),
+        ("top16_coverage", C.c_double),
+        ("n_rows", C.c_int64), ("n_escape_rows", C.c_int64),
+        ("max_len_used", C.c_int32), ("n_symbols", C.c_int32),
+        ("bytes_stream", C.c_int64), ("bytes_offsets", C.c_int64), ("bytes_sm", C.c_int64),
+        ("bytes_escape", C.c_int64), ("bytes_palette_idx", C.c_int64),
+        ("bytes_huffman_bundle", C.c_int64), ("bytes_palette_bundle", C.c_int64),
+    ]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class uw_gemm_config(C.Structure):
+    _fields_ = [("pipeline", C.c_int32), ("tile_n", C.c_int32), ("stages", C.c_int32),
+                ("gemm_ctas", C.c_int32), ("decode_ctas", C.c_int32),
+                ("reserved", C.c_int32 * 3)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k in ("pipeline", "tile_n", "stages", "gemm_ctas",
+                                               "decode_ctas")}
+
+
+_vp, _i32, _i64, _sz = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
+_SIGS = {
+    "uw_status_str": ([C.c_int], C.c_char_p),
+    "uw_abi_version": ([], C.c_int),
+    "uw_default_encode_opts": ([C.POINTER(uw_encode_opts)], None),
+    "uw_encode_host": ([_vp, _i64, _i64, C.POINTER(uw_encode_opts), C.POINTER(_vp)], C.c_int),
+    "uw_host_view": ([_vp, C.POINTER(uw_format)], C.c_int),
+    "uw_host_free": ([_vp], None),
+    "uw_validate_format": ([C.POINTER(uw_format)], C.c_int),
+    "uw_host_stats": ([_vp, C.POINTER(uw_stats_t)], C.c_int),
+    "uw_upload": ([C.POINTER(uw_format), C.POINTER(uw_encode_opts), _vp, C.POINTER(_vp)], C.c_int),
+    "uw_encode": ([_vp, _i64, _i64, C.POINTER(uw_encode_opts), _vp, C.POINTER(_vp)], C.c_int),
+    "uw_free": ([_vp], C.c_int),
+    "uw_set_stream": ([_vp, _vp], C.c_int),
+    "uw_stats": ([_vp, C.POINTER(uw_stats_t)], C.c_int),
+    "uw_workspace_bytes": ([_vp, _i32, _i64, C.POINTER(_sz)], C.c_int),
+    "uw_set_workspace": ([_vp, _vp, _sz], C.c_int),
+    "uw_alloc_workspace": ([_vp, _sz], C.c_int),
+    "uw_decode_full": ([_vp, _vp], C.c_int),
+    "uw_decode_exp": ([_vp, _vp], C.c_int),
+    "uw_transcode_palette": ([_vp, _vp], C.c_int),
+    "uw_gemm": ([_vp, _vp, _vp, _i64, C.c_int], C.c_int),
+    "uw_gemm_f32": ([_vp, _vp, _vp, _i64, C.c_int], C.c_int),
+    "uw_gemm_ex": ([_vp, _vp, _vp, _i64, C.POINTER(uw_gemm_config), _i32], C.c_int),
+    "uw_autotune": ([C.POINTER(_vp), _i32, C.POINTER(_i64), _i32, C.c_char_p], C.c_int),
+    "uw_load_profile": ([C.POINTER(_vp), _i32, C.c_char_p], C.c_int),
+    "uw_get_choice": ([_vp, _i64, C.POINTER(uw_gemm_config)], C.c_int),
+    "uw_last_device_status": ([_vp], C.c_int),
+    "uw_trace_enable": ([_vp, _i32], C.c_int),
+    "uw_trace_read": ([_vp, C.POINTER(_i32), C.POINTER(C.c_float), _i32, C.POINTER(_i32)], C.c_int),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+class UwError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = int(status)
+        super().__init__(f"{what}: {uw_status_str(status)} ({status})")
+
+
+def uw_status_str(status: int) -> str:
+    return lib.uw_status_str(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != UW_OK:
+        raise UwError(status, what)
+
+
+def default_opts(**kw) -> uw_encode_opts:
+    o = uw_encode_opts()
+    lib.uw_default_encode_opts(C.byref(o))
+    for k, v in kw.items():
+        setattr(o, k, int(v))
+    return o
+
+
+def _stream_ptr(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _dptr(t) -> int:
+    return int(t.data_ptr())
+
+
+# ------------------------------------------------------------------ host side --
+
+class HostEncoded:
+    """Host-side encoding (``uw_encode_host``); numpy views via :meth:`arrays`."""
+
+    def __init__(self, ptr):
+        self._ptr = _vp(ptr)
+
+    @property
+    def ptr(self):
+        return self._ptr
+
+    def view(self) -> uw_format:
+        f = uw_format()
+        _check(lib.uw_host_view(self._ptr, C.byref(f)), "uw_host_view")
+        return f
+
+    def arrays(self) -> dict:
+        return format_arrays(self.view())
+
+    def stats(self) -> dict:
+        s = uw_stats_t()
+        _check(lib.uw_host_stats(self._ptr, C.byref(s)), "uw_host_stats")
+        return s.as_dict()
+
+    def __del__(self):
+        if getattr(self, "_ptr", None) and self._ptr.value:
+            lib.uw_host_free(self._ptr)
+            self._ptr = _vp(0)
+
+
+def uw_encode_host(w: np.ndarray, opts: uw_encode_opts | None = None) -> HostEncoded:
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    n, k = w.shape
+    out = _vp()
+    _check(lib.uw_encode_host(w.ctypes.data, n, k, C.byref(opts) if opts else None,
+                              C.byref(out)), "uw_encode_host")
+    return HostEncoded(out.value)
+
+
+def format_arrays(f: uw_format) -> dict:
+    """Copy every array of a format view into numpy."""
+    def arr(ptr, n, dt):
+        n = int(n)
+        if n == 0:
+            return np.zeros(0, dt)
+        return np.ctypeslib.as_array(ptr, shape=(n,)).copy().astype(dt)
+    return dict(
+        N=f.N, K=f.K, max_code_len=f.max_code_len, chunk_syms=f.chunk_syms,
+        code_len=np.array(f.code_len[:], np.uint8), palette=np.array(f.palette[:], np.uint8),
+        words=arr(f.words, f.n_words, np.uint32),
+        chunk_off=arr(f.chunk_off, f.n_chunks + 1, np.uint32),
+        sm=arr(f.sm, f.N * f.K, np.uint8),
+        esc_bits=arr(f.esc_bits, f.n_esc_words, np.uint32),
+        esc_off=arr(f.esc_off, f.n_esc_groups + 1, np.uint32),
+        esc_exp=arr(f.esc_exp, f.n_esc_rows * 64, np.uint8),
+    )
+
+
+class FormatBuffers:
+    """A ``uw_format`` that points into numpy arrays it keeps alive."""
+
+    def __init__(self, N, K, max_code_len, chunk_syms, code_len, palette, words, chunk_off, sm,
+                 esc_bits, esc_off, esc_exp):
+        self._keep = []
+
+        def ptr(a, ct):
+            a = np.ascontiguousarray(a)
+            self._keep.append(a)
+            return a.ctypes.data_as(C.POINTER(ct))
+
+        f = uw_format()
+        f.N, f.K = int(N), int(K)
+        f.max_code_len, f.chunk_syms = int(max_code_len), int(chunk_syms)
+        f.code_len[:] = [int(x) for x in np.asarray(code_len, np.uint8)]
+        f.palette[:] = [int(x) for x in np.asarray(palette, np.uint8)]
+        words = np.asarray(words, np.uint32)
+        f.n_words, f.words = words.size, ptr(words, C.c_uint32)
+        chunk_off = np.asarray(chunk_off, np.uint32)
+        f.n_chunks, f.chunk_off = chunk_off.size - 1, ptr(chunk_off, C.c_uint32)
+        f.sm = ptr(np.asarray(sm, np.uint8).reshape(-1), C.c_uint8)
+        esc_bits = np.asarray(esc_bits, np.uint32).reshape(-1)
+        f.n_esc_words, f.esc_bits = esc_bits.size, ptr(esc_bits, C.c_uint32)
+        esc_off = np.asarray(esc_off, np.uint32)
+        f.n_esc_groups, f.esc_off = esc_off.size - 1, ptr(esc_off, C.c_uint32)
+        esc_exp = np.asarray(esc_exp, np.uint8).reshape(-1)
+        f.n_esc_rows = esc_exp.size // 64
+        f.esc_exp = ptr(esc_exp if esc_exp.size else np.zeros(64, np.uint8), C.c_uint8)
+        self.fmt = f
+
+
+def uw_validate_format(fmt: uw_format) -> int:
+    """Returns the status code (does not raise): UW_OK or an error."""
+    return int(lib.uw_validate_format(C.byref(fmt)))
+
+
+# ---------------------------------------------------------------- device side --
+
+class Handle:
+    """A device-resident encoded matrix (``uw_handle_t``)."""
+
+    def __init__(self, ptr, N, K):
+        self._ptr = _vp(ptr)
+        self.N, self.K = int(N), int(K)
+        self._ws = None  # torch tensor kept alive while registered
+
+    @property
+    def ptr(self):
+        return self._ptr
+
+    def stats(self) -> dict:
+        s = uw_stats_t()
+        _check(lib.uw_stats(self._ptr, C.byref(s)), "uw_stats")
+        return s.as_dict()
+
+    def free(self):
+        if getattr(self, "_ptr", None) is not None and self._ptr.value:
+            lib.uw_free(self._ptr)
+            self._ptr = _vp(0)
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def uw_upload(fmt: uw_format, opts: uw_encode_opts | None = None, stream=None) -> Handle:
+    out = _vp()
+    _check(lib.uw_upload(C.byref(fmt), C.byref(opts) if opts else None,
+                         _vp(_stream_ptr(stream)), C.byref(out)), "uw_upload")
+    return Handle(out.value, fmt.N, fmt.K)
+
+
+def uw_encode(w: np.ndarray, opts: uw_encode_opts | None = None, stream=None) -> Handle:
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    n, k = w.shape
+    out = _vp()
+    _check(lib.uw_encode(w.ctypes.data, n, k, C.byref(opts) if opts else None,
+                         _vp(_stream_ptr(stream)), C.byref(out)), "uw_encode")
+    return Handle(out.value, n, k)
+
+
+def uw_free(h: Handle) -> None:
+    h.free()
+
+
+def uw_set_stream(h: Handle, stream=None) -> None:
+    _check(lib.uw_set_stream(h.ptr, _vp(_stream_ptr(stream))), "uw_set_stream")
+
+
+def uw_stats(h: Handle) -> dict:
+    return h.stats()
+
+
+def uw_workspace_bytes(h: Handle, pipeline: int, M: int) -> int:
+    out = _sz()
+    _check(lib.uw_workspace_bytes(h.ptr, int(pipeline), int(M), C.byref(out)),
+           "uw_workspace_bytes")
+    return int(out.value)
+
+
+def uw_set_workspace(h: Handle, ws) -> None:
+    """Register a caller-owned device buffer (a torch tensor; kept alive here)."""
+    if ws is None:
+        _check(lib.uw_set_workspace(h.ptr, None, 0), "uw_set_workspace")
+        h._ws = None
+        return
+    nbytes = ws.numel() * ws.element_size()
+    _check(lib.uw_set_workspace(h.ptr, _vp(_dptr(ws)), nbytes), "uw_set_workspace")
+    h._ws = ws
+
+
+def uw_alloc_workspace(h: Handle, nbytes: int) -> None:
+    _check(lib.uw_alloc_workspace(h.ptr, int(nbytes)), "uw_alloc_workspace")
+
+
+def uw_decode_full(h: Handle, w_out) -> None:
+    _check(lib.uw_decode_full(h.ptr, _vp(_dptr(w_out))), "uw_decode_full")
+
+
+def uw_decode_exp(h: Handle, e_out) -> None:
+    _check(lib.uw_decode_exp(h.ptr, _vp(_dptr(e_out))), "uw_decode_exp")
+
+
+def uw_transcode_palette(h: Handle, idx_out) -> None:
+    _check(lib.uw_transcode_palette(h.ptr, _vp(_dptr(idx_out))), "uw_transcode_palette")
+
+
+def uw_gemm(h: Handle, X, Y, M: int, pipeline: int = UW_PIPE_AUTO) -> None:
+    _check(lib.uw_gemm(h.ptr, _vp(_dptr(X)), _vp(_dptr(Y)), int(M), int(pipeline)), "uw_gemm")
+
+
+def uw_gemm_f32(h: Handle, X, Y, M: int, pipeline: int = UW_PIPE_AUTO) -> None:
+    _check(lib.uw_gemm_f32(h.ptr, _vp(_dptr(X)), _vp(_dptr(Y)), int(M), int(pipeline)),
+           "uw_gemm_f32")
+
+
+def gemm_config(pipeline: int, tile_n: int = 0, stages: int = 0, gemm_ctas: int = 0,
+                decode_ctas: int = 0) -> uw_gemm_config:
+    c = uw_gemm_config()
+    c.pipeline, c.tile_n, c.stages = int(pipeline), int(tile_n), int(stages)
+    c.gemm_ctas, c.decode_ctas = int(gemm_ctas), int(decode_ctas)
+    return c
+
+
+def uw_gemm_ex(h: Handle, X, Y, M: int, cfg: uw_gemm_config, out_f32: bool) -> None:
+    _check(lib.uw_gemm_ex(h.ptr, _vp(_dptr(X)), _vp(_dptr(Y)), int(M), C.byref(cfg),
+                          1 if out_f32 else 0), "uw_gemm_ex")
+
+
+def uw_autotune(handles, Ms, profile_out_json: str | None = None) -> None:
+    arr = (_vp * len(handles))(*[h.ptr for h in handles])
+    ms = (_i64 * len(Ms))(*[int(m) for m in Ms])
+    _check(lib.uw_autotune(arr, len(handles), ms, len(Ms),
+                           profile_out_json.encode() if profile_out_json else None), "uw_autotune")
+
+
+def uw_load_profile(handles, profile_json: str) -> None:
+    arr = (_vp * len(handles))(*[h.ptr for h in handles])
+    _check(lib.uw_load_profile(arr, len(handles), profile_json.encode()), "uw_load_profile")
+
+
+def uw_get_choice(h: Handle, M: int) -> dict:
+    c = uw_gemm_config()
+    _check(lib.uw_get_choice(h.ptr, int(M), C.byref(c)), "uw_get_choice")
+    return c.as_dict()
+
+
+KERNEL_KINDS = ("decode_full", "decode_exp", "transcode", "gemm_bf16", "gemm_exp",
+                "gemm_palette", "splitk_fixup")
+
+
+def uw_trace_enable(h: Handle, enable: bool = True) -> None:
+    _check(lib.uw_trace_enable(h.ptr, 1 if enable else 0), "uw_trace_enable")
+
+
+def uw_trace_read(h: Handle, capacity: int = 16384):
+    """[(kernel kind name, milliseconds)] of the launches traced since the last read."""
+    kinds = (_i32 * capacity)()
+    ms = (C.c_float * capacity)()
+    n = _i32()
+    _check(lib.uw_trace_read(h.ptr, kinds, ms, capacity, C.byref(n)), "uw_trace_read")
+    return [(KERNEL_KINDS[kinds[i]], float(ms[i])) for i in range(min(n.value, capacity))]
+
+
+def uw_last_device_status(h: Handle) -> int:
+    """Synchronises the handle's stream; returns (does not raise) the device status."""
+    return int(lib.uw_last_device_status(h.ptr))

@@ -1,0 +1,524 @@
+// C ABI, device side: upload, preprocessing entry points, GEMM dispatch over
+// the four pipelines, workspace and status handling.
+//
+// *Unweight*, "Four ways to use compressed weights": pipeline 1 decodes to
+// BF16 in HBM and runs a plain GEMM; pipeline 2 decodes exponent bytes only,
+// pipeline 3 transcodes to 4-bit palette indices at run time, pipeline 4 uses
+// indices transcoded once at load; 2-4 run the reconstructive GEMM.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <new>
+
+#include "handle.h"
+
+using namespace uw;
+
+namespace {
+
+uw_status map_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return UW_OK;
+  if (e == cudaErrorMemoryAllocation) return UW_ERR_OOM;
+  return UW_ERR_CUDA;
+}
+
+#define UW_CK(x)                                  \
+  do {                                            \
+    cudaError_t e_ = (x);                         \
+    if (e_ != cudaSuccess) return map_cuda(e_);   \
+  } while (0)
+
+// Make the handle's device current for the scope of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool changed = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+      changed = cudaSetDevice(dev) == cudaSuccess;
+    }
+  }
+  ~DeviceGuard() {
+    if (changed) cudaSetDevice(prev);
+  }
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+void free_handle(uw_handle_s* h) {
+  if (!h) return;
+  DeviceGuard g(h->device);
+  for (cudaEvent_t ev : h->trace_events) cudaEventDestroy(ev);
+  if (h->d_block) cudaFree(h->d_block);
+  if (h->ws_owned && h->ws) cudaFree(h->ws);
+  delete h;
+}
+
+// bytes of preprocessed weights a pipeline writes to the workspace
+size_t preprocess_bytes(const uw_handle_s* h, int pipeline) {
+  const size_t T = (size_t)h->N * (size_t)h->K;
+  switch (pipeline) {
+    case UW_PIPE_FULL: return 2 * T;
+    case UW_PIPE_EXP: return T;
+    case UW_PIPE_PALETTE_RT: return T / 2;
+    default: return 0;
+  }
+}
+
+GemmArgs base_gemm_args(const uw_handle_s* h) {
+  GemmArgs a;
+  a.N = h->N;
+  a.K = h->K;
+  a.S = h->d_sm;
+  a.esc_bits = h->d_esc_bits;
+  a.esc_off = h->d_esc_off;
+  a.esc_exp = h->d_esc_exp;
+  a.esc_nw = (int32_t)(4 * ((h->N + kEscGroupRows - 1) / kEscGroupRows));
+  std::memcpy(a.palette, h->palette, 16);
+  a.sm_count = h->sm_count;
+  a.status = h->d_status;
+  return a;
+}
+
+bool valid_pipeline(int p) { return p >= UW_PIPE_FULL && p <= UW_PIPE_PALETTE_DIRECT; }
+
+}  // namespace
+
+namespace uw {
+DecodeArgs decode_args(const uw_handle_s* h) {
+  DecodeArgs a;
+  a.words = h->d_words;
+  a.chunk_off = h->d_chunk_off;
+  a.lut = h->d_exp_lut;
+  a.limit = h->d_limit;
+  a.sm = h->d_sm;
+  a.esc_bits = h->d_esc_bits;
+  a.status = h->d_status;
+  a.n_words = h->n_words;
+  a.n_chunks = h->n_chunks;
+  a.total_syms = h->N * h->K;
+  a.chunk_syms = h->chunk_syms;
+  a.kb_per_row = (int32_t)(h->K / kRow);
+  a.esc_nw = (int32_t)(4 * ((h->N + kEscGroupRows - 1) / kEscGroupRows));
+  return a;
+}
+
+// Choose the variant for (handle, M): the profile entry for the smallest tuned
+// M at or above the request (else the largest), otherwise a static default.
+uw_gemm_config choose_variant(const uw_handle_s* h, int64_t M) {
+  uw_gemm_config c;
+  std::memset(&c, 0, sizeof(c));
+  if (!h->profile.empty()) {
+    auto it = h->profile.lower_bound(M);
+    if (it == h->profile.end()) --it;
+    c = it->second;
+    if (c.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) c.pipeline = UW_PIPE_PALETTE_RT;
+    return c;
+  }
+  c.pipeline = h->d_pal_idx ? UW_PIPE_PALETTE_DIRECT : UW_PIPE_PALETTE_RT;
+  return c;
+}
+
+constexpr int kTraceCap = 16384;
+
+int trace_begin(uw_handle_s* h, int kind) {
+  if (!h->trace || (int)h->trace_kinds.size() >= kTraceCap) return -1;
+  const int slot = (int)h->trace_kinds.size();
+  while ((int)h->trace_events.size() < 2 * (slot + 1)) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return -1;
+    h->trace_events.push_back(ev);
+  }
+  if (cudaEventRecord(h->trace_events[2 * slot], h->stream) != cudaSuccess) return -1;
+  h->trace_kinds.push_back(kind);
+  return slot;
+}
+
+void trace_end(uw_handle_s* h, int slot) {
+  if (slot >= 0) cudaEventRecord(h->trace_events[2 * slot + 1], h->stream);
+}
+
+static int hook_begin(void* ctx, int kind) { return trace_begin(static_cast<uw_handle_s*>(ctx), kind); }
+static void hook_end(void* ctx, int slot) { trace_end(static_cast<uw_handle_s*>(ctx), slot); }
+
+uw_status run_decode(uw_handle_s* h, int mode, void* out, int ctas, cudaStream_t s) {
+  DecodeArgs a = decode_args(h);
+  a.lut = mode == kDecodePalette ? h->d_pal_lut : h->d_exp_lut;
+  // kinds: 0 full, 1 exponent, 2 transcode
+  const int kind = mode == kDecodeFull ? 0 : (mode == kDecodeExp ? 1 : 2);
+  const int slot = trace_begin(h, kind);
+  const cudaError_t e = launch_decode(mode, a, out, ctas, s);
+  trace_end(h, slot);
+  return map_cuda(e);
+}
+
+// Resolve a GEMM request into kernel arguments and the workspace it needs.
+uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
+                    const uw_gemm_config& cfg, int out_f32, GemmArgs* ga, size_t* ws_need,
+                    size_t* pre_bytes) {
+  GemmArgs a = base_gemm_args(h);
+  a.M = M;
+  a.X = X;
+  a.Y = Y;
+  a.out_f32 = out_f32;
+  a.tile_n = cfg.tile_n;
+  a.stages = cfg.stages;
+  a.ctas = cfg.gemm_ctas;
+  switch (cfg.pipeline) {
+    case UW_PIPE_FULL: a.mode = kGemmBf16; break;
+    case UW_PIPE_EXP: a.mode = kGemmExp; break;
+    default: a.mode = kGemmPalette; break;
+  }
+  if (!gemm_resolve(&a)) return UW_ERR_UNSUPPORTED;
+  const size_t pre = align_up(preprocess_bytes(h, cfg.pipeline), 256);
+  a.partials_bytes = gemm_partials_bytes(a);
+  *pre_bytes = pre;
+  *ws_need = pre + a.partials_bytes;
+  *ga = a;
+  return UW_OK;
+}
+
+uw_status run_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
+                   const uw_gemm_config& cfg_in, int out_f32) {
+  uw_gemm_config cfg = cfg_in;
+  if (cfg.pipeline == UW_PIPE_AUTO) {
+    const uw_gemm_config c = choose_variant(h, M);
+    cfg = c;
+  }
+  if (!valid_pipeline(cfg.pipeline)) return UW_ERR_ARG;
+  if (cfg.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) return UW_ERR_UNSUPPORTED;
+  if (cfg.tile_n < 0 || cfg.tile_n > 256 || cfg.tile_n % 16) return UW_ERR_ARG;
+  if (cfg.stages < 0 || cfg.stages > 8 || cfg.stages == 1) return UW_ERR_ARG;
+  if (cfg.gemm_ctas < 0 || cfg.decode_ctas < 0) return UW_ERR_ARG;
+  GemmArgs a;
+  size_t need = 0, pre = 0;
+  uw_status st = plan_gemm(h, X, Y, M, cfg, out_f32, &a, &need, &pre);
+  if (st != UW_OK) return st;
+  if (need > 0 && (!h->ws || h->ws_bytes < need)) return UW_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(h->ws);
+  a.partials = a.partials_bytes ? reinterpret_cast<float*>(ws + pre) : nullptr;
+  cudaStream_t s = h->stream;
+  switch (cfg.pipeline) {
+    case UW_PIPE_FULL:
+      st = run_decode(h, kDecodeFull, ws, cfg.decode_ctas, s);
+      a.W = reinterpret_cast<const uint16_t*>(ws);
+      break;
+    case UW_PIPE_EXP:
+      st = run_decode(h, kDecodeExp, ws, cfg.decode_ctas, s);
+      a.E = ws;
+      break;
+    case UW_PIPE_PALETTE_RT:
+      st = run_decode(h, kDecodePalette, ws, cfg.decode_ctas, s);
+      a.I = ws;
+      break;
+    default:
+      a.I = h->d_pal_idx;
+      break;
+  }
+  if (st != UW_OK) return st;
+  LaunchHooks hooks;
+  hooks.ctx = h;
+  hooks.begin = hook_begin;
+  hooks.end = hook_end;
+  return map_cuda(launch_gemm(a, s, &hooks));
+}
+}  // namespace uw
+
+extern "C" {
+
+uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream,
+                    uw_handle_t* out) {
+  if (!out) return UW_ERR_ARG;
+  *out = nullptr;
+  const uw_status vs = uw_validate_format(f);
+  if (vs != UW_OK) return vs;
+  uw_encode_opts o;
+  uw_default_encode_opts(&o);
+  if (opts) o = *opts;
+  uw_handle_s* h = new (std::nothrow) uw_handle_s();
+  if (!h) return UW_ERR_OOM;
+  if (!build_decode_tables(f->code_len, f->palette, &h->tables)) {
+    delete h;
+    return UW_ERR_FORMAT;
+  }
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return UW_ERR_CUDA;
+  }
+  cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device);
+  h->stream = static_cast<cudaStream_t>(stream);
+  h->N = f->N;
+  h->K = f->K;
+  h->chunk_syms = f->chunk_syms;
+  h->max_code_len = f->max_code_len;
+  std::memcpy(h->code_len, f->code_len, 256);
+  std::memcpy(h->palette, f->palette, 16);
+  h->n_words = f->n_words;
+  h->n_chunks = f->n_chunks;
+  h->n_esc_words = f->n_esc_words;
+  h->n_esc_groups = f->n_esc_groups;
+  h->n_esc_rows = f->n_esc_rows;
+
+  const size_t T = (size_t)f->N * (size_t)f->K;
+  struct Part { void** dst; const void* src; size_t bytes; };
+  size_t off = 0;
+  auto place = [&](size_t bytes) { size_t at = off; off = align_up(off + bytes, 256); return at; };
+  const size_t o_words = place((size_t)f->n_words * 4);
+  const size_t o_coff = place((size_t)(f->n_chunks + 1) * 4);
+  const size_t o_elut = place(kLutSize * 4);
+  const size_t o_plut = place(kLutSize * 4);
+  const size_t o_lim = place(16 * 4);
+  const size_t o_sm = place(T);
+  const size_t o_ebits = place((size_t)std::max<int64_t>(f->n_esc_words, 1) * 4);
+  const size_t o_eoff = place((size_t)(f->n_esc_groups + 1) * 4);
+  const size_t o_eexp = place((size_t)std::max<int64_t>(f->n_esc_rows, 1) * kRow);
+  const size_t o_stat = place(256);
+  const size_t o_pidx = o.prepare_direct ? place(T / 2) : 0;
+  cudaError_t e = cudaMalloc(&h->d_block, off);
+  if (e != cudaSuccess) {
+    delete h;
+    return map_cuda(e);
+  }
+  uint8_t* base = static_cast<uint8_t*>(h->d_block);
+  h->d_words = reinterpret_cast<uint32_t*>(base + o_words);
+  h->d_chunk_off = reinterpret_cast<uint32_t*>(base + o_coff);
+  h->d_exp_lut = reinterpret_cast<uint32_t*>(base + o_elut);
+  h->d_pal_lut = reinterpret_cast<uint32_t*>(base + o_plut);
+  h->d_limit = reinterpret_cast<uint32_t*>(base + o_lim);
+  h->d_sm = base + o_sm;
+  h->d_esc_bits = reinterpret_cast<uint32_t*>(base + o_ebits);
+  h->d_esc_off = reinterpret_cast<uint32_t*>(base + o_eoff);
+  h->d_esc_exp = base + o_eexp;
+  h->d_status = reinterpret_cast<uint32_t*>(base + o_stat);
+  h->d_pal_idx = o.prepare_direct ? base + o_pidx : nullptr;
+  cudaStream_t s = h->stream;
+  const Part parts[] = {
+      {(void**)&h->d_words, f->words, (size_t)f->n_words * 4},
+      {(void**)&h->d_chunk_off, f->chunk_off, (size_t)(f->n_chunks + 1) * 4},
+      {(void**)&h->d_exp_lut, h->tables.exp_lut.data(), kLutSize * 4},
+      {(void**)&h->d_pal_lut, h->tables.pal_lut.data(), kLutSize * 4},
+      {(void**)&h->d_limit, h->tables.limit, 16 * 4},
+      {(void**)&h->d_sm, f->sm, T},
+      {(void**)&h->d_esc_bits, f->esc_bits, (size_t)f->n_esc_words * 4},
+      {(void**)&h->d_esc_off, f->esc_off, (size_t)(f->n_esc_groups + 1) * 4},
+      {(void**)&h->d_esc_exp, f->esc_exp, (size_t)f->n_esc_rows * kRow},
+  };
+  for (const Part& p : parts) {
+    if (p.bytes == 0) continue;
+    e = cudaMemcpyAsync(*p.dst, p.src, p.bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) break;
+  }
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->d_status, 0, 256, s);
+  if (e == cudaSuccess && h->d_pal_idx) {
+    // load-time transcode: the resident palette form of pipeline 4
+    DecodeArgs a = decode_args(h);
+    a.lut = h->d_pal_lut;
+    e = launch_decode(kDecodePalette, a, h->d_pal_idx, 0, s);
+  }
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    free_handle(h);
+    return map_cuda(e);
+  }
+  *out = h;
+  return UW_OK;
+}
+
+uw_status uw_encode(const uint16_t* w_host, int64_t N, int64_t K, const uw_encode_opts* opts,
+                    void* stream, uw_handle_t* out) {
+  if (!out) return UW_ERR_ARG;
+  *out = nullptr;
+  uw_host_t hh = nullptr;
+  uw_status st = uw_encode_host(w_host, N, K, opts, &hh);
+  if (st != UW_OK) return st;
+  uw_format f;
+  uw_host_view(hh, &f);
+  st = uw_upload(&f, opts, stream, out);
+  if (st == UW_OK) (*out)->hist = hh->enc.hist;
+  uw_host_free(hh);
+  return st;
+}
+
+uw_status uw_free(uw_handle_t h) {
+  if (!h) return UW_ERR_ARG;
+  free_handle(h);
+  return UW_OK;
+}
+
+uw_status uw_set_stream(uw_handle_t h, void* stream) {
+  if (!h) return UW_ERR_ARG;
+  h->stream = static_cast<cudaStream_t>(stream);
+  return UW_OK;
+}
+
+uw_status uw_stats(uw_handle_t h, uw_stats_t* out) {
+  if (!h || !out) return UW_ERR_ARG;
+  uw_format f;
+  std::memset(&f, 0, sizeof(f));
+  f.N = h->N;
+  f.K = h->K;
+  std::memcpy(f.code_len, h->code_len, 256);
+  std::memcpy(f.palette, h->palette, 16);
+  f.n_chunks = h->n_chunks;
+  f.n_words = h->n_words;
+  f.n_esc_words = h->n_esc_words;
+  f.n_esc_groups = h->n_esc_groups;
+  f.n_esc_rows = h->n_esc_rows;
+  // total bits = last chunk offset (read back from the device)
+  uint32_t last = 0;
+  DeviceGuard g(h->device);
+  UW_CK(cudaMemcpy(&last, h->d_chunk_off + h->n_chunks, 4, cudaMemcpyDeviceToHost));
+  std::vector<uint32_t> coff((size_t)h->n_chunks + 1, 0);
+  coff.back() = last;
+  f.chunk_off = coff.data();
+  fill_stats(f, h->hist.empty() ? nullptr : h->hist.data(), out);
+  return UW_OK;
+}
+
+uw_status uw_workspace_bytes(uw_handle_t h, int32_t pipeline, int64_t M, size_t* bytes) {
+  if (!h || !bytes) return UW_ERR_ARG;
+  if (M < 0) return UW_ERR_SHAPE;
+  uw_gemm_config c;
+  std::memset(&c, 0, sizeof(c));
+  c.pipeline = pipeline;
+  if (pipeline == UW_PIPE_AUTO) c = choose_variant(h, M);
+  if (!valid_pipeline(c.pipeline)) return UW_ERR_ARG;
+  if (M == 0) {
+    *bytes = 0;
+    return UW_OK;
+  }
+  // enough for any variant: every token tile (16..256) and up to one CTA per SM
+  size_t worst = 0;
+  for (int tn = 16; tn <= 256; tn += 16) {
+    uw_gemm_config v = c;
+    v.tile_n = tn;
+    v.stages = 2;
+    v.gemm_ctas = h->sm_count;
+    GemmArgs a;
+    size_t need = 0, pre = 0;
+    if (plan_gemm(h, nullptr, nullptr, M, v, 1, &a, &need, &pre) == UW_OK)
+      worst = std::max(worst, need);
+  }
+  if (!worst) return UW_ERR_UNSUPPORTED;
+  *bytes = worst;
+  return UW_OK;
+}
+
+uw_status uw_set_workspace(uw_handle_t h, void* ws_dev, size_t bytes) {
+  if (!h) return UW_ERR_ARG;
+  if (ws_dev && (reinterpret_cast<uintptr_t>(ws_dev) & 255)) return UW_ERR_ARG;
+  DeviceGuard g(h->device);
+  if (h->ws_owned && h->ws) cudaFree(h->ws);
+  h->ws = ws_dev;
+  h->ws_bytes = ws_dev ? bytes : 0;
+  h->ws_owned = false;
+  return UW_OK;
+}
+
+uw_status uw_alloc_workspace(uw_handle_t h, size_t bytes) {
+  if (!h) return UW_ERR_ARG;
+  DeviceGuard g(h->device);
+  void* p = nullptr;
+  if (bytes) UW_CK(cudaMalloc(&p, bytes));
+  if (h->ws_owned && h->ws) cudaFree(h->ws);
+  h->ws = p;
+  h->ws_bytes = bytes;
+  h->ws_owned = bytes != 0;
+  return UW_OK;
+}
+
+static uw_status check_out_ptr(const void* p) {
+  if (!p) return UW_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(p) & 15) return UW_ERR_ARG;
+  return UW_OK;
+}
+
+uw_status uw_decode_full(uw_handle_t h, uint16_t* w_dev) {
+  if (!h) return UW_ERR_ARG;
+  uw_status st = check_out_ptr(w_dev);
+  if (st != UW_OK) return st;
+  DeviceGuard g(h->device);
+  return run_decode(h, kDecodeFull, w_dev, 0, h->stream);
+}
+
+uw_status uw_decode_exp(uw_handle_t h, uint8_t* e_dev) {
+  if (!h) return UW_ERR_ARG;
+  uw_status st = check_out_ptr(e_dev);
+  if (st != UW_OK) return st;
+  DeviceGuard g(h->device);
+  return run_decode(h, kDecodeExp, e_dev, 0, h->stream);
+}
+
+uw_status uw_transcode_palette(uw_handle_t h, uint8_t* idx_dev) {
+  if (!h) return UW_ERR_ARG;
+  uw_status st = check_out_ptr(idx_dev);
+  if (st != UW_OK) return st;
+  DeviceGuard g(h->device);
+  return run_decode(h, kDecodePalette, idx_dev, 0, h->stream);
+}
+
+uw_status uw_gemm_ex(uw_handle_t h, const uint16_t* X_dev, void* Y_dev, int64_t M,
+                     const uw_gemm_config* cfg, int32_t out_f32) {
+  if (!h || !cfg) return UW_ERR_ARG;
+  if (M < 0 || M > (int64_t(1) << 24)) return UW_ERR_SHAPE;
+  if (M == 0) return UW_OK;
+  if (check_out_ptr(X_dev) != UW_OK || check_out_ptr(Y_dev) != UW_OK) return UW_ERR_ARG;
+  DeviceGuard g(h->device);
+  return run_gemm(h, X_dev, Y_dev, M, *cfg, out_f32 ? 1 : 0);
+}
+
+uw_status uw_gemm(uw_handle_t h, const uint16_t* X_dev, uint16_t* Y_dev, int64_t M,
+                  uw_pipeline pipeline) {
+  uw_gemm_config c;
+  std::memset(&c, 0, sizeof(c));
+  c.pipeline = pipeline;
+  if (pipeline != UW_PIPE_AUTO && !valid_pipeline(pipeline)) return UW_ERR_ARG;
+  return uw_gemm_ex(h, X_dev, Y_dev, M, &c, 0);
+}
+
+uw_status uw_gemm_f32(uw_handle_t h, const uint16_t* X_dev, float* Y_dev, int64_t M,
+                      uw_pipeline pipeline) {
+  uw_gemm_config c;
+  std::memset(&c, 0, sizeof(c));
+  c.pipeline = pipeline;
+  if (pipeline != UW_PIPE_AUTO && !valid_pipeline(pipeline)) return UW_ERR_ARG;
+  return uw_gemm_ex(h, X_dev, Y_dev, M, &c, 1);
+}
+
+uw_status uw_trace_enable(uw_handle_t h, int32_t enable) {
+  if (!h) return UW_ERR_ARG;
+  h->trace = enable != 0;
+  return UW_OK;
+}
+
+uw_status uw_trace_read(uw_handle_t h, int32_t* kinds, float* ms, int32_t capacity,
+                        int32_t* count) {
+  if (!h || !count || capacity < 0 || (capacity > 0 && (!kinds || !ms))) return UW_ERR_ARG;
+  DeviceGuard g(h->device);
+  UW_CK(cudaStreamSynchronize(h->stream));
+  const int n = (int)h->trace_kinds.size();
+  *count = n;
+  for (int i = 0; i < n && i < capacity; ++i) {
+    kinds[i] = h->trace_kinds[i];
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, h->trace_events[2 * i], h->trace_events[2 * i + 1]) != cudaSuccess)
+      t = -1.f;
+    ms[i] = t;
+  }
+  h->trace_kinds.clear();
+  return UW_OK;
+}
+
+uw_status uw_last_device_status(uw_handle_t h) {
+  if (!h) return UW_ERR_ARG;
+  DeviceGuard g(h->device);
+  UW_CK(cudaStreamSynchronize(h->stream));
+  uint32_t st = 0;
+  UW_CK(cudaMemcpy(&st, h->d_status, 4, cudaMemcpyDeviceToHost));
+  UW_CK(cudaMemset(h->d_status, 0, 4));
+  if (st & kStatusTimeout) return UW_ERR_TIMEOUT;
+  if (st & kStatusBadChunk) return UW_ERR_DEVICE;
+  return UW_OK;
+}
+
+}  // extern "C"

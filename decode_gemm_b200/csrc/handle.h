@@ -1,0 +1,59 @@
+// Device-resident encoded matrix (the object behind uw_handle_t).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <map>
+#include <vector>
+
+#include "uw_internal.h"
+#include "uw_kernels.h"
+
+struct uw_handle_s {
+  int device = 0;
+  int sm_count = 148;
+  cudaStream_t stream = nullptr;
+
+  int64_t N = 0, K = 0;
+  int32_t chunk_syms = 1024, max_code_len = 12;
+  uint8_t code_len[256] = {0};
+  uint8_t palette[16] = {0};
+  uw::DecodeTables tables;
+  int64_t n_words = 0, n_chunks = 0, n_esc_words = 0, n_esc_groups = 0, n_esc_rows = 0;
+  std::vector<int64_t> hist;  // exponent histogram when known (for statistics)
+
+  // one device allocation holding every array below
+  void* d_block = nullptr;
+  uint32_t* d_words = nullptr;
+  uint32_t* d_chunk_off = nullptr;
+  uint32_t* d_exp_lut = nullptr;
+  uint32_t* d_pal_lut = nullptr;
+  uint32_t* d_limit = nullptr;
+  uint8_t* d_sm = nullptr;
+  uint32_t* d_esc_bits = nullptr;
+  uint32_t* d_esc_off = nullptr;
+  uint8_t* d_esc_exp = nullptr;
+  uint32_t* d_status = nullptr;
+  uint8_t* d_pal_idx = nullptr;  // resident palette indices (pipeline 4), may be null
+
+  // workspace for pipelines 1-3 and split-K partial sums
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  bool ws_owned = false;
+
+  // autotuned choices: M -> variant (nearest M at or above is used)
+  std::map<int64_t, uw_gemm_config> profile;
+
+  // kernel tracing (uw_trace_enable): event pairs around each launch
+  bool trace = false;
+  std::vector<cudaEvent_t> trace_events;  // pool, 2 per launch
+  std::vector<int32_t> trace_kinds;
+};
+
+namespace uw {
+DecodeArgs decode_args(const uw_handle_s* h);
+// Record the start event of a traced launch (no-op unless tracing); returns the
+// slot to pass to trace_end, or -1.
+int trace_begin(uw_handle_s* h, int kind);
+void trace_end(uw_handle_s* h, int slot);
+}

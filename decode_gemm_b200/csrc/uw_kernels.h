@@ -1,0 +1,83 @@
+// Kernel launch interfaces (device code lives in decode.cu and gemm.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace uw {
+
+enum DecodeMode { kDecodeExp = 0, kDecodeFull = 1, kDecodePalette = 2 };
+
+// Everything a decode/transcode launch reads, as device pointers.
+struct DecodeArgs {
+  const uint32_t* words;      // Huffman stream, n_words (a multiple of 4) words
+  const uint32_t* chunk_off;  // n_chunks + 1 bit offsets
+  const uint32_t* lut;        // 4096-entry decode table (exponent or palette flavour)
+  const uint32_t* limit;      // 16 words: first-code-length limits (see DecodeTables)
+  const uint8_t* sm;          // sign+mantissa bytes (full decode only)
+  const uint32_t* esc_bits;   // escape bitmap (palette transcode only)
+  uint32_t* status;           // device status word (bit 0: bad chunk)
+  int64_t n_words;
+  int64_t n_chunks;
+  int64_t total_syms;         // N*K
+  int32_t chunk_syms;
+  int32_t kb_per_row;         // K / 64
+  int32_t esc_nw;             // escape-bitmap words per K block: 4*ceil(N/128)
+};
+
+// Decode/transcode every chunk into `out` (layout per mode: BF16 [N*K],
+// exponent bytes [N*K], packed nibbles [N*K/2]).  ctas <= 0: one CTA per 256
+// chunks.  Returns the launch error.
+cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cudaStream_t s);
+int decode_ctas_needed(int64_t n_chunks);
+
+// Device status bits.
+constexpr uint32_t kStatusBadChunk = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+
+}  // namespace uw
+
+namespace uw {
+
+// Reconstructive / plain GEMM: Y[M, N] = X[M, K] * W^T.
+enum GemmMode { kGemmBf16 = 0, kGemmExp = 1, kGemmPalette = 2 };
+
+struct GemmArgs {
+  int mode = kGemmBf16;
+  int64_t M = 0, N = 0, K = 0;
+  const uint16_t* X = nullptr;   // [M, K] bf16
+  const uint16_t* W = nullptr;   // [N, K] bf16 (kGemmBf16)
+  const uint8_t* S = nullptr;    // [N, K] sign+mantissa (kGemmExp, kGemmPalette)
+  const uint8_t* E = nullptr;    // [N, K] exponents (kGemmExp)
+  const uint8_t* I = nullptr;    // [N, K/2] packed palette indices (kGemmPalette)
+  const uint32_t* esc_bits = nullptr;
+  const uint32_t* esc_off = nullptr;
+  const uint8_t* esc_exp = nullptr;
+  int32_t esc_nw = 0;
+  uint8_t palette[16] = {0};
+  void* Y = nullptr;             // [M, N] bf16 or f32
+  int out_f32 = 0;
+  float* partials = nullptr;     // workspace for split partial sums
+  size_t partials_bytes = 0;
+  int tile_n = 0;                // tokens per tile (0 = auto)
+  int stages = 0;                // ring depth (0 = auto)
+  int ctas = 0;                  // persistent CTAs (0 = SM count)
+  int sm_count = 148;
+  uint32_t* status = nullptr;
+};
+
+// Optional launch hooks (kernel tracing): begin(ctx, kind) returns a slot that
+// end(ctx, slot) closes; kinds follow uw_kernel_kind.
+struct LaunchHooks {
+  void* ctx = nullptr;
+  int (*begin)(void* ctx, int kind) = nullptr;
+  void (*end)(void* ctx, int slot) = nullptr;
+};
+
+// Fill in automatic tile_n / stages / ctas; returns false for unsupported shapes.
+bool gemm_resolve(GemmArgs* a);
+size_t gemm_partials_bytes(const GemmArgs& a);  // after gemm_resolve
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* hooks = nullptr);
+
+}  // namespace uw

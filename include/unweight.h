@@ -1,0 +1,263 @@
+/*
+ * unweight.h - C ABI of libunweight: lossless BF16 weight compression fused
+ * with the matmul that consumes the weights, for NVIDIA B200 (sm_100a).
+ *
+ * Method: Cloudflare, "Unweight: how we compressed an LLM 22% without
+ * sacrificing quality" (cited as *Unweight* with the section heading).
+ *
+ *   - "How model weights compress effectively": a BF16 weight is sign (1 bit),
+ *     exponent (8 bits), mantissa (7 bits).
+ *   - "Exponents are surprisingly predictable": sign and mantissa are kept
+ *     verbatim; the exponent byte is Huffman coded; the 16 most frequent
+ *     exponents form a palette; a 64-weight row holding any exponent outside
+ *     the palette is stored verbatim.
+ *   - "Four ways to use compressed weights": full decode to BF16 + plain GEMM;
+ *     exponent-only decode; runtime palette transcode; palette transcoded once
+ *     at load.  The last three feed a reconstructive matmul.
+ *   - "How the reconstructive matmul works": compressed tiles are staged in
+ *     shared memory, rebuilt to BF16 there and fed to the tensor cores; the
+ *     rebuilt weights never reach main memory.
+ *   - "Sharing the GPU between decode and compute": the decoder's ~16 KB
+ *     lookup table, the decoder/GEMM SM split, the autotuner, easy/hard layers
+ *     overlapped on side streams.
+ *
+ * Conventions (every call):
+ *   - Weights W are [N, K] row-major BF16 bit patterns (torch Linear.weight);
+ *     activations X are [M, K] row-major BF16; outputs Y are [M, N] row-major.
+ *     K must be a positive multiple of 64.
+ *   - "_dev" pointers are CUDA device pointers owned by the caller; "_host"
+ *     pointers are host memory owned by the caller.  The library never frees a
+ *     caller pointer and never keeps one after the call returns (except the
+ *     workspace registered with uw_set_workspace, see there).
+ *   - Device calls are asynchronous on the stream bound to the handle
+ *     (uw_set_stream; default: the legacy default stream).  Argument errors are
+ *     detected on the host before anything is launched.  Kernel-side errors
+ *     (corrupt stream, bounded wait expired) set a status word in the handle,
+ *     read by uw_last_device_status.  No call aborts, traps or throws.
+ *   - Thread safety: a handle may be used by one host thread at a time.
+ */
+#ifndef UNWEIGHT_H
+#define UNWEIGHT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define UW_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define UW_API __attribute__((visibility("default")))
+#else
+#define UW_API
+#endif
+
+typedef enum uw_status {
+  UW_OK = 0,
+  UW_ERR_ARG = 1,          /* null pointer, bad enum, bad option value          */
+  UW_ERR_SHAPE = 2,        /* N, K or M out of range, K not a multiple of 64    */
+  UW_ERR_FORMAT = 3,       /* encoded data fails validation                     */
+  UW_ERR_UNSUPPORTED = 4,  /* valid request this build cannot serve             */
+  UW_ERR_OOM = 5,          /* device or host allocation failed                  */
+  UW_ERR_CUDA = 6,         /* a CUDA runtime call failed                        */
+  UW_ERR_DEVICE = 7,       /* a kernel reported corrupt input                   */
+  UW_ERR_TIMEOUT = 8,      /* a kernel's bounded wait expired                   */
+  UW_ERR_WORKSPACE = 9     /* the pipeline needs a (larger) workspace           */
+} uw_status;
+
+/* Execution pipelines (*Unweight*, "Four ways to use compressed weights"). */
+typedef enum uw_pipeline {
+  UW_PIPE_AUTO = 0,            /* per-(M) choice from the loaded profile, else a default */
+  UW_PIPE_FULL = 1,            /* Huffman decode to BF16 in HBM, then plain GEMM         */
+  UW_PIPE_EXP = 2,             /* decode exponent bytes to HBM, reconstructive GEMM      */
+  UW_PIPE_PALETTE_RT = 3,      /* transcode to 4-bit palette indices, reconstructive GEMM */
+  UW_PIPE_PALETTE_DIRECT = 4   /* palette indices prepared at load, reconstructive GEMM  */
+} uw_pipeline;
+
+/* Encoder options.  uw_default_encode_opts fills the defaults. */
+typedef struct uw_encode_opts {
+  int32_t max_code_len;    /* Huffman length cap, 1..12 (default 12: a 2^12-entry
+                              4-byte decode table is 16 KB, "Sharing the GPU ...") */
+  int32_t chunk_syms;      /* symbols per independently decodable chunk; a positive
+                              multiple of 64 (default 1024)                        */
+  int32_t prepare_direct;  /* nonzero: at upload, transcode once into resident
+                              palette indices so UW_PIPE_PALETTE_DIRECT works      */
+  int32_t reserved;
+} uw_encode_opts;
+
+/*
+ * Read-only view of an encoded matrix (host pointers).  Layout of each array:
+ *   sm        [N*K]  u8  sign<<7 | mantissa, row-major
+ *   code_len  [256]  u8  Huffman code length of each exponent value (0 = absent);
+ *                        codes are canonical (RFC 1951 section 3.2.2)
+ *   words     [n_words] u32  codes of E in row-major order, MSB first: stream bit
+ *                        p is bit 31 - p%32 of words[p/32]; n_words % 4 == 0
+ *   chunk_off [n_chunks+1] u32  start bit of each chunk of chunk_syms symbols;
+ *                        chunk_off[n_chunks] = total bits
+ *   palette   [16]   u8  most frequent exponents, most frequent first
+ *   esc_bits  [(K/64) * NWp] u32, NWp = 4*ceil(N/128): bit n%32 of word
+ *                        [kb*NWp + n/32] set when the 64-weight row (n, kb) is an
+ *                        escape row (16 bytes per 128-row block; padding bits 0)
+ *   esc_off   [n_esc_groups+1] u32  groups are (n/128, kb) in row-major order;
+ *                        group g owns escape rows esc_off[g] .. esc_off[g+1]-1
+ *   esc_exp   [n_esc_rows*64] u8  verbatim exponent bytes of each escape row
+ */
+typedef struct uw_format {
+  int64_t N, K;
+  int32_t max_code_len, chunk_syms;
+  uint8_t code_len[256];
+  uint8_t palette[16];
+  int64_t n_words;       const uint32_t* words;
+  int64_t n_chunks;      const uint32_t* chunk_off;
+  const uint8_t* sm;
+  int64_t n_esc_words;   const uint32_t* esc_bits;
+  int64_t n_esc_groups;  const uint32_t* esc_off;
+  int64_t n_esc_rows;    const uint8_t* esc_exp;
+} uw_format;
+
+typedef struct uw_stats_t {
+  int64_t N, K;
+  double bits_per_exponent;   /* Huffman stream bits / (N*K)                 */
+  double entropy_bits;        /* empirical exponent entropy                  */
+  double top16_coverage;      /* fraction of weights whose E is in the palette */
+  int64_t n_rows, n_escape_rows;
+  int32_t max_len_used, n_symbols;
+  int64_t bytes_stream, bytes_offsets, bytes_sm, bytes_escape, bytes_palette_idx;
+  int64_t bytes_huffman_bundle;   /* stream + offsets + S + code lengths          */
+  int64_t bytes_palette_bundle;   /* indices + S + escape rows/bits/offsets       */
+} uw_stats_t;
+
+/* Explicit GEMM variant (what the autotuner chooses; 0 = library default). */
+typedef struct uw_gemm_config {
+  int32_t pipeline;      /* uw_pipeline, not AUTO                                  */
+  int32_t tile_n;        /* tokens per MMA tile: 16..256, multiple of 16 (0=auto)  */
+  int32_t stages;        /* shared-memory ring depth, 2..8 (0 = auto)              */
+  int32_t gemm_ctas;     /* persistent GEMM CTAs (0 = one per SM)                   */
+  int32_t decode_ctas;   /* CTAs of the preprocessing kernel (0 = auto)            */
+  int32_t reserved[3];
+} uw_gemm_config;
+
+typedef struct uw_host_s* uw_host_t;       /* host-side encoded matrix         */
+typedef struct uw_handle_s* uw_handle_t;   /* device-resident encoded matrix   */
+
+/* Human-readable name of a status code (static string, never NULL). */
+UW_API const char* uw_status_str(uw_status s);
+UW_API int uw_abi_version(void);
+UW_API void uw_default_encode_opts(uw_encode_opts* opts);
+
+/* ---- host side (no GPU needed) ------------------------------------------- */
+
+/* Compress W (host, [N, K] BF16 bits) on the host.  Steps ("Exponents are
+ * surprisingly predictable"): exponent histogram, palette, escape rows,
+ * optimal length-limited code lengths (package-merge, cap max_code_len),
+ * canonical codes, chunked bitstream with bit offsets, S stream.
+ * Errors: UW_ERR_ARG (null), UW_ERR_SHAPE (N<1, K<64, K%64), UW_ERR_UNSUPPORTED
+ * (stream >= 2^32 bits), UW_ERR_OOM.  *out is owned by the caller: uw_host_free. */
+UW_API uw_status uw_encode_host(const uint16_t* w_host, int64_t N, int64_t K,
+                         const uw_encode_opts* opts, uw_host_t* out);
+/* Fill *view with pointers into h (valid until uw_host_free(h)). */
+UW_API uw_status uw_host_view(uw_host_t h, uw_format* view);
+UW_API void uw_host_free(uw_host_t h);
+/* Structural validation of an encoded matrix: shapes, Kraft inequality, length
+ * cap, monotone chunk offsets within the stream, per-chunk bit counts between
+ * min and max code length, distinct palette, escape bitmap consistent with
+ * the group offsets.  UW_OK or UW_ERR_FORMAT / UW_ERR_SHAPE / UW_ERR_ARG. */
+UW_API uw_status uw_validate_format(const uw_format* f);
+/* Statistics of a host-side encoding (no GPU). */
+UW_API uw_status uw_host_stats(uw_host_t h, uw_stats_t* out);
+
+/* ---- device side ---------------------------------------------------------- */
+
+/* Validate f, copy it to the current CUDA device on `stream` (a cudaStream_t,
+ * may be NULL), build the decode tables, and if opts->prepare_direct run the
+ * load-time palette transcode.  The host data is not retained.  *out is
+ * owned by the caller: uw_free.  Errors: as uw_validate_format, UW_ERR_OOM,
+ * UW_ERR_CUDA. */
+UW_API uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream,
+                    uw_handle_t* out);
+/* uw_encode_host + uw_upload (the load-time entry point). */
+UW_API uw_status uw_encode(const uint16_t* w_host, int64_t N, int64_t K,
+                    const uw_encode_opts* opts, void* stream, uw_handle_t* out);
+UW_API uw_status uw_free(uw_handle_t h);
+UW_API uw_status uw_set_stream(uw_handle_t h, void* stream);
+UW_API uw_status uw_stats(uw_handle_t h, uw_stats_t* out);
+
+/* Workspace: pipelines FULL, EXP and PALETTE_RT write their preprocessed
+ * weights (2*N*K, N*K, N*K/2 bytes) and the GEMM its split-K partial sums to a
+ * device workspace.  uw_workspace_bytes gives a size that serves (pipeline, M)
+ * with any variant (token tile up to 256, up to one CTA per SM);
+ * uw_set_workspace registers caller-owned device memory (kept by pointer until
+ * replaced or the handle is freed; ptr NULL unregisters); uw_alloc_workspace
+ * makes the handle allocate and own one of `bytes` bytes.  Calls that need
+ * more workspace than registered return UW_ERR_WORKSPACE and launch nothing. */
+UW_API uw_status uw_workspace_bytes(uw_handle_t h, int32_t pipeline, int64_t M, size_t* bytes);
+UW_API uw_status uw_set_workspace(uw_handle_t h, void* ws_dev, size_t bytes);
+UW_API uw_status uw_alloc_workspace(uw_handle_t h, size_t bytes);
+
+/* Full Huffman decode ("Four ways...", pipeline 1 preprocessing): writes the
+ * N*K BF16 weights to w_dev (caller-owned, 16-byte aligned).  Bit-exact. */
+UW_API uw_status uw_decode_full(uw_handle_t h, uint16_t* w_dev);
+/* Exponent-only decode (pipeline 2 preprocessing): N*K exponent bytes to e_dev
+ * (16-byte aligned), row-major. */
+UW_API uw_status uw_decode_exp(uw_handle_t h, uint8_t* e_dev);
+/* Palette transcode (pipeline 3 preprocessing; also the load-time step of
+ * pipeline 4): N*K/2 bytes of packed 4-bit indices to idx_dev (16-byte
+ * aligned); byte j of row n holds element 2j (low nibble) and 2j+1 (high
+ * nibble); all indices of an escape row are 0. */
+UW_API uw_status uw_transcode_palette(uw_handle_t h, uint8_t* idx_dev);
+
+/* Y[M, N] = X[M, K] W^T with BF16 inputs, FP32 accumulation, BF16 output
+ * (round to nearest even).  pipeline AUTO takes the profile's choice for M.
+ * M == 0 returns UW_OK and launches nothing.  X and Y are device pointers,
+ * 16-byte aligned, row-major, not overlapping. */
+UW_API uw_status uw_gemm(uw_handle_t h, const uint16_t* X_dev, uint16_t* Y_dev, int64_t M,
+                  uw_pipeline pipeline);
+/* As uw_gemm with FP32 output (no final rounding). */
+UW_API uw_status uw_gemm_f32(uw_handle_t h, const uint16_t* X_dev, float* Y_dev, int64_t M,
+                      uw_pipeline pipeline);
+/* As uw_gemm / uw_gemm_f32 with an explicit variant; out_f32 selects the
+ * output type of Y_dev (float* when nonzero, uint16_t* BF16 otherwise). */
+UW_API uw_status uw_gemm_ex(uw_handle_t h, const uint16_t* X_dev, void* Y_dev, int64_t M,
+                     const uw_gemm_config* cfg, int32_t out_f32);
+
+/* Autotuner ("Sharing the GPU between decode and compute", last paragraphs):
+ * for every handle and every M in Ms, measure candidate variants (pipeline,
+ * token tile, ring depth, decoder/GEMM CTA split) with CUDA events on the
+ * handle's stream, by coordinate descent over the projections until no
+ * change improves the total time; store the winners in the handles and, when
+ * profile_out_json is not NULL, write them as JSON.  Needs a workspace on
+ * each handle large enough for the largest M (UW_ERR_WORKSPACE otherwise). */
+UW_API uw_status uw_autotune(uw_handle_t* hs, int32_t n_handles, const int64_t* Ms, int32_t n_M,
+                      const char* profile_out_json);
+/* Load a profile written by uw_autotune into the handles (matched by order and
+ * shape).  UW_ERR_FORMAT on a malformed file or a shape mismatch. */
+UW_API uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profile_json);
+/* The variant uw_gemm(..., UW_PIPE_AUTO) would use for M. */
+UW_API uw_status uw_get_choice(uw_handle_t h, int64_t M, uw_gemm_config* cfg);
+
+/* Kernel tracing.  While enabled, every kernel the handle launches is
+ * bracketed by two CUDA events recorded on the handle's stream (no extra
+ * synchronisation).  uw_trace_read synchronises the stream and returns, in
+ * launch order, each recorded launch's kind (uw_kernel_kind) and device time
+ * in milliseconds, then clears the record.  At most 16384 launches are kept;
+ * *count gets the number recorded, of which min(count, capacity) are copied. */
+typedef enum uw_kernel_kind {
+  UW_KERNEL_DECODE_FULL = 0, UW_KERNEL_DECODE_EXP = 1, UW_KERNEL_TRANSCODE = 2,
+  UW_KERNEL_GEMM_BF16 = 3, UW_KERNEL_GEMM_EXP = 4, UW_KERNEL_GEMM_PALETTE = 5,
+  UW_KERNEL_SPLITK_FIXUP = 6
+} uw_kernel_kind;
+UW_API uw_status uw_trace_enable(uw_handle_t h, int32_t enable);
+UW_API uw_status uw_trace_read(uw_handle_t h, int32_t* kinds, float* ms, int32_t capacity,
+                               int32_t* count);
+
+/* Synchronise the handle's stream, then return and clear the device status
+ * word: UW_OK, UW_ERR_DEVICE (a chunk decoded to the wrong bit count or hit an
+ * invalid code) or UW_ERR_TIMEOUT (a bounded wait in a kernel expired). */
+UW_API uw_status uw_last_device_status(uw_handle_t h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* UNWEIGHT_H */

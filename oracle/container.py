@@ -15,8 +15,9 @@ Everything in one encoded matrix W[N, K] (K a multiple of 64):
 * ``words``    uint32         the Huffman stream of E (see ``huffman``).
 * ``offsets``  [C+1] uint32   chunk start bits, last entry = total bits.
 * ``palette``  [16] uint8     the 16 most frequent exponents (see ``palette``).
-* ``esc_bits`` [K/64, ceil(N/32)] uint32: bit n%32 of word [kb, n//32] is set
-  when row (n, kb) is an escape row.
+* ``esc_bits`` [K/64, 4*ceil(N/128)] uint32: bit n%32 of word [kb, n//32] is
+  set when row (n, kb) is an escape row (each K block's words are padded to a
+  multiple of 4, i.e. 16 bytes per 128-row block; padding bits are 0).
 * ``esc_off``  [G+1] uint32 and ``esc_exp`` [R, 64] uint8: the verbatim exponent
   bytes of the R escape rows, grouped by (n // 128, kb) with groups in
   row-major order over (n // 128, kb) and rows ascending by n inside a group;
@@ -59,9 +60,9 @@ class Encoded:
 
 
 def escape_bitmap(esc: np.ndarray) -> np.ndarray:
-    """Pack the [N, K/64] escape flags into words [K/64, ceil(N/32)]."""
+    """Pack the [N, K/64] escape flags into words [K/64, 4*ceil(N/128)]."""
     n, kb = esc.shape
-    nw = (n + 31) // 32
+    nw = 4 * ((n + ESC_GROUP_ROWS - 1) // ESC_GROUP_ROWS)
     out = np.zeros((kb, nw), dtype=np.uint64)
     for r in range(n):
         out[:, r // 32] |= esc[r, :].astype(np.uint64) << np.uint64(r % 32)

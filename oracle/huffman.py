@@ -176,13 +176,15 @@ def _decode_tables(lengths):
 def decode_chunk(words: np.ndarray, start_bit: int, n_syms: int, lengths):
     """Bit-by-bit canonical decode of ``n_syms`` symbols starting at ``start_bit``.
 
+    ``words`` is the uint32 stream (an array, or a list of ints).
+
     The textbook procedure for a canonical code: read one bit at a time; after
     each bit, if the code read so far minus the first code of this length is
     below the number of codes of this length, it names a symbol (codes of one
     length are consecutive and ordered by symbol).  Returns (symbols, end_bit).
     """
     max_bits, count, sorted_syms = _decode_tables(lengths)
-    w = [int(x) for x in np.asarray(words, dtype=np.uint32)]
+    w = words if isinstance(words, list) else [int(x) for x in np.asarray(words, dtype=np.uint32)]
     pos = int(start_bit)
     out = np.empty(n_syms, dtype=np.uint8)
     for i in range(n_syms):
@@ -205,6 +207,7 @@ def decode_chunk(words: np.ndarray, start_bit: int, n_syms: int, lengths):
 def decode_bitstream(words, offsets, lengths, n_syms: int, chunk_syms: int) -> np.ndarray:
     """Decode every chunk and check that chunk c ends exactly at off[c+1]."""
     offsets = np.asarray(offsets, dtype=np.int64)
+    words = [int(x) for x in np.asarray(words, dtype=np.uint32)]  # one conversion per stream
     out = np.empty(n_syms, dtype=np.uint8)
     n_chunks = offsets.size - 1
     for c in range(n_chunks):

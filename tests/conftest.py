@@ -8,6 +8,19 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def build_library():
+    """Compile libunweight.so in-tree (nvcc, sm_100a) before importing the binding.
+
+    The build script is loaded by path: importing it as a submodule would run
+    the package __init__, which refuses to load without the library."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "uw_build", os.path.join(ROOT, "decode_gemm_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: long CPU test")

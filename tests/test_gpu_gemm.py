@@ -1,0 +1,212 @@
+"""GPU parity of the four pipelines' GEMM against the FP64 oracle, through the C ABI.
+
+Acceptance: |y - y_ref| <= 1e-3 * sum_k |x w| + 1e-6 per element (FP32 output),
+plus 2^-8 |y_ref| for the final rounding when the output is BF16.
+P2, P3 and P4 rebuild identical BF16 tiles, so with the same variant (token
+tile, CTA count) their outputs must be bitwise identical.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synthdata
+
+pytestmark = pytest.mark.gpu
+
+PIPES = ["full", "exp", "palette_rt", "palette_direct"]
+
+
+@pytest.fixture(scope="module")
+def uw():
+    import torch
+    assert torch.cuda.is_available()
+    from tests.conftest import build_library
+    build_library()
+    import decode_gemm_b200
+    return decode_gemm_b200
+
+
+def _upload(uw, w, chunk=1024):
+    import torch
+    h = uw.uw_encode(w, uw.default_opts(chunk_syms=chunk))
+    return h
+
+
+def _workspace(uw, h, M, pipes=PIPES, **cfg):
+    import torch
+    need = max(uw.uw_workspace_bytes(h, uw.PIPELINES[p], M) for p in pipes)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    uw.uw_set_workspace(h, ws)
+    return ws
+
+
+def _gemm(uw, h, x_bits, pipe, out_f32=True, **cfg):
+    import torch
+    M = x_bits.shape[0]
+    X = torch.from_numpy(x_bits.view(np.int16)).cuda()
+    if out_f32:
+        Y = torch.empty((M, h.N), dtype=torch.float32, device="cuda")
+    else:
+        Y = torch.empty((M, h.N), dtype=torch.bfloat16, device="cuda")
+    Y.fill_(float("nan"))  # poison
+    c = uw.gemm_config(uw.PIPELINES[pipe], **cfg)
+    uw.uw_gemm_ex(h, X, Y, M, c, out_f32)
+    torch.cuda.synchronize()
+    assert uw.uw_last_device_status(h) == uw.UW_OK
+    if out_f32:
+        return Y.cpu().numpy().astype(np.float64)
+    return Y.float().cpu().numpy().astype(np.float64)
+
+
+def _check(y, x, w, bf16_out=False):
+    ref = oracle.gemm_fp64(x, w)
+    bound = oracle.abs_product_sum(x, w)
+    ok, worst = oracle.within_tolerance(y, ref, bound, bf16_output=bf16_out)
+    assert ok, f"worst err/tol = {worst}"
+    return worst
+
+
+SHAPES = [
+    # (M, N, K, weight maker)
+    (8, 1024, 1024, "normal"),      # the 1024x1024 single-matrix case
+    (1, 256, 512, "normal"),
+    (17, 200, 192, "student_t"),    # ragged M, ragged N (not a multiple of 128), tiny K
+    (64, 384, 640, "student_t"),
+    (130, 256, 256, "normal"),      # M spans two token tiles
+    (300, 128, 128, "special_finite"),
+]
+
+
+def _weights(kind, n, k, seed):
+    if kind == "normal":
+        return synthdata.normal(n, k, 0.02, seed)
+    if kind == "student_t":
+        return synthdata.student_t(n, k, 3.0, 0.015, seed)
+    # finite corner cases: +-0 and subnormals, no Inf/NaN (they poison every sum)
+    w = synthdata.normal(n, k, 0.02, seed)
+    rng = np.random.default_rng(seed)
+    pos = rng.choice(w.size, size=64, replace=False)
+    w.reshape(-1)[pos] = np.resize(np.array([0x0000, 0x8000, 0x0001, 0x807F, 0x0080], np.uint16),
+                                   64)
+    return w
+
+
+@pytest.mark.parametrize("M,N,K,kind", SHAPES)
+@pytest.mark.parametrize("pipe", PIPES)
+def test_gemm_matches_fp64(uw, M, N, K, kind, pipe):
+    w = _weights(kind, N, K, seed=60 + M)
+    x = synthdata.activations(M, K, seed=61 + N)
+    h = _upload(uw, w, chunk=128)
+    ws = _workspace(uw, h, M)
+    _check(_gemm(uw, h, x, pipe), x, w)
+    _check(_gemm(uw, h, x, pipe, out_f32=False), x, w, bf16_out=True)
+    h.free()
+
+
+def test_mat1024_public_calls(uw):
+    """uw_gemm / uw_gemm_f32 with every pipeline on the 1024x1024, M=8 case."""
+    import torch
+    w = synthdata.workload("mat1024")
+    x = synthdata.activation_for("mat1024", 8)
+    h = _upload(uw, w)
+    ws = _workspace(uw, h, 8)
+    X = torch.from_numpy(x.view(np.int16)).cuda()
+    for p in PIPES:
+        Y = torch.empty((8, 1024), dtype=torch.float32, device="cuda")
+        uw.uw_gemm_f32(h, X, Y, 8, uw.PIPELINES[p])
+        torch.cuda.synchronize()
+        _check(Y.cpu().numpy().astype(np.float64), x, w)
+        Yb = torch.empty((8, 1024), dtype=torch.bfloat16, device="cuda")
+        uw.uw_gemm(h, X, Yb, 8, uw.PIPELINES[p])
+        torch.cuda.synchronize()
+        _check(Yb.float().cpu().numpy().astype(np.float64), x, w, bf16_out=True)
+    assert uw.uw_last_device_status(h) == uw.UW_OK
+    h.free()
+
+
+@pytest.mark.parametrize("tile_n,ctas", [(16, 0), (32, 7), (64, 148), (128, 33)])
+def test_reconstructive_pipelines_bitwise_identical(uw, tile_n, ctas):
+    w = synthdata.student_t(512, 1024, 3.0, 0.015, seed=70)
+    x = synthdata.activations(40, 1024, seed=71)
+    h = _upload(uw, w, chunk=256)
+    ws = _workspace(uw, h, 40, tile_n=tile_n)
+    outs = [_gemm(uw, h, x, p, tile_n=tile_n, gemm_ctas=ctas) for p in PIPES[1:]]
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    _check(outs[0], x, w)
+    h.free()
+
+
+def test_escape_overflow_path(uw):
+    """More than the 32 escape rows a stage stages: rows past the cap come from HBM."""
+    w = synthdata.exponent_pattern(256, 512, range(90, 140), seed=72)  # ~every row escapes
+    x = synthdata.activations(24, 512, seed=73)
+    h = _upload(uw, w, chunk=64)
+    st = h.stats()
+    assert st["n_escape_rows"] > 0.9 * st["n_rows"]
+    ws = _workspace(uw, h, 24)
+    for p in ("palette_rt", "palette_direct"):
+        _check(_gemm(uw, h, x, p), x, w)
+    h.free()
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_gate_proj_full_size(uw, M):
+    w = synthdata.workload("gate_14336x4096")
+    x = synthdata.activation_for("gate_14336x4096", M)
+    h = _upload(uw, w)
+    ws = _workspace(uw, h, M)
+    ref = oracle.gemm_fp64(x, w)
+    bound = oracle.abs_product_sum(x, w)
+    outs = {}
+    for p in PIPES:
+        y = _gemm(uw, h, x, p)
+        ok, worst = oracle.within_tolerance(y, ref, bound)
+        assert ok, (p, worst)
+        outs[p] = y
+    assert np.array_equal(outs["exp"], outs["palette_rt"])
+    assert np.array_equal(outs["exp"], outs["palette_direct"])
+    h.free()
+
+
+@pytest.mark.parametrize("M", [256, 1024])
+def test_down_proj_full_size_sampled(uw, M):
+    w = synthdata.workload("down_4096x14336")
+    x = synthdata.activation_for("down_4096x14336", M)
+    h = _upload(uw, w)
+    ws = _workspace(uw, h, M)
+    rng = np.random.default_rng(M)
+    rows = rng.choice(M, size=min(M, 24), replace=False)
+    ref = oracle.gemm_fp64(x[rows], w)
+    bound = oracle.abs_product_sum(x[rows], w)
+    for p in PIPES:
+        y = _gemm(uw, h, x, p)[rows]
+        ok, worst = oracle.within_tolerance(y, ref, bound)
+        assert ok, (p, worst)
+    h.free()
+
+
+def test_gemm_argument_errors(uw):
+    import ctypes as C
+    import torch
+    w = synthdata.normal(128, 256, 0.02, seed=80)
+    h = uw.uw_encode(w, uw.default_opts(prepare_direct=0))
+    X = torch.zeros((4, 256), dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")
+    # M == 0: nothing to do
+    assert uw.lib.uw_gemm(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 0, 3) == uw.UW_OK
+    # pipelines 1-3 need a workspace; none registered
+    for p in (1, 2, 3):
+        assert uw.lib.uw_gemm(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 4, p) \
+            == uw.UW_ERR_WORKSPACE
+    # pipeline 4 needs the load-time transcode, which this handle skipped
+    assert uw.lib.uw_gemm(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 4, 4) \
+        == uw.UW_ERR_UNSUPPORTED
+    assert uw.lib.uw_gemm(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 4, 9) \
+        == uw.UW_ERR_ARG
+    assert uw.lib.uw_gemm(h.ptr, None, C.c_void_p(Y.data_ptr()), 4, 3) == uw.UW_ERR_ARG
+    assert uw.lib.uw_gemm(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), -1, 3) \
+        == uw.UW_ERR_SHAPE
+    bad = uw.gemm_config(3, tile_n=24)
+    assert uw.lib.uw_gemm_ex(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 4,
+                             C.byref(bad), 0) == uw.UW_ERR_ARG
+    h.free()
