@@ -22,8 +22,8 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
           "-I", INCLUDE, "-I", CSRC]
-CU_FLAGS = ARCH + ["-lineinfo", "--expt-relaxed-constexpr", "-Xptxas", "-v"] + COMMON
-CPP_FLAGS = COMMON
+CU_FLAGS = ARCH + ["-lineinfo", "--expt-relaxed-constexpr", "-Xptxas", "-v", "-Wno-deprecated-gpu-targets"] + COMMON
+CPP_FLAGS = COMMON + ["-Wno-deprecated-gpu-targets"]
 
 SOURCES = ["encode.cpp", "api.cu", "decode.cu", "gemm.cu", "autotune.cu"]
 HEADERS = ["uw_internal.h", "uw_kernels.h", "handle.h", "gemm_sm100.cuh"]

@@ -89,8 +89,9 @@ DecodeArgs decode_args(const uw_handle_s* h) {
   DecodeArgs a;
   a.words = h->d_words;
   a.chunk_off = h->d_chunk_off;
-  a.lut = h->d_exp_lut;
-  a.limit = h->d_limit;
+  a.lut = h->d_lut;
+  a.canon = h->d_canon;
+  std::memcpy(a.palette, h->palette, 16);
   a.sm = h->d_sm;
   a.esc_bits = h->d_esc_bits;
   a.status = h->d_status;
@@ -143,7 +144,6 @@ static void hook_end(void* ctx, int slot) { trace_end(static_cast<uw_handle_s*>(
 
 uw_status run_decode(uw_handle_s* h, int mode, void* out, int ctas, cudaStream_t s) {
   DecodeArgs a = decode_args(h);
-  a.lut = mode == kDecodePalette ? h->d_pal_lut : h->d_exp_lut;
   // kinds: 0 full, 1 exponent, 2 transcode
   const int kind = mode == kDecodeFull ? 0 : (mode == kDecodeExp ? 1 : 2);
   const int slot = trace_begin(h, kind);
@@ -265,9 +265,8 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   auto place = [&](size_t bytes) { size_t at = off; off = align_up(off + bytes, 256); return at; };
   const size_t o_words = place((size_t)f->n_words * 4);
   const size_t o_coff = place((size_t)(f->n_chunks + 1) * 4);
-  const size_t o_elut = place(kLutSize * 4);
-  const size_t o_plut = place(kLutSize * 4);
-  const size_t o_lim = place(16 * 4);
+  const size_t o_lut = place(kLutSize * 4);
+  const size_t o_canon = place(kCanonWords * 4);
   const size_t o_sm = place(T);
   const size_t o_ebits = place((size_t)std::max<int64_t>(f->n_esc_words, 1) * 4);
   const size_t o_eoff = place((size_t)(f->n_esc_groups + 1) * 4);
@@ -282,9 +281,8 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   uint8_t* base = static_cast<uint8_t*>(h->d_block);
   h->d_words = reinterpret_cast<uint32_t*>(base + o_words);
   h->d_chunk_off = reinterpret_cast<uint32_t*>(base + o_coff);
-  h->d_exp_lut = reinterpret_cast<uint32_t*>(base + o_elut);
-  h->d_pal_lut = reinterpret_cast<uint32_t*>(base + o_plut);
-  h->d_limit = reinterpret_cast<uint32_t*>(base + o_lim);
+  h->d_lut = reinterpret_cast<uint32_t*>(base + o_lut);
+  h->d_canon = reinterpret_cast<uint32_t*>(base + o_canon);
   h->d_sm = base + o_sm;
   h->d_esc_bits = reinterpret_cast<uint32_t*>(base + o_ebits);
   h->d_esc_off = reinterpret_cast<uint32_t*>(base + o_eoff);
@@ -295,9 +293,8 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   const Part parts[] = {
       {(void**)&h->d_words, f->words, (size_t)f->n_words * 4},
       {(void**)&h->d_chunk_off, f->chunk_off, (size_t)(f->n_chunks + 1) * 4},
-      {(void**)&h->d_exp_lut, h->tables.exp_lut.data(), kLutSize * 4},
-      {(void**)&h->d_pal_lut, h->tables.pal_lut.data(), kLutSize * 4},
-      {(void**)&h->d_limit, h->tables.limit, 16 * 4},
+      {(void**)&h->d_lut, h->tables.lut.data(), kLutSize * 4},
+      {(void**)&h->d_canon, h->tables.canon, kCanonWords * 4},
       {(void**)&h->d_sm, f->sm, T},
       {(void**)&h->d_esc_bits, f->esc_bits, (size_t)f->n_esc_words * 4},
       {(void**)&h->d_esc_off, f->esc_off, (size_t)(f->n_esc_groups + 1) * 4},
@@ -312,7 +309,6 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   if (e == cudaSuccess && h->d_pal_idx) {
     // load-time transcode: the resident palette form of pipeline 4
     DecodeArgs a = decode_args(h);
-    a.lut = h->d_pal_lut;
     e = launch_decode(kDecodePalette, a, h->d_pal_idx, 0, s);
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -132,41 +132,51 @@ bool build_decode_tables(const uint8_t code_len[256], const uint8_t palette[16],
       first_len[v] = (uint8_t)l;
     }
   }
-  uint8_t rank[256] = {0};
-  for (int i = 15; i >= 0; --i) rank[palette[i]] = (uint8_t)i;
-  out->exp_lut.assign(kLutSize, 0);
-  out->pal_lut.assign(kLutSize, 0);
+  int rank[256];
+  for (int v = 0; v < 256; ++v) rank[v] = -1;
+  for (int i = 0; i < 16; ++i) rank[palette[i]] = i;
+  out->lut.assign(kLutSize, 0);
   for (int v = 0; v < kLutSize; ++v) {
-    for (int table = 0; table < 2; ++table) {
-      const int cap = table == 0 ? kExpCap : kPalCap;
-      uint32_t vals = 0, cnt = 0, pos = 0;
-      while ((int)cnt < cap && pos < (uint32_t)kLutBits) {
-        const uint32_t w = ((uint32_t)v << pos) & (kLutSize - 1);
-        const int s = first_sym[w];
-        const int l = first_len[w];
-        if (s < 0 || pos + l > (uint32_t)kLutBits) break;
-        if (table == 0)
-          vals |= (uint32_t)s << (8 * cnt);
-        else
-          vals |= (uint32_t)rank[s] << (4 * cnt);
-        cnt++;
-        pos += l;
-      }
-      const uint32_t e = vals | (cnt << 24) | (cnt ? (pos << 28) : 0u);
-      (table == 0 ? out->exp_lut : out->pal_lut)[v] = e;
+    const int s0 = first_sym[v];
+    if (s0 < 0) continue;  // no code starts this window: entry 0 (invalid)
+    if (rank[s0] < 0) {    // an exponent outside the palette: one raw symbol
+      out->lut[v] = (uint32_t)s0 | kLutRaw | ((uint32_t)first_len[v] << 28);
+      continue;
     }
+    uint32_t vals = 0, cnt = 0, pos = 0;
+    while ((int)cnt < kPalCap && pos < (uint32_t)kLutBits) {
+      const uint32_t w = ((uint32_t)v << pos) & (kLutSize - 1);
+      const int s = first_sym[w];
+      const int l = first_len[w];
+      if (s < 0 || rank[s] < 0 || pos + l > (uint32_t)kLutBits) break;
+      vals |= (uint32_t)rank[s] << (4 * cnt);
+      cnt++;
+      pos += l;
+    }
+    out->lut[v] = vals | (cnt << 24) | (pos << 28);
   }
-  // limit[l]: windows below it start with a code of length <= l
+  // canonical tables
   int count[kLutBits + 2] = {0};
   for (int s = 0; s < 256; ++s)
     if (code_len[s]) count[code_len[s]]++;
-  uint32_t first = 0;
-  for (int l = 0; l < 16; ++l) out->limit[l] = 0;
+  uint32_t* lim = out->canon + kCanonLimit;
+  uint32_t* fst = out->canon + kCanonFirst;
+  uint32_t* ofs = out->canon + kCanonOffset;
+  uint8_t* syms = reinterpret_cast<uint8_t*>(out->canon + kCanonSymbols);
+  for (int i = 0; i < kCanonWords; ++i) out->canon[i] = 0;
+  uint32_t first = 0, index = 0;
   for (int l = 1; l <= kLutBits; ++l) {
     first = (first + (uint32_t)count[l - 1]) << 1;
-    out->limit[l] = (first + (uint32_t)count[l]) << (kLutBits - l);
+    fst[l] = first;
+    ofs[l] = index;
+    index += (uint32_t)count[l];
+    lim[l] = (first + (uint32_t)count[l]) << (kLutBits - l);
   }
-  for (int l = kLutBits + 1; l < 16; ++l) out->limit[l] = kLutSize;
+  for (int l = kLutBits + 1; l < 16; ++l) lim[l] = kLutSize;
+  int k = 0;
+  for (int l = 1; l <= kLutBits; ++l)
+    for (int s = 0; s < 256; ++s)
+      if (code_len[s] == l) syms[k++] = (uint8_t)s;
   return true;
 }
 

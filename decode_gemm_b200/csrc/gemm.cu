@@ -50,11 +50,15 @@ constexpr int kBM = 128;           // W rows per tile (MMA M)
 constexpr int kBK = 64;            // K per stage: one 128-byte swizzle row of BF16
 constexpr int kWTileBytes = kBM * kBK * 2;
 constexpr int kEscCap = 32;        // escape rows staged per stage (more: read from global)
-constexpr int kWSlots = 2;         // rebuilt-W ring depth
+constexpr int kMaxWSlots = 8;      // rebuilt-W ring depth (runtime, <= this)
 constexpr int kNumEpiWarps = 4;
-constexpr int kNumRebuildWarps = 8;
-constexpr int kEpiWarp0 = 2;
+constexpr int kNumRebuildWarps = 8;  // two groups of 4, alternating stages
+constexpr int kGroupWarps = kNumRebuildWarps / 2;
+constexpr int kMmaWarp0 = 1;         // MMA issuers: warps 1 and 2
+constexpr int kNumMmaWarps = 2;
+constexpr int kEpiWarp0 = kMmaWarp0 + kNumMmaWarps;  // warps 3..6 (quadrants 3,0,1,2)
 constexpr int kRebuildWarp0 = kEpiWarp0 + kNumEpiWarps;
+constexpr uint32_t kEpiSleepNs = 200;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
 
 __host__ __device__ constexpr int threads_for(int mode) {
@@ -73,7 +77,7 @@ struct GemmParams {
   uint32_t* status;
   int64_t M, N, K;
   int64_t units;      // output tiles * K blocks
-  int32_t tile_n, stages, NT, MT, KB, esc_nwp, out_f32, tmem_cols;
+  int32_t tile_n, stages, wslots, n_mma, NT, MT, KB, esc_nwp, out_f32, tmem_cols;
   uint32_t palette[4];
   uint32_t stage_bytes, x_bytes;
   uint64_t wait_ns;
@@ -116,6 +120,8 @@ __device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t units, int64_t 
 
 __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 
+
+
 __device__ __forceinline__ void set_abort(volatile int* abort, uint32_t* status) {
   if (!*abort) {
     *abort = 1;
@@ -131,14 +137,16 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
                                              ~uintptr_t(1023));
   const StageLayout L = stage_layout(MODE, p.tile_n);
   const int S = p.stages;
+  const int WS = MODE == kGemmBf16 ? 0 : p.wslots;
+  const int NM = p.n_mma;  // MMA-issuing warps (K blocks split by parity)
   uint8_t* ring = smem;
   uint8_t* wring = ring + (size_t)S * L.bytes;  // rebuilt W tiles (reconstructive modes)
-  uint8_t* tail = wring + (MODE == kGemmBf16 ? 0 : kWSlots * kWTileBytes);
+  uint8_t* tail = wring + (size_t)WS * kWTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   // barrier indices
-  const int b_full = 0, b_empty = S, b_wfull = 2 * S, b_wfree = 2 * S + kWSlots,
-            b_tfull = 2 * S + 2 * kWSlots, b_tempty = b_tfull + 2, b_drain = b_tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + b_drain + 1);
+  const int b_full = 0, b_empty = S, b_wfull = 2 * S, b_wfree = 2 * S + WS,
+            b_tfull = 2 * S + 2 * WS, b_tempty = b_tfull + 2, b_drain = b_tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + b_drain + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -148,17 +156,17 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(bar(b_full + s), 1);
-      mbar_init(bar(b_empty + s), 1 + (MODE == kGemmBf16 ? 0 : kNumRebuildWarps));
+      mbar_init(bar(b_empty + s), 1 + (MODE == kGemmBf16 ? 0 : kGroupWarps));
     }
-    for (int w = 0; w < kWSlots; ++w) {
-      mbar_init(bar(b_wfull + w), kNumRebuildWarps);
+    for (int w = 0; w < WS; ++w) {
+      mbar_init(bar(b_wfull + w), kGroupWarps);
       mbar_init(bar(b_wfree + w), 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(bar(b_tfull + a), 1);
+      mbar_init(bar(b_tfull + a), (uint32_t)NM);
       mbar_init(bar(b_tempty + a), kNumEpiWarps);
+      mbar_init(bar(b_drain + a), 1);
     }
-    mbar_init(bar(b_drain), 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -167,7 +175,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     prefetch_tensormap(&p.tm_w0);
     if (MODE != kGemmBf16) prefetch_tensormap(&p.tm_w1);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp0) {
     tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
     tmem_relinquish();
   }
@@ -263,72 +271,83 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         mbar_wait_bounded(bar(b_full + s), ph, &no_abort, p.wait_ns);
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer --
-    const uint32_t idesc = idesc_bf16(kBM, p.tile_n);
-    int stage = 0, wslot = 0;
-    uint32_t phase = 0, wphase = 0;
-    int seg = 0;
-    bool ok = true;
-    for (int64_t u = u0; u < u1 && ok; ++seg) {
-      const int64_t t = u / KB;
-      const int kb0 = (int)(u - t * KB);
-      const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
-      const int acc = seg & 1;
-      const uint32_t acc_phase = (uint32_t)(seg >> 1) & 1u;
-      if (lane == 0 &&
-          !mbar_wait_bounded(bar(b_tempty + acc), acc_phase ^ 1u, abort, p.wait_ns)) {
-        set_abort(abort, p.status);
-        ok = false;
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.tile_n);
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (lane == 0) {
-          bool got = mbar_wait_bounded(bar(b_full + stage), phase, abort, p.wait_ns);
-          if (got && MODE != kGemmBf16)
-            got = mbar_wait_bounded(bar(b_wfull + wslot), wphase, abort, p.wait_ns);
-          if (!got) {
-            set_abort(abort, p.status);
-            ok = false;
-          } else {
-            tc_fence_after();
-            uint8_t* st = ring + (size_t)stage * L.bytes;
-            const uint32_t a_addr =
-                MODE == kGemmBf16 ? smem_u32(st + L.w0) : smem_u32(wring + wslot * kWTileBytes);
-            const uint64_t a_desc = smem_desc_sw128(a_addr);
-            const uint64_t b_desc = smem_desc_sw128(smem_u32(st + L.x));
-#pragma unroll
-            for (int k = 0; k < kBK / 16; ++k)
-              mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
-                       (kb > kb0 || k > 0) ? 1u : 0u);
-            mma_commit(bar(b_empty + stage));
-            if (MODE != kGemmBf16) mma_commit(bar(b_wfree + wslot));
-            if (kb == kb1 - 1) mma_commit(bar(b_tfull + acc));
-          }
+  } else if (warp < kMmaWarp0 + kNumMmaWarps) {
+    // ---------------------------------------------------------- MMA issuers --
+    // Warp kMmaWarp0 + par takes the K blocks with kb % 2 == par (all of them
+    // when NM == 1) and accumulates into its own TMEM columns.
+    const int par = warp - kMmaWarp0;
+    if (par < NM) {
+      const uint32_t idesc = idesc_bf16(kBM, p.tile_n);
+      // ring positions of the current unit, advanced for every unit of the CTA
+      int stage = 0, wslot = 0;
+      uint32_t phase = 0, wphase = 0;
+      int seg = 0;
+      bool ok = true;
+      for (int64_t u = u0; u < u1 && ok; ++seg) {
+        const int64_t t = u / KB;
+        const int kb0 = (int)(u - t * KB);
+        const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
+        const int acc = seg & 1;
+        const uint32_t acc_phase = (uint32_t)(seg >> 1) & 1u;
+        if (lane == 0 &&
+            !mbar_wait_bounded(bar(b_tempty + acc), acc_phase ^ 1u, abort, p.wait_ns)) {
+          set_abort(abort, p.status);
+          ok = false;
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)((acc * NM + par) * p.tile_n);
+        bool first = true;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const bool mine = NM == 1 || (kb & 1) == par;
+          if (mine && lane == 0) {
+            bool got = mbar_wait_bounded(bar(b_full + stage), phase, abort, p.wait_ns);
+            if (got && MODE != kGemmBf16)
+              got = mbar_wait_bounded(bar(b_wfull + wslot), wphase, abort, p.wait_ns);
+            if (!got) {
+              set_abort(abort, p.status);
+              ok = false;
+            } else {
+              tc_fence_after();
+              uint8_t* st = ring + (size_t)stage * L.bytes;
+              const uint32_t a_addr = MODE == kGemmBf16
+                                          ? smem_u32(st + L.w0)
+                                          : smem_u32(wring + (size_t)wslot * kWTileBytes);
+              const uint64_t a_desc = smem_desc_sw128(a_addr);
+              const uint64_t b_desc = smem_desc_sw128(smem_u32(st + L.x));
+#pragma unroll
+              for (int k = 0; k < kBK / 16; ++k)
+                mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
+                         (!first || k > 0) ? 1u : 0u);
+              mma_commit(bar(b_empty + stage));
+              if (MODE != kGemmBf16) mma_commit(bar(b_wfree + wslot));
+            }
+          }
+          if (mine) first = false;
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          if (WS && ++wslot == WS) {
+            wslot = 0;
+            wphase ^= 1u;
+          }
         }
-        if (MODE != kGemmBf16 && ++wslot == kWSlots) {
-          wslot = 0;
-          wphase ^= 1u;
-        }
+        // the segment's accumulator is complete once this warp's MMAs finish
+        if (ok && lane == 0) mma_commit(bar(b_tfull + acc));
+        u += kb1 - kb0;
       }
-      u += kb1 - kb0;
+      // every issued MMA completes before TMEM is released
+      if (lane == 0) {
+        mma_commit(bar(b_drain + par));
+        volatile int no_abort = 0;
+        mbar_wait_bounded(bar(b_drain + par), 0, &no_abort, p.wait_ns);
+      }
+      __syncwarp();
     }
-    // every issued MMA completes before TMEM is released
-    if (lane == 0) {
-      mma_commit(bar(b_drain));
-      volatile int no_abort = 0;
-      mbar_wait_bounded(bar(b_drain), 0, &no_abort, p.wait_ns);
-    }
-    __syncwarp();
   } else if (warp < kRebuildWarp0) {
     // ------------------------------------------------------------ epilogue --
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
@@ -342,8 +361,10 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int slot = (u == u0) ? 0 : 1;
       const int acc = seg & 1;
       const uint32_t acc_phase = (uint32_t)(seg >> 1) & 1u;
-      // every lane observes the accumulator barrier before reading TMEM
-      const bool got = mbar_wait_bounded(bar(b_tfull + acc), acc_phase, abort, p.wait_ns);
+      // every lane observes the accumulator barrier before reading TMEM; the
+      // wait is long (a whole segment), so it sleeps between polls
+      const bool got =
+          mbar_wait_bounded(bar(b_tfull + acc), acc_phase, abort, p.wait_ns, kEpiSleepNs);
       if (!got) set_abort(abort, p.status);
       if (__any_sync(0xffffffffu, !got)) break;
       tc_fence_after();
@@ -351,16 +372,23 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int64_t n = nt * kBM + row;
       const int64_t m0 = mt * p.tile_n;
       const int cols = (int)imin64(p.tile_n, p.M - m0);
-      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * p.tile_n);
+      // which parity accumulators received MMAs in this segment
+      const bool has0 = NM == 1 || (kb1 - kb0 >= 2) || ((kb0 & 1) == 0);
+      const bool has1 = NM == 2 && ((kb1 - kb0 >= 2) || ((kb0 & 1) == 1));
+      const uint32_t lanebase = (uint32_t)(quad * 32) << 16;
+      const uint32_t t0 = tmem_base + lanebase + (uint32_t)((acc * NM + 0) * p.tile_n);
+      const uint32_t t1 = tmem_base + lanebase + (uint32_t)((acc * NM + 1) * p.tile_n);
       float* part = p.partials + ((int64_t)blockIdx.x * 2 + slot) * (int64_t)p.tile_n * kBM;
       for (int c = 0; c < cols; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(taddr + (uint32_t)c, r);
+        uint32_t r0[16], r1[16];
+        if (has0) tmem_ld16(t0 + (uint32_t)c, r0);
+        if (has1) tmem_ld16(t1 + (uint32_t)c, r1);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           if (c + j < cols) {
-            const float v = __uint_as_float(r[j]);
+            float v = has0 ? __uint_as_float(r0[j]) : 0.f;
+            if (has1) v += __uint_as_float(r1[j]);
             if (full) {
               if (n < p.N) {
                 const int64_t o = (m0 + c + j) * p.N + n;
@@ -380,72 +408,99 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       if (lane == 0) mbar_arrive(bar(b_tempty + acc));
       u += kb1 - kb0;
     }
-  } else {
+  } else if constexpr (MODE != kGemmBf16) {
     // ------------------------------------------------------------- rebuild --
+    // Two groups of 4 warps take alternate stages (unit q of this CTA goes to
+    // group q % 2), so two tiles are rebuilt while the tensor core consumes.
     const int rt = threadIdx.x - kRebuildWarp0 * 32;  // 0..255
+    const int grp = rt >> 7;                           // 0 or 1
+    const int gt = rt & 127;                           // thread within the group
+    bool ok = true;
+    int q = 0;  // index of the unit among this CTA's units
+    // ring positions of unit q, advanced for every unit of the CTA
     int stage = 0, wslot = 0;
     uint32_t phase = 0, wphase = 0;
-    bool ok = true;
     for (int64_t u = u0; u < u1 && ok;) {
       const int64_t t = u / KB;
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
       const int64_t nt = t / p.MT;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb, ++q) {
+        const int cur_stage = stage, cur_wslot = wslot;
+        const uint32_t cur_phase = phase, cur_wphase = wphase;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++wslot == WS) {
+          wslot = 0;
+          wphase ^= 1u;
+        }
+        if ((q & 1) != grp) continue;
         // every thread observes the stage's TMA completion before reading it
-        const bool got = mbar_wait_bounded(bar(b_full + stage), phase, abort, p.wait_ns) &&
-                         mbar_wait_bounded(bar(b_wfree + wslot), wphase ^ 1u, abort, p.wait_ns);
+        const bool got = mbar_wait_bounded(bar(b_full + cur_stage), cur_phase, abort, p.wait_ns) &&
+                         mbar_wait_bounded(bar(b_wfree + cur_wslot), cur_wphase ^ 1u, abort, p.wait_ns);
         if (!got) set_abort(abort, p.status);
         ok = !__any_sync(0xffffffffu, !got);
         if (!ok) break;
-        const uint8_t* st = ring + (size_t)stage * L.bytes;
-        uint8_t* wt = wring + wslot * kWTileBytes;
-        const uint32_t* ebits = reinterpret_cast<const uint32_t*>(st + L.ebits);
+        const uint8_t* st = ring + (size_t)cur_stage * L.bytes;
+        uint8_t* wt = wring + (size_t)cur_wslot * kWTileBytes;
+        // all inputs first (the stores below may alias nothing they read, but
+        // the compiler cannot know that), then rebuild and store
+        uint2 s8[8];
+        uint2 e8[8];
+        uint32_t v4[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int q = rt + 256 * i;
-          const int r = q >> 3, c = q & 7;
-          const uint2 s8 = *reinterpret_cast<const uint2*>(st + L.w0 + r * 64 + c * 8);
-          uint2 e8;
-          if (MODE == kGemmExp) {
-            e8 = *reinterpret_cast<const uint2*>(st + L.w1 + r * 64 + c * 8);
-          } else {
-            const uint32_t word = ebits[r >> 5];
+        for (int i = 0; i < 8; ++i) {
+          const int c8 = gt + 128 * i;
+          const int r = c8 >> 3, c = c8 & 7;
+          s8[i] = *reinterpret_cast<const uint2*>(st + L.w0 + r * 64 + c * 8);
+          if (MODE == kGemmExp)
+            e8[i] = *reinterpret_cast<const uint2*>(st + L.w1 + r * 64 + c * 8);
+          else
+            v4[i] = *reinterpret_cast<const uint32_t*>(st + L.w1 + r * 32 + c * 4);
+        }
+        uint32_t eb[4] = {0u, 0u, 0u, 0u};
+        if (MODE == kGemmPalette) {
+          const uint4 w4 = *reinterpret_cast<const uint4*>(st + L.ebits);
+          eb[0] = w4.x;
+          eb[1] = w4.y;
+          eb[2] = w4.z;
+          eb[3] = w4.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c8 = gt + 128 * i;
+          const int r = c8 >> 3, c = c8 & 7;
+          if (MODE == kGemmPalette) {
+            e8[i].x = palette4(v4[i] & 0xFFFFu, p.palette[0], p.palette[1], p.palette[2],
+                               p.palette[3]);
+            e8[i].y = palette4(v4[i] >> 16, p.palette[0], p.palette[1], p.palette[2],
+                               p.palette[3]);
+            // row r = 32*(i/2) + ... : its escape bit, decided once for the row
+            const uint32_t word = eb[r >> 5];
             if ((word >> (r & 31)) & 1u) {
-              // escape row: verbatim exponents, decided once for the row
               uint32_t slot = (uint32_t)__popc(word & ((1u << (r & 31)) - 1u));
-              for (int w = 0; w < (r >> 5); ++w) slot += (uint32_t)__popc(ebits[w]);
+              for (int w = 0; w < (r >> 5); ++w) slot += (uint32_t)__popc(eb[w]);
               if (slot < (uint32_t)kEscCap) {
-                e8 = *reinterpret_cast<const uint2*>(st + L.erows + slot * 64 + c * 8);
+                e8[i] = *reinterpret_cast<const uint2*>(st + L.erows + slot * 64 + c * 8);
               } else {
                 const uint32_t first = __ldg(p.esc_off + nt * KB + kb);
-                e8 = __ldg(reinterpret_cast<const uint2*>(p.esc_exp + (int64_t)(first + slot) * 64 +
-                                                          c * 8));
+                e8[i] = __ldg(reinterpret_cast<const uint2*>(p.esc_exp +
+                                                             (int64_t)(first + slot) * 64 + c * 8));
               }
-            } else {
-              const uint32_t v = *reinterpret_cast<const uint32_t*>(st + L.w1 + r * 32 + c * 4);
-              e8.x = palette4(v & 0xFFFFu, p.palette[0], p.palette[1], p.palette[2], p.palette[3]);
-              e8.y = palette4(v >> 16, p.palette[0], p.palette[1], p.palette[2], p.palette[3]);
             }
           }
-          const uint2 lo = merge4(s8.x, e8.x);
-          const uint2 hi = merge4(s8.y, e8.y);
+          const uint2 lo = merge4(s8[i].x, e8[i].x);
+          const uint2 hi = merge4(s8[i].y, e8[i].y);
           *reinterpret_cast<uint4*>(wt + r * 128 + ((c ^ (r & 7)) << 4)) =
               make_uint4(lo.x, lo.y, hi.x, hi.y);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(bar(b_wfull + wslot));
-          mbar_arrive(bar(b_empty + stage));
-        }
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
-        if (++wslot == kWSlots) {
-          wslot = 0;
-          wphase ^= 1u;
+          mbar_arrive(bar(b_wfull + cur_wslot));
+          mbar_arrive(bar(b_empty + cur_stage));
         }
       }
       u += kb1 - kb0;
@@ -454,39 +509,59 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
   }
 }
 
 // Finish tiles whose K range was split between CTAs: add the partial sums in
-// K order (CTA order) and write Y.
+// K order (CTA order) and write Y.  One block per output tile, one thread per
+// W row of the tile; the contributing CTAs' slots are resolved once per block.
+constexpr int kMaxSplit = 256;  // a tile spans at most gridDim CTAs (<= SM count)
+constexpr int kFixCols = 16;    // output columns (tokens) per fix-up block
+
 __global__ void __launch_bounds__(128) splitk_fixup_kernel(const __grid_constant__ GemmParams p,
                                                            int64_t G) {
+  __shared__ int64_t base[kMaxSplit];
   const int64_t t = blockIdx.x;
   const int64_t ua = t * p.KB, ub = ua + p.KB - 1;
   const int64_t i0 = unit_owner(ua, p.units, G), i1 = unit_owner(ub, p.units, G);
   if (i0 == i1) return;  // written by the GEMM itself
+  const int nsplit = (int)(i1 - i0 + 1);
+  for (int q = threadIdx.x; q < nsplit && q < kMaxSplit; q += blockDim.x) {
+    const int64_t i = i0 + q;
+    const int64_t s = unit_begin(i, p.units, G), e = unit_begin(i + 1, p.units, G);
+    // first segment of CTA i lives in slot 0, its last in slot 1
+    base[q] = (s == e) ? -1 : (i * 2 + ((s / p.KB == t) ? 0 : 1)) * (int64_t)p.tile_n * kBM;
+  }
+  __syncthreads();
   const int row = threadIdx.x;
   const int64_t nt = t / p.MT, mt = t - nt * p.MT;
   const int64_t n = nt * kBM + row;
   const int64_t m0 = mt * p.tile_n;
   const int cols = (int)imin64(p.tile_n, p.M - m0);
-  if (n >= p.N) return;
-  for (int j = 0; j < cols; ++j) {
-    float acc = 0.f;
-    for (int64_t i = i0; i <= i1; ++i) {
-      const int64_t s = unit_begin(i, p.units, G), e = unit_begin(i + 1, p.units, G);
-      if (s == e) continue;
-      const int slot = (s / p.KB == t) ? 0 : 1;  // first segment of CTA i, or its last
-      acc += p.partials[((i * 2 + slot) * p.tile_n + j) * kBM + row];
-    }
-    const int64_t o = (m0 + j) * p.N + n;
+  const int j0 = blockIdx.y * kFixCols;  // this block's columns (tokens)
+  if (n >= p.N || j0 >= cols) return;
+  const int ns = nsplit < kMaxSplit ? nsplit : kMaxSplit;
+  float acc[kFixCols];
+#pragma unroll
+  for (int jj = 0; jj < kFixCols; ++jj) acc[jj] = 0.f;
+  for (int q = 0; q < ns; ++q) {
+    if (base[q] < 0) continue;
+    const float* src = p.partials + base[q] + (int64_t)j0 * kBM + row;
+#pragma unroll
+    for (int jj = 0; jj < kFixCols; ++jj)  // independent loads in flight
+      if (j0 + jj < cols) acc[jj] += src[(int64_t)jj * kBM];
+  }
+#pragma unroll
+  for (int jj = 0; jj < kFixCols; ++jj) {
+    if (j0 + jj >= cols) break;
+    const int64_t o = (m0 + j0 + jj) * p.N + n;
     if (p.out_f32)
-      static_cast<float*>(p.Y)[o] = acc;
+      static_cast<float*>(p.Y)[o] = acc[jj];
     else
-      static_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(acc);
+      static_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(acc[jj]);
   }
 }
 
@@ -535,17 +610,20 @@ uint64_t wait_limit_ns() {
   return ns;
 }
 
+int mma_warps_for(int tile_n) { return tile_n <= 128 ? 2 : 1; }
+
 int tmem_cols_for(int tile_n) {
   int c = 32;
-  while (c < 2 * tile_n) c *= 2;
+  while (c < 2 * mma_warps_for(tile_n) * tile_n) c *= 2;
   return c;
 }
 
-size_t smem_bytes(int mode, int tile_n, int stages) {
+size_t smem_bytes(int mode, int tile_n, int stages, int wslots) {
   const StageLayout L = stage_layout(mode, tile_n);
+  const int ws = mode == kGemmBf16 ? 0 : wslots;
   size_t b = 1024 /* alignment slack */ + (size_t)stages * L.bytes;
-  if (mode != kGemmBf16) b += kWSlots * kWTileBytes;
-  b += (size_t)(2 * stages + 2 * kWSlots + 5) * 8 + 16;
+  b += (size_t)ws * kWTileBytes;
+  b += (size_t)(2 * stages + 2 * ws + 6) * 8 + 16;
   return b;
 }
 
@@ -566,13 +644,23 @@ bool gemm_resolve(GemmArgs* a) {
     a->tile_n = (int)((per + 15) / 16 * 16);
   }
   if (a->tile_n < 16 || a->tile_n > 256 || a->tile_n % 16) return false;
-  const int max_stages = 8;
+  const int max_stages = a->mode == kGemmBf16 ? 12 : 8;
+  // rebuilt-W ring: 4 slots, fewer only when shared memory is short
+  if (a->wslots == 0) a->wslots = a->mode == kGemmBf16 ? 0 : 4;
+  if (a->mode != kGemmBf16 && (a->wslots < 2 || a->wslots > kMaxWSlots)) return false;
   if (a->stages == 0) {
-    int s = max_stages;
-    while (s > 2 && smem_bytes(a->mode, a->tile_n, s) > (size_t)kSmemLimit) --s;
-    a->stages = s;
+    for (;;) {
+      int s = max_stages;
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots) > (size_t)kSmemLimit) --s;
+      if (smem_bytes(a->mode, a->tile_n, s, a->wslots) <= (size_t)kSmemLimit || a->wslots <= 2) {
+        a->stages = s;
+        break;
+      }
+      a->wslots -= 1;
+    }
   }
-  if (a->stages < 2 || smem_bytes(a->mode, a->tile_n, a->stages) > (size_t)kSmemLimit)
+  if (a->stages < 2 ||
+      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots) > (size_t)kSmemLimit)
     return false;
   const int64_t NT = (a->N + kBM - 1) / kBM;
   const int64_t MT = (a->M + a->tile_n - 1) / a->tile_n;
@@ -620,18 +708,20 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.K = a.K;
   p.tile_n = a.tile_n;
   p.stages = a.stages;
+  p.wslots = a.wslots;
   p.NT = (int32_t)((a.N + kBM - 1) / kBM);
   p.MT = (int32_t)((a.M + a.tile_n - 1) / a.tile_n);
   p.KB = (int32_t)KB;
   p.units = (int64_t)p.NT * p.MT * KB;
   p.esc_nwp = a.esc_nw;
   p.out_f32 = a.out_f32;
+  p.n_mma = mma_warps_for(a.tile_n);
   p.tmem_cols = tmem_cols_for(a.tile_n);
   std::memcpy(p.palette, a.palette, 16);
   p.x_bytes = (uint32_t)a.tile_n * kBK * 2;
   p.stage_bytes = stage_layout(a.mode, a.tile_n).bytes;
   p.wait_ns = wait_limit_ns();
-  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages);
+  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots);
   const int G = a.ctas;
   cudaError_t e = cudaSuccess;
   auto begin = [&](int kind) { return hooks && hooks->begin ? hooks->begin(hooks->ctx, kind) : -1; };
@@ -661,7 +751,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   // tiles split between CTAs get their sum here (only when some tile is split)
   if (p.units % G != 0 || (p.units / G) % KB != 0) {
     const int fs = begin(6);
-    splitk_fixup_kernel<<<(unsigned)(p.NT * p.MT), kBM, 0, s>>>(p, G);
+    const dim3 fgrid((unsigned)(p.NT * p.MT), (unsigned)((a.tile_n + kFixCols - 1) / kFixCols));
+    splitk_fixup_kernel<<<fgrid, kBM, 0, s>>>(p, G);
     end(fs);
     e = cudaGetLastError();
   }

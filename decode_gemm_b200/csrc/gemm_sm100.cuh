@@ -53,11 +53,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete, giving up after
 // limit_ns of wall time or when *abort is raised by another warp.
+// A nonzero sleep_ns makes the waiting thread back off between polls (for
+// waits that are expected to be long).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort, uint64_t limit_ns) {
+                                                  volatile int* abort, uint64_t limit_ns,
+                                                  uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255) == 0) {
       if (*abort) return false;

@@ -26,9 +26,8 @@ struct uw_handle_s {
   void* d_block = nullptr;
   uint32_t* d_words = nullptr;
   uint32_t* d_chunk_off = nullptr;
-  uint32_t* d_exp_lut = nullptr;
-  uint32_t* d_pal_lut = nullptr;
-  uint32_t* d_limit = nullptr;
+  uint32_t* d_lut = nullptr;
+  uint32_t* d_canon = nullptr;
   uint8_t* d_sm = nullptr;
   uint32_t* d_esc_bits = nullptr;
   uint32_t* d_esc_off = nullptr;

@@ -14,21 +14,29 @@ constexpr int kEscGroupRows = 128;  // rows per escape-row group (one GEMM row t
 constexpr int kLutBits = 12;        // decode-table index width (= largest code length)
 constexpr int kLutSize = 1 << kLutBits;
 
-// Decode-table entry (one u32 per 12-bit window of the stream):
-//   bits  0..23  decoded values, first one in the lowest bits
-//                (exponent table: 8-bit exponents, up to 3;
-//                 palette table: 4-bit palette indices, up to 6)
-//   bits 24..26  number of values decoded from this window (0 = invalid code)
-//   bits 28..31  number of stream bits those values consume
-constexpr int kExpCap = 3;
+// Decode-table entry (one u32 per 12-bit window of the stream).  The table
+// decodes to 4-bit palette ranks; all three preprocessing outputs derive from
+// them (exponent = palette[rank]).
+//   bits  0..23  ranks of the codes that fit in the window, first one lowest,
+//                at most kPalCap of them, stopping before any exponent that is
+//                not in the palette
+//   bits 24..26  number of ranks (0: see bit 27)
+//   bit  27      raw: the window starts with the code of an exponent outside the
+//                palette; bits 0..7 hold that exponent (one symbol)
+//   bits 28..31  stream bits consumed (0: the window starts with no code)
 constexpr int kPalCap = 6;
+constexpr uint32_t kLutRaw = 1u << 27;
+
+// Canonical-code tables for one-symbol-at-a-time decoding (chunk tails, slow
+// path): limit[l] = first 12-bit window whose first code is longer than l;
+// first[l] = first code of length l; offset[l] = index in `symbols` of the
+// first symbol of length l; symbols = exponents ordered by (length, value).
+constexpr int kCanonLimit = 0, kCanonFirst = 16, kCanonOffset = 32, kCanonSymbols = 48;
+constexpr int kCanonWords = 48 + 64;
 
 struct DecodeTables {
-  std::vector<uint32_t> exp_lut;   // kLutSize entries
-  std::vector<uint32_t> pal_lut;   // kLutSize entries
-  // limit[l] (l = 1..12): first 12-bit window value whose first code is longer
-  // than l; a window's first code length is the least l with window < limit[l].
-  uint32_t limit[16];
+  std::vector<uint32_t> lut;      // kLutSize entries
+  uint32_t canon[kCanonWords];
 };
 
 // Build the decode tables for canonical codes with the given lengths.

@@ -13,8 +13,9 @@ enum DecodeMode { kDecodeExp = 0, kDecodeFull = 1, kDecodePalette = 2 };
 struct DecodeArgs {
   const uint32_t* words;      // Huffman stream, n_words (a multiple of 4) words
   const uint32_t* chunk_off;  // n_chunks + 1 bit offsets
-  const uint32_t* lut;        // 4096-entry decode table (exponent or palette flavour)
-  const uint32_t* limit;      // 16 words: first-code-length limits (see DecodeTables)
+  const uint32_t* lut;        // 4096-entry rank table (see DecodeTables)
+  const uint32_t* canon;      // canonical-code tables (kCanonWords words)
+  uint32_t palette[4];        // the 16 palette exponents, byte i = rank i
   const uint8_t* sm;          // sign+mantissa bytes (full decode only)
   const uint32_t* esc_bits;   // escape bitmap (palette transcode only)
   uint32_t* status;           // device status word (bit 0: bad chunk)
@@ -61,7 +62,8 @@ struct GemmArgs {
   float* partials = nullptr;     // workspace for split partial sums
   size_t partials_bytes = 0;
   int tile_n = 0;                // tokens per tile (0 = auto)
-  int stages = 0;                // ring depth (0 = auto)
+  int stages = 0;                // load ring depth (0 = auto)
+  int wslots = 0;                // rebuilt-W ring depth (0 = auto)
   int ctas = 0;                  // persistent CTAs (0 = SM count)
   int sm_count = 148;
   uint32_t* status = nullptr;
