@@ -273,14 +273,17 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     }
   } else if (warp < kMmaWarp0 + kNumMmaWarps) {
     // ---------------------------------------------------------- MMA issuers --
-    // Warp kMmaWarp0 + par takes the K blocks with kb % 2 == par (all of them
-    // when NM == 1) and accumulates into its own TMEM columns.
+    // Warp kMmaWarp0 + par takes the CTA's units q with q % 2 == par (all of
+    // them when NM == 1) and accumulates into its own TMEM columns.  The ring
+    // depths are even, so a stage or W slot is always consumed by the same
+    // warp, in order: a parity wait can then never see a stale phase.
     const int par = warp - kMmaWarp0;
     if (par < NM) {
       const uint32_t idesc = idesc_bf16(kBM, p.tile_n);
       // ring positions of the current unit, advanced for every unit of the CTA
       int stage = 0, wslot = 0;
       uint32_t phase = 0, wphase = 0;
+      int q = 0;  // index of the unit among this CTA's units
       int seg = 0;
       bool ok = true;
       for (int64_t u = u0; u < u1 && ok; ++seg) {
@@ -299,8 +302,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)((acc * NM + par) * p.tile_n);
         bool first = true;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          const bool mine = NM == 1 || (kb & 1) == par;
+        for (int kb = kb0; kb < kb1; ++kb, ++q) {
+          const bool mine = NM == 1 || (q & 1) == par;
           if (mine && lane == 0) {
             bool got = mbar_wait_bounded(bar(b_full + stage), phase, abort, p.wait_ns);
             if (got && MODE != kGemmBf16)
@@ -353,6 +356,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
     int seg = 0;
+    int64_t qa = 0;  // index (among this CTA's units) of the segment's first unit
     for (int64_t u = u0; u < u1; ++seg) {
       const int64_t t = u / KB;
       const int kb0 = (int)(u - t * KB);
@@ -373,8 +377,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int64_t m0 = mt * p.tile_n;
       const int cols = (int)imin64(p.tile_n, p.M - m0);
       // which parity accumulators received MMAs in this segment
-      const bool has0 = NM == 1 || (kb1 - kb0 >= 2) || ((kb0 & 1) == 0);
-      const bool has1 = NM == 2 && ((kb1 - kb0 >= 2) || ((kb0 & 1) == 1));
+      const bool has0 = NM == 1 || (kb1 - kb0 >= 2) || ((qa & 1) == 0);
+      const bool has1 = NM == 2 && ((kb1 - kb0 >= 2) || ((qa & 1) == 1));
       const uint32_t lanebase = (uint32_t)(quad * 32) << 16;
       const uint32_t t0 = tmem_base + lanebase + (uint32_t)((acc * NM + 0) * p.tile_n);
       const uint32_t t1 = tmem_base + lanebase + (uint32_t)((acc * NM + 1) * p.tile_n);
@@ -407,6 +411,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(b_tempty + acc));
       u += kb1 - kb0;
+      qa += kb1 - kb0;
     }
   } else if constexpr (MODE != kGemmBf16) {
     // ------------------------------------------------------------- rebuild --
@@ -644,22 +649,26 @@ bool gemm_resolve(GemmArgs* a) {
     a->tile_n = (int)((per + 15) / 16 * 16);
   }
   if (a->tile_n < 16 || a->tile_n > 256 || a->tile_n % 16) return false;
+  // Ring depths are even: consumers alternate units, so an even depth keeps
+  // every slot with one consumer (see the MMA issuers in the kernel).
   const int max_stages = a->mode == kGemmBf16 ? 12 : 8;
-  // rebuilt-W ring: 4 slots, fewer only when shared memory is short
+  // rebuilt-W ring: 4 slots, 2 when shared memory is short
   if (a->wslots == 0) a->wslots = a->mode == kGemmBf16 ? 0 : 4;
-  if (a->mode != kGemmBf16 && (a->wslots < 2 || a->wslots > kMaxWSlots)) return false;
+  if (a->mode != kGemmBf16 &&
+      (a->wslots < 2 || a->wslots > kMaxWSlots || (a->wslots & 1)))
+    return false;
   if (a->stages == 0) {
     for (;;) {
       int s = max_stages;
-      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots) > (size_t)kSmemLimit) --s;
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots) > (size_t)kSmemLimit) s -= 2;
       if (smem_bytes(a->mode, a->tile_n, s, a->wslots) <= (size_t)kSmemLimit || a->wslots <= 2) {
         a->stages = s;
         break;
       }
-      a->wslots -= 1;
+      a->wslots -= 2;
     }
   }
-  if (a->stages < 2 ||
+  if (a->stages < 2 || (a->stages & 1) ||
       smem_bytes(a->mode, a->tile_n, a->stages, a->wslots) > (size_t)kSmemLimit)
     return false;
   const int64_t NT = (a->N + kBM - 1) / kBM;

@@ -210,3 +210,32 @@ def test_gemm_argument_errors(uw):
     assert uw.lib.uw_gemm_ex(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 4,
                              C.byref(bad), 0) == uw.UW_ERR_ARG
     h.free()
+
+
+@pytest.mark.parametrize("pipe,M,tile_n", [("exp", 256, 0), ("palette_direct", 256, 0),
+                                           ("full", 1, 16), ("palette_rt", 64, 32)])
+def test_gemm_repeatable_bitwise(uw, pipe, M, tile_n):
+    """The same call eight times gives bitwise the same Y (races show up here)."""
+    w = synthdata.student_t(1024, 3584, 3.0, 0.015, seed=100 + M)
+    x = synthdata.activations(M, 3584, seed=101 + M)
+    h = _upload(uw, w, chunk=256)
+    ws = _workspace(uw, h, M)
+    first = _gemm(uw, h, x, pipe, tile_n=tile_n)
+    _check(first, x, w)
+    for _ in range(7):
+        assert np.array_equal(_gemm(uw, h, x, pipe, tile_n=tile_n), first)
+    h.free()
+
+
+def test_odd_ring_depth_rejected(uw):
+    import ctypes as C
+    import torch
+    w = synthdata.normal(128, 256, 0.02, seed=102)
+    h = uw.uw_encode(w)
+    X = torch.zeros((4, 256), dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")
+    for st in (1, 3, 5):
+        cfg = uw.gemm_config(4, stages=st)
+        assert uw.lib.uw_gemm_ex(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 4,
+                                 C.byref(cfg), 0) == uw.UW_ERR_ARG
+    h.free()
