@@ -109,6 +109,7 @@ _SIGS = {
     "uw_get_choice": ([_vp, _i64, C.POINTER(uw_gemm_config)], C.c_int),
     "uw_last_device_status": ([_vp], C.c_int),
     "uw_trace_enable": ([_vp, _i32], C.c_int),
+    "uw_gemm_palette_noalloc": ([_vp, _vp, _vp, _i64, _i32], C.c_int),
     "uw_trace_read": ([_vp, C.POINTER(_i32), C.POINTER(C.c_float), _i32, C.POINTER(_i32)], C.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -362,6 +363,13 @@ def gemm_config(pipeline: int, tile_n: int = 0, stages: int = 0, gemm_ctas: int 
 def uw_gemm_ex(h: Handle, X, Y, M: int, cfg: uw_gemm_config, out_f32: bool) -> None:
     _check(lib.uw_gemm_ex(h.ptr, _vp(_dptr(X)), _vp(_dptr(Y)), int(M), C.byref(cfg),
                           1 if out_f32 else 0), "uw_gemm_ex")
+
+
+def uw_gemm_palette_noalloc(h: Handle, X, Y, M: int, out_f32: bool = False) -> None:
+    """Pipeline-4 matmul that allocates nothing (split-K scratch is a fixed
+    array inside the library); M <= 64.  See include/unweight.h."""
+    _check(lib.uw_gemm_palette_noalloc(h.ptr, _vp(_dptr(X)), _vp(_dptr(Y)), int(M),
+                                       1 if out_f32 else 0), "uw_gemm_palette_noalloc")
 
 
 def uw_autotune(handles, Ms, profile_out_json: str | None = None) -> None:

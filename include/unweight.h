@@ -222,6 +222,29 @@ UW_API uw_status uw_gemm_f32(uw_handle_t h, const uint16_t* X_dev, float* Y_dev,
 UW_API uw_status uw_gemm_ex(uw_handle_t h, const uint16_t* X_dev, void* Y_dev, int64_t M,
                      const uw_gemm_config* cfg, int32_t out_f32);
 
+/* Allocation-free matmul, pipeline 4 only (the paper has no counterpart to
+ * this call; it exists for callers that cannot allocate).  Some callers cannot
+ * allocate device memory while they run a matmul: their allocator is locked or
+ * already committed to a fixed memory plan, or they run where a cudaMalloc
+ * would stall or fail.  uw_gemm needs a registered workspace for split-K
+ * partial sums; this call keeps them in a fixed array compiled into the
+ * library instead, so it allocates nothing (no cudaMalloc, no workspace).
+ *   - Computes Y[M, N] = X W^T like uw_gemm(..., UW_PIPE_PALETTE_DIRECT);
+ *     Y is float* when out_f32 is nonzero, else BF16.  Needs a handle
+ *     uploaded with prepare_direct (UW_ERR_UNSUPPORTED otherwise).
+ *   - Limit: M <= 64 (UW_ERR_SHAPE above that).  The array is 10 MiB and is
+ *     held on every GPU where the library's device code is loaded, until the
+ *     process exits.
+ *   - The handle's device must be current (UW_ERR_ARG otherwise).  The first
+ *     call on a device looks up the array's device address once; make that
+ *     first call before any stream capture.
+ *   - All calls on one GPU share the one array: calls whose kernels overlap
+ *     on that GPU (for example on two streams) race and give wrong results.
+ *     Nothing in it needs to start at zero, and its contents after a call
+ *     are meaningless. */
+UW_API uw_status uw_gemm_palette_noalloc(uw_handle_t h, const uint16_t* X_dev, void* Y_dev,
+                                         int64_t M, int32_t out_f32);
+
 /* Autotuner ("Sharing the GPU between decode and compute", last paragraphs):
  * for every handle and every M in Ms, measure candidate variants (pipeline,
  * token tile, ring depth, decoder/GEMM CTA split) with CUDA events on the
