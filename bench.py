@@ -52,8 +52,14 @@ CPU_BASELINE_ROWS = 300   # oracle rows for the cpu_baseline leg (~12 s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum), valid only while the kernel source is unchanged.
-TRAFFIC = {}
+# dram__bytes_write.sum; profiles/*.md), valid only while the kernel source
+# (src_sha, see _kernel_src_sha) is unchanged.
+TRAFFIC = {
+    "gemm_palette": {"bytes_per_launch": 90.173952e6 + 3.2064e6, "src_sha": "42f5962f3a4e66ea",
+                     "capture": "profiles/gemm_palette_gate_14336x4096_M1.md (M = 1 launch)"},
+    "transcode": {"bytes_per_launch": 19.4304e6 + 0.097024e6, "src_sha": "42f5962f3a4e66ea",
+                  "capture": "profiles/transcode_gate_14336x4096.md (output still in L2)"},
+}
 
 
 def _args():

@@ -424,7 +424,7 @@ int uw_abi_version(void) { return UW_ABI_VERSION; }
 void uw_default_encode_opts(uw_encode_opts* o) {
   if (!o) return;
   o->max_code_len = 12;
-  o->chunk_syms = 1024;
+  o->chunk_syms = 256;
   o->prepare_direct = 1;
   o->reserved = 0;
 }

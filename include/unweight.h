@@ -81,7 +81,7 @@ typedef struct uw_encode_opts {
   int32_t max_code_len;    /* Huffman length cap, 1..12 (default 12: a 2^12-entry
                               4-byte decode table is 16 KB, "Sharing the GPU ...") */
   int32_t chunk_syms;      /* symbols per independently decodable chunk; a positive
-                              multiple of 64 (default 1024)                        */
+                              multiple of 64 (default 256)                         */
   int32_t prepare_direct;  /* nonzero: at upload, transcode once into resident
                               palette indices so UW_PIPE_PALETTE_DIRECT works      */
   int32_t reserved;

@@ -107,16 +107,17 @@ def test_decode_full_size_bit_exact(uw, name):
     assert np.array_equal(gw, w)
     s, e = oracle.split_fields(w)
     assert np.array_equal(ge, e)
-    pal = np.asarray(h_palette(uw, h, w, 1024))
+    pal = np.asarray(h_palette(uw, h, w, 256))
     esc = oracle.escape_rows(e, pal)
     assert np.array_equal(gi, oracle.pack_nibbles(oracle.transcode(e, pal, esc)))
     # sampled chunks through the oracle's bit-by-bit decoder on the library stream
     a = uw.uw_encode_host(w).arrays()
+    cs = int(a["chunk_syms"])
     rng = np.random.default_rng(3)
     for c in rng.choice(a["chunk_off"].size - 1, size=6, replace=False):
-        syms, end = oracle.decode_chunk(a["words"], int(a["chunk_off"][c]), 1024, a["code_len"])
+        syms, end = oracle.decode_chunk(a["words"], int(a["chunk_off"][c]), cs, a["code_len"])
         assert end == int(a["chunk_off"][c + 1])
-        assert np.array_equal(syms, ge.reshape(-1)[c * 1024:(c + 1) * 1024])
+        assert np.array_equal(syms, ge.reshape(-1)[c * cs:(c + 1) * cs])
     h.free()
 
 
