@@ -80,6 +80,18 @@ class uw_gemm_config(C.Structure):
                                                "decode_ctas")}
 
 
+class uw_mlp_layer(C.Structure):
+    _fields_ = [("gate", C.c_void_p), ("up", C.c_void_p), ("down", C.c_void_p)]
+
+
+class uw_mlp_opts(C.Structure):
+    _fields_ = [("overlap", C.c_int32), ("decode_ctas", C.c_int32), ("gemm_ctas", C.c_int32),
+                ("reserved", C.c_int32)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k in ("overlap", "decode_ctas", "gemm_ctas")}
+
+
 _vp, _i32, _i64, _sz = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
 _SIGS = {
     "uw_status_str": ([C.c_int], C.c_char_p),
@@ -110,6 +122,13 @@ _SIGS = {
     "uw_last_device_status": ([_vp], C.c_int),
     "uw_trace_enable": ([_vp, _i32], C.c_int),
     "uw_gemm_palette_noalloc": ([_vp, _vp, _vp, _i64, _i32], C.c_int),
+    "uw_swiglu": ([_vp, _vp, _vp, _i64, _vp], C.c_int),
+    "uw_mlp_workspace_bytes": ([C.POINTER(uw_mlp_layer), _i32, _i64, C.POINTER(uw_mlp_opts),
+                                C.POINTER(_sz)], C.c_int),
+    "uw_mlp_forward": ([C.POINTER(uw_mlp_layer), _i32, _vp, _vp, _i64, _vp, _sz, _vp, _vp,
+                        C.POINTER(uw_mlp_opts)], C.c_int),
+    "uw_mlp_tune_split": ([C.POINTER(uw_mlp_layer), _i32, _vp, _vp, _i64, _vp, _sz, _vp, _vp,
+                           C.POINTER(uw_mlp_opts)], C.c_int),
     "uw_trace_read": ([_vp, C.POINTER(_i32), C.POINTER(C.c_float), _i32, C.POINTER(_i32)], C.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -370,6 +389,55 @@ def uw_gemm_palette_noalloc(h: Handle, X, Y, M: int, out_f32: bool = False) -> N
     array inside the library); M <= 64.  See include/unweight.h."""
     _check(lib.uw_gemm_palette_noalloc(h.ptr, _vp(_dptr(X)), _vp(_dptr(Y)), int(M),
                                        1 if out_f32 else 0), "uw_gemm_palette_noalloc")
+
+
+def uw_swiglu(g, u, h, n: int | None = None, stream=None) -> None:
+    n = g.numel() if n is None else int(n)
+    _check(lib.uw_swiglu(_vp(_dptr(g)), _vp(_dptr(u)), _vp(_dptr(h)), n,
+                         _vp(_stream_ptr(stream))), "uw_swiglu")
+
+
+def mlp_layers(layers):
+    """[(gate, up, down) Handles] -> ctypes array of uw_mlp_layer."""
+    arr = (uw_mlp_layer * len(layers))()
+    for i, (g, u, d) in enumerate(layers):
+        arr[i].gate, arr[i].up, arr[i].down = g.ptr.value, u.ptr.value, d.ptr.value
+    return arr
+
+
+def mlp_opts(overlap=False, decode_ctas=0, gemm_ctas=0) -> uw_mlp_opts:
+    o = uw_mlp_opts()
+    o.overlap, o.decode_ctas, o.gemm_ctas = int(bool(overlap)), int(decode_ctas), int(gemm_ctas)
+    return o
+
+
+def uw_mlp_workspace_bytes(layers, M: int, opts: uw_mlp_opts | None = None) -> int:
+    arr = mlp_layers(layers)
+    out = _sz()
+    _check(lib.uw_mlp_workspace_bytes(arr, len(layers), int(M), C.byref(opts) if opts else None,
+                                      C.byref(out)), "uw_mlp_workspace_bytes")
+    return int(out.value)
+
+
+def uw_mlp_forward(layers, X, Y, M: int, ws, opts: uw_mlp_opts | None = None, stream=None,
+                   side_stream=None) -> None:
+    arr = mlp_layers(layers)
+    nbytes = ws.numel() * ws.element_size()
+    side = _vp(_stream_ptr(side_stream)) if side_stream is not None else None
+    _check(lib.uw_mlp_forward(arr, len(layers), _vp(_dptr(X)), _vp(_dptr(Y)), int(M),
+                              _vp(_dptr(ws)), nbytes, _vp(_stream_ptr(stream)), side,
+                              C.byref(opts) if opts else None), "uw_mlp_forward")
+
+
+def uw_mlp_tune_split(layers, X, Y, M: int, ws, stream=None, side_stream=None) -> uw_mlp_opts:
+    arr = mlp_layers(layers)
+    best = uw_mlp_opts()
+    nbytes = ws.numel() * ws.element_size()
+    _check(lib.uw_mlp_tune_split(arr, len(layers), _vp(_dptr(X)), _vp(_dptr(Y)), int(M),
+                                 _vp(_dptr(ws)), nbytes, _vp(_stream_ptr(stream)),
+                                 _vp(_stream_ptr(side_stream)), C.byref(best)),
+           "uw_mlp_tune_split")
+    return best
 
 
 def uw_autotune(handles, Ms, profile_out_json: str | None = None) -> None:

@@ -29,19 +29,6 @@ uw_status map_cuda(cudaError_t e) {
     if (e_ != cudaSuccess) return map_cuda(e_);   \
   } while (0)
 
-// Make the handle's device current for the scope of a call.
-struct DeviceGuard {
-  int prev = -1;
-  bool changed = false;
-  explicit DeviceGuard(int dev) {
-    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
-      changed = cudaSetDevice(dev) == cudaSuccess;
-    }
-  }
-  ~DeviceGuard() {
-    if (changed) cudaSetDevice(prev);
-  }
-};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -85,6 +72,14 @@ bool valid_pipeline(int p) { return p >= UW_PIPE_FULL && p <= UW_PIPE_PALETTE_DI
 }  // namespace
 
 namespace uw {
+// Make the handle's device current for the scope of a call.
+DeviceGuard::DeviceGuard(int dev) {
+  if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) changed = cudaSetDevice(dev) == cudaSuccess;
+}
+DeviceGuard::~DeviceGuard() {
+  if (changed) cudaSetDevice(prev);
+}
+
 DecodeArgs decode_args(const uw_handle_s* h) {
   DecodeArgs a;
   a.words = h->d_words;
@@ -178,6 +173,52 @@ uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
   return UW_OK;
 }
 
+uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg) {
+  if (!valid_pipeline(cfg.pipeline)) return UW_ERR_ARG;
+  if (cfg.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) return UW_ERR_UNSUPPORTED;
+  if (cfg.tile_n < 0 || cfg.tile_n > 256 || cfg.tile_n % 16) return UW_ERR_ARG;
+  if (cfg.stages < 0 || cfg.stages > 12 || (cfg.stages & 1)) return UW_ERR_ARG;
+  if (cfg.gemm_ctas < 0 || cfg.decode_ctas < 0) return UW_ERR_ARG;
+  return UW_OK;
+}
+
+size_t preprocessed_bytes(const uw_handle_s* h, int pipeline) {
+  return preprocess_bytes(h, pipeline);
+}
+
+uw_status run_preprocess(uw_handle_s* h, int pipeline, void* out, int ctas, cudaStream_t s) {
+  switch (pipeline) {
+    case UW_PIPE_FULL: return run_decode(h, kDecodeFull, out, ctas, s);
+    case UW_PIPE_EXP: return run_decode(h, kDecodeExp, out, ctas, s);
+    case UW_PIPE_PALETTE_RT: return run_decode(h, kDecodePalette, out, ctas, s);
+    default: return UW_OK;
+  }
+}
+
+// The GEMM of a pipeline on weights already preprocessed into `pre` (ignored
+// for pipeline 4), partial sums in `partials` (gemm_partials_bytes of the plan).
+uw_status run_gemm_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
+                      const uw_gemm_config& cfg, int out_f32, const void* pre, float* partials,
+                      size_t partials_bytes, cudaStream_t s) {
+  GemmArgs a;
+  size_t need = 0, pre_b = 0;
+  uw_status st = plan_gemm(h, X, Y, M, cfg, out_f32, &a, &need, &pre_b);
+  if (st != UW_OK) return st;
+  if (a.partials_bytes > partials_bytes) return UW_ERR_WORKSPACE;
+  a.partials = a.partials_bytes ? partials : nullptr;
+  switch (cfg.pipeline) {
+    case UW_PIPE_FULL: a.W = static_cast<const uint16_t*>(pre); break;
+    case UW_PIPE_EXP: a.E = static_cast<const uint8_t*>(pre); break;
+    case UW_PIPE_PALETTE_RT: a.I = static_cast<const uint8_t*>(pre); break;
+    default: a.I = h->d_pal_idx; break;
+  }
+  LaunchHooks hooks;
+  hooks.ctx = h;
+  hooks.begin = hook_begin;
+  hooks.end = hook_end;
+  return map_cuda(launch_gemm(a, s, &hooks));
+}
+
 uw_status run_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
                    const uw_gemm_config& cfg_in, int out_f32) {
   uw_gemm_config cfg = cfg_in;
@@ -185,14 +226,11 @@ uw_status run_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
     const uw_gemm_config c = choose_variant(h, M);
     cfg = c;
   }
-  if (!valid_pipeline(cfg.pipeline)) return UW_ERR_ARG;
-  if (cfg.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) return UW_ERR_UNSUPPORTED;
-  if (cfg.tile_n < 0 || cfg.tile_n > 256 || cfg.tile_n % 16) return UW_ERR_ARG;
-  if (cfg.stages < 0 || cfg.stages > 12 || (cfg.stages & 1)) return UW_ERR_ARG;
-  if (cfg.gemm_ctas < 0 || cfg.decode_ctas < 0) return UW_ERR_ARG;
+  uw_status st = check_config(h, cfg);
+  if (st != UW_OK) return st;
   GemmArgs a;
   size_t need = 0, pre = 0;
-  uw_status st = plan_gemm(h, X, Y, M, cfg, out_f32, &a, &need, &pre);
+  st = plan_gemm(h, X, Y, M, cfg, out_f32, &a, &need, &pre);
   if (st != UW_OK) return st;
   if (need > 0 && (!h->ws || h->ws_bytes < need)) return UW_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(h->ws);

@@ -51,6 +51,25 @@ struct uw_handle_s {
 
 namespace uw {
 DecodeArgs decode_args(const uw_handle_s* h);
+// Shared by the C ABI, the autotuner and the MLP driver (api.cu).
+uw_gemm_config choose_variant(const uw_handle_s* h, int64_t M);
+uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg);
+size_t preprocessed_bytes(const uw_handle_s* h, int pipeline);
+uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
+                    const uw_gemm_config& cfg, int out_f32, GemmArgs* ga, size_t* ws_need,
+                    size_t* pre_bytes);
+uw_status run_preprocess(uw_handle_s* h, int pipeline, void* out, int ctas, cudaStream_t s);
+uw_status run_gemm_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
+                      const uw_gemm_config& cfg, int out_f32, const void* pre, float* partials,
+                      size_t partials_bytes, cudaStream_t s);
+uw_status run_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
+                   const uw_gemm_config& cfg, int out_f32);
+struct DeviceGuard {
+  int prev = -1;
+  bool changed = false;
+  explicit DeviceGuard(int dev);
+  ~DeviceGuard();
+};
 // Record the start event of a traced launch (no-op unless tracing); returns the
 // slot to pass to trace_end, or -1.
 int trace_begin(uw_handle_s* h, int kind);

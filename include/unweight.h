@@ -246,12 +246,16 @@ UW_API uw_status uw_gemm_palette_noalloc(uw_handle_t h, const uint16_t* X_dev, v
                                          int64_t M, int32_t out_f32);
 
 /* Autotuner ("Sharing the GPU between decode and compute", last paragraphs):
- * for every handle and every M in Ms, measure candidate variants (pipeline,
- * token tile, ring depth, decoder/GEMM CTA split) with CUDA events on the
- * handle's stream, by coordinate descent over the projections until no
- * change improves the total time; store the winners in the handles and, when
- * profile_out_json is not NULL, write them as JSON.  Needs a workspace on
- * each handle large enough for the largest M (UW_ERR_WORKSPACE otherwise). */
+ * for every M in Ms, coordinate descent over the handles (projections): each
+ * handle in turn tries every candidate variant (pipeline, token tile, ring
+ * depth) while the others keep theirs, scored by the device time (CUDA
+ * events on the first handle's stream) of all handles' matmuls in order;
+ * sweeps repeat until no change gains 1 %.  The winners are stored in the
+ * handles (uw_gemm with UW_PIPE_AUTO uses them) and, when profile_out_json is
+ * not NULL, written as JSON.  Candidates that need more workspace than a
+ * handle has registered are skipped (UW_ERR_WORKSPACE when none fits).  The
+ * tuner allocates its own X/Y buffers.  The decoder/GEMM SM split is tuned
+ * for the overlapped stack by uw_mlp_tune_split. */
 UW_API uw_status uw_autotune(uw_handle_t* hs, int32_t n_handles, const int64_t* Ms, int32_t n_M,
                       const char* profile_out_json);
 /* Load a profile written by uw_autotune into the handles (matched by order and
@@ -274,6 +278,51 @@ typedef enum uw_kernel_kind {
 UW_API uw_status uw_trace_enable(uw_handle_t h, int32_t enable);
 UW_API uw_status uw_trace_read(uw_handle_t h, int32_t* kinds, float* ms, int32_t capacity,
                                int32_t* count);
+
+/* ---- MLP stack ("Sharing the GPU between decode and compute") ------------ */
+
+/* One SwiGLU block: gate and up are [F, D] weights, down is [D, F]. */
+typedef struct uw_mlp_layer {
+  uw_handle_t gate, up, down;
+} uw_mlp_layer;
+
+typedef struct uw_mlp_opts {
+  int32_t overlap;      /* nonzero: projections whose pipeline needs preprocessing
+                           ("hard": 1-3) are preprocessed on side_stream one hard
+                           projection ahead, into two alternating workspace slots,
+                           while the main stream runs the GEMMs                     */
+  int32_t decode_ctas;  /* SM split, decoder share: CTAs of each side-stream
+                           preprocessing kernel (0 = as many as it needs)            */
+  int32_t gemm_ctas;    /* SM split, GEMM share: CTAs of each GEMM while the stack
+                           runs (0 = one per SM); a profile's own value wins         */
+  int32_t reserved;
+} uw_mlp_opts;
+
+/* h[i] = SiLU(g[i]) * u[i] for n BF16 values (SiLU and product in FP32, result
+ * rounded to nearest even); device pointers, 16-byte aligned, on `stream`. */
+UW_API uw_status uw_swiglu(const uint16_t* g_dev, const uint16_t* u_dev, uint16_t* h_dev,
+                           int64_t n, void* stream);
+/* Workspace uw_mlp_forward needs for these layers, M and options. */
+UW_API uw_status uw_mlp_workspace_bytes(const uw_mlp_layer* layers, int32_t n_layers, int64_t M,
+                                        const uw_mlp_opts* opts, size_t* bytes);
+/* x_0 = X [M, D]; x_{l+1} = (SiLU(x_l Wg^T) * (x_l Wu^T)) Wd^T; Y = x_L [M, D].
+ * Each projection uses the variant its handle's profile picks for M (see
+ * uw_autotune / uw_load_profile; default otherwise).  X, Y device pointers
+ * (16-byte aligned, may alias); ws_dev caller-owned, 256-byte aligned, at least
+ * uw_mlp_workspace_bytes; the handles' own workspaces are not used.  Work is
+ * enqueued on `stream` (and side_stream when overlapping; the call orders it
+ * after all earlier work on `stream`).  Errors as uw_gemm, UW_ERR_SHAPE when
+ * the layers' shapes do not chain. */
+UW_API uw_status uw_mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uint16_t* X_dev,
+                                uint16_t* Y_dev, int64_t M, void* ws_dev, size_t ws_bytes,
+                                void* stream, void* side_stream, const uw_mlp_opts* opts);
+/* Decoder/GEMM SM split for the overlapped stack: time uw_mlp_forward (overlap
+ * on) for a few (decode_ctas, gemm_ctas) pairs and no split, return the
+ * fastest in *best.  Synchronises `stream`. */
+UW_API uw_status uw_mlp_tune_split(const uw_mlp_layer* layers, int32_t n_layers,
+                                   const uint16_t* X_dev, uint16_t* Y_dev, int64_t M, void* ws_dev,
+                                   size_t ws_bytes, void* stream, void* side_stream,
+                                   uw_mlp_opts* best);
 
 /* Synchronise the handle's stream, then return and clear the device status
  * word: UW_OK, UW_ERR_DEVICE (a chunk decoded to the wrong bit count or hit an

@@ -26,7 +26,7 @@ from .huffman import (package_merge_lengths, canonical_codes, encode_bitstream,
                       decode_bitstream, decode_chunk, chunk_offsets, kraft_sum,
                       entropy_bits, average_code_length)
 from .container import encode, decode_full, decode_exp, transcode_from_stream, Encoded
-from .gemm import gemm_fp64, abs_product_sum, within_tolerance, gemm_entry_fsum
+from .gemm import gemm_fp64, abs_product_sum, within_tolerance, gemm_entry_fsum, swiglu
 
 __all__ = [
     "split_fields", "join_fields", "exponent_bytes", "to_float64",
@@ -35,5 +35,5 @@ __all__ = [
     "package_merge_lengths", "canonical_codes", "encode_bitstream", "decode_bitstream",
     "decode_chunk", "chunk_offsets", "kraft_sum", "entropy_bits", "average_code_length",
     "encode", "decode_full", "decode_exp", "transcode_from_stream", "Encoded",
-    "gemm_fp64", "abs_product_sum", "within_tolerance", "gemm_entry_fsum",
+    "gemm_fp64", "abs_product_sum", "within_tolerance", "gemm_entry_fsum", "swiglu",
 ]

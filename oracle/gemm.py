@@ -39,6 +39,17 @@ def gemm_entry_fsum(x_bits: np.ndarray, w_bits: np.ndarray, m: int, n: int) -> f
     return math.fsum((x * w).tolist())
 
 
+def swiglu(g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
+    """SwiGLU of the MLP block between the gate/up and the down projection:
+    ``h = SiLU(g) * u`` with ``SiLU(g) = g / (1 + exp(-g))``, from BF16 inputs,
+    in float64 (*Unweight*, results section: the method targets SwiGLU MLPs).
+    Reading taken: the GPU computes it in FP32 and rounds h once to BF16, so a
+    result within one BF16 rounding (2**-8 relative) of this value is exact."""
+    g = to_float64(g_bits)
+    u = to_float64(u_bits)
+    return g / (1.0 + np.exp(-g)) * u
+
+
 def tolerance(bound: np.ndarray, y_ref: np.ndarray, bf16_output: bool) -> np.ndarray:
     tol = 1e-3 * bound + 1e-6
     if bf16_output:

@@ -338,3 +338,14 @@ def test_synthetic_row_prefix_is_stable():
     a = synthdata.workload("gate_14336x4096", rows=8)
     b = synthdata.normal(32, 4096, 0.02, seed=10)[:8]
     assert np.array_equal(a, b)
+
+
+def test_swiglu_closed_forms():
+    g = synthdata.to_bf16_bits(np.array([0.0, 1.0, -1.0, 8.0, -8.0, 2.0], np.float32))
+    u = synthdata.to_bf16_bits(np.array([5.0, 1.0, 1.0, 1.0, 1.0, 0.0], np.float32))
+    h = oracle.swiglu(g, u)
+    assert h[0] == 0.0                                  # SiLU(0) = 0
+    assert h[1] == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)  # sigmoid(1)
+    assert h[1] - h[2] == pytest.approx(1.0, rel=1e-15)  # SiLU(x) - SiLU(-x) = x
+    assert h[3] == pytest.approx(8.0, rel=1e-3) and abs(h[4]) < 3e-3  # tails -> x and 0
+    assert h[5] == 0.0                                  # u = 0
