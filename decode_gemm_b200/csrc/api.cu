@@ -301,7 +301,9 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   struct Part { void** dst; const void* src; size_t bytes; };
   size_t off = 0;
   auto place = [&](size_t bytes) { size_t at = off; off = align_up(off + bytes, 256); return at; };
-  const size_t o_words = place((size_t)f->n_words * 4);
+  // the stream is followed by zero words: the decoder reads past a chunk's end
+  const int64_t pad_words = stream_pad_words(f->chunk_syms);
+  const size_t o_words = place((size_t)(f->n_words + pad_words) * 4);
   const size_t o_coff = place((size_t)(f->n_chunks + 1) * 4);
   const size_t o_lut = place(kLutSize * 4);
   const size_t o_canon = place(kCanonWords * 4);
@@ -343,6 +345,8 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
     e = cudaMemcpyAsync(*p.dst, p.src, p.bytes, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) break;
   }
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(h->d_words + f->n_words, 0, (size_t)pad_words * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->d_status, 0, 256, s);
   if (e == cudaSuccess && h->d_pal_idx) {
     // load-time transcode: the resident palette form of pipeline 4

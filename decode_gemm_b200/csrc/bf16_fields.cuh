@@ -24,4 +24,15 @@ __device__ __forceinline__ uint32_t palette4(uint32_t v16, uint32_t p0, uint32_t
   return __byte_perm(lo, hi, pick);
 }
 
+// Exponent bytes of eight 4-bit palette indices (nibble i of v -> byte i of
+// the pair, low word first).
+__device__ __forceinline__ uint2 palette8(uint32_t v, uint32_t p0, uint32_t p1, uint32_t p2,
+                                          uint32_t p3) {
+  const uint32_t sel = v & 0x77777777u;                        // index mod 8 per nibble
+  const uint32_t pick = ((v >> 1) & 0x44444444u) | 0x32103210u;  // byte of lo or of hi
+  const uint32_t lo0 = __byte_perm(p0, p1, sel), hi0 = __byte_perm(p2, p3, sel);
+  const uint32_t lo1 = __byte_perm(p0, p1, sel >> 16), hi1 = __byte_perm(p2, p3, sel >> 16);
+  return make_uint2(__byte_perm(lo0, hi0, pick), __byte_perm(lo1, hi1, pick >> 16));
+}
+
 }  // namespace uw

@@ -7,26 +7,34 @@
 //
 // Design (B200):
 //   * One lane decodes one chunk (its start bit is stored, so chunks are
-//     independent); a warp owns 32 consecutive chunks; 16 warps share the
-//     table in shared memory.
-//   * The 4096-entry table maps the next 12 stream bits to up to 6 palette
-//     ranks and the bits they use.  Every output derives from ranks: the
-//     transcode writes them, the exponent and full decodes expand them through
-//     the 16-entry palette with byte permutes.  A code for an exponent outside
-//     the palette (rare; only inside escape rows) is a one-symbol "raw" entry:
-//     the transcode writes rank 0 (the row is zeroed anyway); the other modes
-//     record the exponent as a per-lane exception and patch it after the
-//     coalesced write, or, when a lane's exception list overflows, replay the
-//     whole chunk one symbol at a time.
-//   * Bit buffer in two registers with funnel shifts; it is topped up 32 bits
-//     at a time from 8-byte loads (next pair prefetched), once per two lookups.
-//   * In the last few symbols of a chunk the lane decodes one symbol per lookup
-//     (first-code length from the canonical limits) so it stops exactly at the
-//     chunk's end bit, which is checked against the stored offset.
-//   * Each lane stages 256 decoded symbols (4 rows of 64) in shared memory;
-//     the warp then writes its 32 lanes' rows so each row is one contiguous,
-//     fully used run of 32-byte sectors (full decode merges the sign+mantissa
-//     bytes on the way out).
+//     independent); a warp owns 32 consecutive chunks; one CTA per SM, whose
+//     16-32 warps share the table in shared memory, strides over the chunk
+//     groups (the warp count is picked so the last pass is nearly full).
+//   * The 4096-entry table maps the next 12 stream bits to up to 5 palette
+//     ranks, the number of stream bits they use and 4x their count.  Every
+//     output derives from ranks: the transcode writes them, the exponent and
+//     full decodes expand them through the 16-entry palette with byte
+//     permutes.  A window that starts with the code of an exponent outside the
+//     palette (rare; only inside escape rows) yields a rank-0 placeholder and
+//     is flagged: the transcode ignores it (the row is zeroed anyway); the
+//     other modes record the exponent as a per-lane exception and patch it
+//     after the coalesced write, or, when a lane's exception list overflows,
+//     replay the whole chunk one symbol at a time.
+//   * Bit reader: a window of four stream words and a bit offset q < 32 into
+//     the first; a lookup reads the 12 bits at q with one funnel shift, and the
+//     window slides by a word (one predicated load, no branch) once q passes
+//     32.  Lookups go in pairs with one slide per pair.
+//   * While at least 2 x 5 symbols of the chunk are left every lookup takes
+//     its whole entry with no per-lookup checks; the last few symbols go one
+//     code at a time where an entry holds more than are left, so a lane stops
+//     exactly at its chunk's last symbol, and its end bit is checked against
+//     the stored offset.
+//   * Ranks are packed into words (8 per word) in registers and each completed
+//     word goes to a per-lane shared-memory row (stride 17 words: lanes that
+//     store their k-th word at the same time hit distinct banks).  After a
+//     128-symbol round the warp writes its 32 chunks' outputs with 128-bit
+//     stores, each warp-wide store covering contiguous, fully used lines.
+//     Shared memory stays small so L1 can hold every lane's stream lines.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -40,82 +48,78 @@ namespace uw {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kRoundSyms = 256;                 // symbols per lane per staging round
-constexpr int kRoundWords = kRoundSyms / 8;     // 32 words of 4-bit ranks
-constexpr int kStageStride = kRoundWords + 1;   // lanes spread over banks
-constexpr int kExcCap = 8;                      // exceptions held per lane
+constexpr int kMaxWarps = 32;                   // one CTA per SM, up to 1024 threads
+constexpr int kMinWarps = 16;
+constexpr int kRoundSyms = 128;                 // symbols per lane per staging round
+constexpr int kRoundWords = kRoundSyms / 8;     // 16 words of 4-bit ranks
+constexpr int kStageStride = kRoundWords + 1;   // 17: lanes spread over banks
+constexpr int kExcCap = 4;                      // exceptions held per lane
+constexpr int kFullPair = 2 * 4 * kPalCap;      // 4x symbols two whole lookups may yield
+constexpr int kFullOne = 4 * kPalCap;
 
-struct __align__(16) Smem {
+// Shared memory: the tables, then per warp its ranks stage (32 lanes x 17
+// words) and exception lists.  At most ~104 KB, so L1 keeps over 120 KB for the
+// lanes' stream lines (each lane streams its own).
+struct __align__(16) SmemHead {
   uint32_t lut[kLutSize];
   uint32_t canon[kCanonWords];
-  uint32_t stage[kWarps][32 * kStageStride];
-  uint32_t exc[kWarps][32 * kExcCap];  // (chunk symbol index << 8) | exponent
+};
+constexpr int kWarpSmemWords = 32 * kStageStride + 32 * kExcCap;
+
+size_t smem_bytes(int warps) {
+  return sizeof(SmemHead) + (size_t)warps * kWarpSmemWords * 4;
+}
+
+__device__ __forceinline__ void st_shared_if(uint32_t addr, uint32_t v, bool p) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.shared.u32 [%0], %1;\n\t}"
+               :: "r"(addr), "r"(v), "r"((uint32_t)p) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_global_if(const uint32_t* ptr, uint32_t old, bool p) {
+  uint32_t v = old;
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q ld.global.nc.u32 %0, [%1];\n\t}"
+      : "+r"(v) : "l"(ptr), "r"((uint32_t)p));
+  return v;
+}
+
+// Four consecutive stream words; bit q (MSB first) of w0 is the next bit.
+struct Bits {
+  uint32_t w0, w1, w2, w3;
+  uint32_t q;
+  uint32_t nxt;  // index of the word after w3
 };
 
-struct Reader {
-  uint32_t hi, lo;  // next stream bits, most significant first
-  int nb;           // valid bits in hi:lo
-  uint2 c, cn;      // current and next 8-byte stream words
-  int ci;           // next word of c to use
-  int64_t gi;       // index of the 8-byte group after cn
-  int fed;          // 32-bit words fed into the buffer after the first
-};
-
-__device__ __forceinline__ uint2 ld_pair(const uint2* p, int64_t i, int64_t n) {
-  return i < n ? __ldg(p + i) : make_uint2(0u, 0u);
+__device__ __forceinline__ void bits_init(Bits& b, const uint32_t* words, uint32_t start) {
+  const uint32_t i = start >> 5;
+  b.w0 = __ldg(words + i);
+  b.w1 = __ldg(words + i + 1);
+  b.w2 = __ldg(words + i + 2);
+  b.w3 = __ldg(words + i + 3);
+  b.q = start & 31u;
+  b.nxt = i + 4;
 }
 
-__device__ __forceinline__ void reader_init(Reader& r, const uint2* src, int64_t ng,
-                                            uint32_t start) {
-  const int64_t g = start >> 6;
-  r.c = ld_pair(src, g, ng);
-  r.cn = ld_pair(src, g + 1, ng);
-  r.gi = g + 2;
-  r.ci = (int)((start >> 5) & 1);
-  const uint32_t w = r.ci ? r.c.y : r.c.x;
-  r.hi = w << (start & 31);
-  r.lo = 0;
-  r.nb = 32 - (int)(start & 31);
-  r.fed = 0;
-  if (r.ci) {
-    r.c = r.cn;
-    r.cn = ld_pair(src, r.gi++, ng);
-    r.ci = 0;
-  } else {
-    r.ci = 1;
-  }
+// The 32 stream bits starting at the next bit (q < 32).
+__device__ __forceinline__ uint32_t bits_peek(const Bits& b) {
+  return __funnelshift_l(b.w1, b.w0, b.q);
 }
 
-// Top the buffer up with one 32-bit word when it holds 32 bits or fewer.
-__device__ __forceinline__ void reader_refill(Reader& r, const uint2* src, int64_t ng) {
-  if (r.nb <= 32) {
-    const uint32_t w = r.ci ? r.c.y : r.c.x;
-    r.hi |= __funnelshift_rc(w, 0u, (uint32_t)r.nb);          // w >> nb
-    r.lo |= __funnelshift_lc(0u, w, (uint32_t)(32 - r.nb));   // w << (32 - nb)
-    r.nb += 32;
-    r.fed += 1;
-    if (r.ci) {
-      r.c = r.cn;
-      r.cn = ld_pair(src, r.gi++, ng);
-      r.ci = 0;
-    } else {
-      r.ci = 1;
-    }
-  }
+// Slide the window by one word once q has passed 32 (q < 64).  Reads stay in
+// the padded stream buffer: a lane never reads more than 12 bits per symbol
+// past its chunk's start, plus the window.
+__device__ __forceinline__ void bits_slide(Bits& b, const uint32_t* words) {
+  const bool s = b.q >= 32u;
+  const uint32_t nw = ld_global_if(words + b.nxt, b.w3, s);
+  b.w0 = s ? b.w1 : b.w0;
+  b.w1 = s ? b.w2 : b.w1;
+  b.w2 = s ? b.w3 : b.w2;
+  b.w3 = nw;
+  b.nxt += s ? 1u : 0u;
+  b.q &= 31u;
 }
 
-// Stream bits consumed since reader_init(start).
-__device__ __forceinline__ uint32_t reader_consumed(const Reader& r, uint32_t start) {
-  return (uint32_t)(32 - (int)(start & 31) + 32 * r.fed - r.nb);
-}
-
-__device__ __forceinline__ void reader_consume(Reader& r, uint32_t len) {
-  r.hi = __funnelshift_l(r.lo, r.hi, len);
-  r.lo = __funnelshift_l(0u, r.lo, len);
-  r.nb -= (int)len;
-}
+// Stream bit position of the next bit.
+__device__ __forceinline__ uint32_t bits_pos(const Bits& b) { return (b.nxt - 4u) * 32u + b.q; }
 
 // Length of the code that starts the 12-bit window (canonical limits).
 __device__ __forceinline__ uint32_t first_code_len(const uint32_t* canon, uint32_t idx) {
@@ -124,216 +128,281 @@ __device__ __forceinline__ uint32_t first_code_len(const uint32_t* canon, uint32
   return len;
 }
 
-// One symbol, one lookup at a time (slow path): returns the exponent.
-__device__ __forceinline__ uint32_t slow_symbol(Reader& r, const uint2* src, int64_t ng,
-                                                const uint32_t* canon) {
-  reader_refill(r, src, ng);
-  const uint32_t idx = r.hi >> 20;
+// Exponent whose code starts the 12-bit window, and that code's length.
+__device__ __forceinline__ uint32_t canon_symbol(const uint32_t* canon, uint32_t idx,
+                                                 uint32_t* len_out) {
   const uint32_t len = first_code_len(canon, idx);
   const uint32_t code = idx >> (12 - len);
   const uint32_t k = canon[kCanonOffset + len] + code - canon[kCanonFirst + len];
-  const uint8_t* syms = reinterpret_cast<const uint8_t*>(canon + kCanonSymbols);
-  reader_consume(r, len);
-  return syms[k & 255];
+  *len_out = len;
+  return reinterpret_cast<const uint8_t*>(canon + kCanonSymbols)[k & 255];
+}
+
+// Ranks are appended to a_lo (ab valid bits, < 32 between appends); each
+// completed word is stored at shared address sp, which then moves on.
+struct Packer {
+  uint32_t a_lo, ab;
+  uint32_t sp;
+};
+
+__device__ __forceinline__ void pack(Packer& pk, uint32_t e) {
+  const uint32_t v = e >> 12;
+  const uint32_t c4 = (e >> 4) & 31u;
+  const uint32_t lo = pk.a_lo | (v << pk.ab);
+  const uint32_t hi = __funnelshift_l(v, 0u, pk.ab);  // bits of v past bit 31
+  const uint32_t ab = pk.ab + c4;
+  const bool full = ab >= 32u;
+  st_shared_if(pk.sp, lo, full);
+  pk.sp += full ? 4u : 0u;
+  pk.a_lo = full ? hi : lo;
+  pk.ab = ab & 31u;
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(32 * kMaxWarps, 1)
     decode_kernel(const DecodeArgs a, void* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  for (int i = threadIdx.x; i < kLutSize / 4; i += kThreads)
+  SmemHead& sm = *reinterpret_cast<SmemHead*>(smem_raw);
+  for (int i = threadIdx.x; i < kLutSize / 4; i += blockDim.x)
     reinterpret_cast<uint4*>(sm.lut)[i] = __ldg(reinterpret_cast<const uint4*>(a.lut) + i);
-  for (int i = threadIdx.x; i < kCanonWords; i += kThreads) sm.canon[i] = __ldg(a.canon + i);
+  for (int i = threadIdx.x; i < kCanonWords; i += blockDim.x) sm.canon[i] = __ldg(a.canon + i);
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  uint32_t* stage = sm.stage[warp];
-  uint32_t* exc = sm.exc[warp] + lane * kExcCap;
+  const int n_warps = blockDim.x >> 5;
+  uint32_t* const stage =
+      reinterpret_cast<uint32_t*>(smem_raw + sizeof(SmemHead)) + warp * kWarpSmemWords;
+  const uint32_t st_addr = (uint32_t)__cvta_generic_to_shared(stage + lane * kStageStride);
+  uint32_t* const exc = stage + 32 * kStageStride + lane * kExcCap;
+  const uint32_t* const lut = sm.lut;
   const int64_t groups = (a.n_chunks + 31) / 32;
-  const uint2* src = reinterpret_cast<const uint2*>(a.words);
-  const int64_t ng = a.n_words / 2;
+  const uint32_t* const words = a.words;
+  const uint32_t stream_bits = (uint32_t)(a.n_words * 32);
   const int64_t cs = a.chunk_syms;
   const int rows_per_chunk = (int)(cs / 64);
   const uint32_t p0 = a.palette[0], p1 = a.palette[1], p2 = a.palette[2], p3 = a.palette[3];
+  const int64_t grid_warps = (int64_t)gridDim.x * n_warps;
 
-  for (int64_t grp = (int64_t)blockIdx.x * kWarps + warp; grp < groups;
-       grp += (int64_t)gridDim.x * kWarps) {
+  for (int64_t grp = (int64_t)blockIdx.x * n_warps + warp; grp < groups; grp += grid_warps) {
     const int64_t c0 = grp * 32;
     const int64_t c = c0 + lane;
     const bool live = c < a.n_chunks;
     uint32_t start = 0, end = 0;
     int nsyms = 0;
+    bool bad = false;
     if (live) {
-      start = a.chunk_off[c];
-      end = a.chunk_off[c + 1];
+      start = __ldg(a.chunk_off + c);
+      end = __ldg(a.chunk_off + c + 1);
       const int64_t left = a.total_syms - c * cs;
       nsyms = (int)(left < cs ? left : cs);
+      if (start > stream_bits) {  // corrupt offset: nothing is read
+        bad = true;
+        start = 0;
+        nsyms = 0;
+      }
     }
-    // (output row n, K block kb) of this chunk's first 64-symbol row
-    int n0 = 0, kb0 = 0;
-    if (MODE == kDecodePalette && live) {
-      const int64_t row0 = c * rows_per_chunk;
-      n0 = (int)(row0 / a.kb_per_row);
-      kb0 = (int)(row0 - (int64_t)n0 * a.kb_per_row);
+    // the stream of this warp's next group: into L2 while this one decodes
+    {
+      const int64_t cn = c + grid_warps * 32;
+      if (cn < a.n_chunks) {
+        const uint32_t nb = __ldg(a.chunk_off + cn) >> 3;
+        if (nb < stream_bits / 8) {
+          const char* p = reinterpret_cast<const char*>(words) + nb;
+          asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+          asm volatile("prefetch.global.L2 [%0];" :: "l"(p + 128));
+        }
+      }
     }
     const int my_rounds = (nsyms + kRoundSyms - 1) / kRoundSyms;
     const int warp_rounds = __reduce_max_sync(0xffffffffu, my_rounds);
+    // symbols from the group's first one to the end of the matrix
+    const int64_t grp_syms_left = a.total_syms - c0 * cs;
 
-    Reader rd;
-    reader_init(rd, src, live ? ng : 0, start);
-    uint32_t a_lo = 0, a_hi = 0;  // ranks waiting to be staged (ab bits)
-    int ab = 0;
+    // (row, K block) of the 64-weight row where this lane's round starts
+    int row_n = 0, row_kb = 0;
+    if (MODE == kDecodePalette && live) {
+      const int64_t row0 = c * rows_per_chunk;
+      row_n = (int)(row0 / a.kb_per_row);
+      row_kb = (int)(row0 - (int64_t)row_n * a.kb_per_row);
+    }
+
+    Bits b;
+    bits_init(b, words, start);
+    Packer pk{0u, 0u, st_addr};
+    int left4 = 4 * nsyms;  // 4 x symbols of the chunk not yet decoded
     int nx = 0;
-    bool bad = false, overflow = false;
-    uint32_t* st = stage + lane * kStageStride;
-    // rounds before every lane's last one cannot reach a chunk's end
-    const int fast_rounds = __reduce_min_sync(0xffffffffu, my_rounds) - 1;
+    bool overflow = false;
+
+    // A flagged entry: record the exception (position = symbols decoded so far).
+    auto special = [&](uint32_t e, uint32_t win, int left4_before) {
+      if (e & kLutInvalid) {
+        bad = true;
+      } else if (MODE != kDecodePalette) {
+        uint32_t len;
+        const uint32_t ex = canon_symbol(sm.canon, win >> 20, &len);
+        const uint32_t pos = (uint32_t)((4 * nsyms - left4_before) >> 2);
+        if (nx < kExcCap)
+          exc[nx++] = (pos << 8) | ex;
+        else
+          overflow = true;
+      }
+    };
+    // Two whole lookups (at least 2 x kPalCap symbols left, q < 32).
+    auto lookup_pair = [&]() {
+      const uint32_t win1 = bits_peek(b);
+      const uint32_t e1 = lut[win1 >> 20];
+      const uint32_t q1 = b.q + (e1 & 15u);
+      const bool up = q1 >= 32u;
+      const uint32_t x0 = up ? b.w1 : b.w0, x1 = up ? b.w2 : b.w1;
+      const uint32_t win2 = __funnelshift_l(x1, x0, q1);
+      const uint32_t e2 = lut[win2 >> 20];
+      if ((e1 | e2) & kLutSpecial) {
+        if (e1 & kLutSpecial) special(e1, win1, left4);
+        if (e2 & kLutSpecial) special(e2, win2, left4 - (int)((e1 >> 4) & 31u));
+      }
+      b.q = q1 + (e2 & 15u);
+      left4 -= (int)(((e1 >> 4) & 31u) + ((e2 >> 4) & 31u));
+      pack(pk, e1);
+      pack(pk, e2);
+      bits_slide(b, words);
+    };
+    // One lookup; TAIL: fewer than kPalCap symbols may be left, so an entry
+    // holding more than are left gives way to its first code alone.
+    auto lookup_one = [&](auto tail_tag) {
+      constexpr bool TAIL = decltype(tail_tag)::value;
+      const uint32_t win = bits_peek(b);
+      uint32_t e = lut[win >> 20];
+      if (TAIL && (int)((e >> 4) & 31u) > left4)
+        e = (e & 0xF000u) | (4u << 4) | first_code_len(sm.canon, win >> 20);
+      if (e & kLutSpecial) special(e, win, left4);
+      b.q += e & 15u;
+      left4 -= (int)((e >> 4) & 31u);
+      pack(pk, e);
+      bits_slide(b, words);
+    };
 
     for (int r = 0; r < warp_rounds; ++r) {
-      const int rsyms = min(kRoundSyms, max(0, nsyms - r * kRoundSyms));
-      const int rwords = rsyms / 8;
-      int filled = 0;  // fewer than 32 bits (whole ranks) carry over between rounds
-      // One lookup: decodes up to kPalCap ranks; TAIL selects the careful
-      // variant that stops exactly at the chunk's last symbol.
-      auto lookup = [&](auto tail_tag) {
-        constexpr bool TAIL = decltype(tail_tag)::value;
-        const uint32_t idx = rd.hi >> 20;
-        uint32_t e = sm.lut[idx];
-        uint32_t cnt = (e >> 24) & 7u;
-        uint32_t len = e >> 28;
-        int rem = kPalCap;
-        if (TAIL) rem = nsyms - r * kRoundSyms - filled * 8 - (ab >> 2);
-        if (cnt == 0u || (TAIL && rem < kPalCap)) {
-          if (TAIL && rem <= 0) {  // chunk done (second lookup of a pair)
-            cnt = 0;
-            len = 0;
-            e = 0;
-          } else if (e & kLutRaw) {  // exponent outside the palette
-            if (MODE != kDecodePalette) {
-              const uint32_t pos = (uint32_t)(r * kRoundSyms + filled * 8 + (ab >> 2));
-              if (nx < kExcCap)
-                exc[nx++] = (pos << 8) | (e & 0xFFu);
-              else
-                overflow = true;
-            }
-            cnt = 1;
-            e = 0;
-          } else if (len == 0u) {  // no code starts here: corrupt stream
-            bad = true;
-            cnt = 1;
-            len = 1;
-            e = 0;
-          } else {  // last symbols of the chunk: one at a time
-            len = first_code_len(sm.canon, idx);
-            cnt = 1;
-            e &= 0xFu;
-          }
-        }
-        reader_consume(rd, len);
-        const uint32_t v = e & 0xFFFFFFu;
-        a_lo |= v << ab;
-        a_hi |= __funnelshift_l(v, 0u, (uint32_t)ab);
-        ab += 4 * (int)cnt;
-        if (ab >= 32 && filled < rwords) {
-          st[filled++] = a_lo;
-          a_lo = a_hi;
-          a_hi = 0;
-          ab -= 32;
-        }
-      };
-      if (r < fast_rounds) {
-        while (filled < rwords) {
-          reader_refill(rd, src, ng);
-          lookup(std::false_type());
-          // a pair's second lookup only while the round still needs words, so
-          // fewer than 32 bits are pending whenever ranks are appended
-          if (filled < rwords) lookup(std::false_type());
-        }
-      } else {
-        while (filled < rwords) {
-          reader_refill(rd, src, ng);
-          lookup(std::true_type());
-          if (filled < rwords) lookup(std::true_type());
-        }
+      pk.sp = st_addr;
+      if (MODE == kDecodeFull && r < my_rounds) {
+        // this round's sign+mantissa bytes into L2 while the round decodes
+        const uint8_t* sp8 = a.sm + c * cs + (int64_t)r * kRoundSyms;
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(sp8));
+      }
+      if (r < my_rounds - 1) {
+        // a round that ends inside the chunk: fill exactly kRoundWords words,
+        // the ranks past them (fewer than 32 bits) carry into the next round
+        while (pk.sp < st_addr + 4 * (kRoundWords - 1)) lookup_pair();
+        while (pk.sp < st_addr + 4 * kRoundWords) lookup_one(std::false_type());
+      } else if (r == my_rounds - 1) {
+        while (left4 >= kFullPair) lookup_pair();
+        while (left4 >= kFullOne) lookup_one(std::false_type());
+        while (left4 > 0) lookup_one(std::true_type());
       }
       __syncwarp();
 
-      // coalesced write-out: row slot rs of each of the 32 lanes
-#pragma unroll 1
-      for (int rs = 0; rs < kRoundSyms / 64; ++rs) {
-        // operands fetched for all 8 passes first so their latencies overlap
-        uint2 pre[8];
-        uint32_t okmask = 0;
-        const int w = lane & 7;
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const int j = 4 * p + (lane >> 3);
-          const int nj = __shfl_sync(0xffffffffu, nsyms, j);
-          const bool ok = (c0 + j < a.n_chunks) && (r * kRoundSyms + rs * 64 < nj);
-          okmask |= ok ? (1u << p) : 0u;
-          const int64_t row = (c0 + j) * rows_per_chunk + r * (kRoundSyms / 64) + rs;
-          pre[p] = make_uint2(0u, 0u);
-          int n_j = 0, kb_j = 0;
-          if (MODE == kDecodePalette) {
-            n_j = __shfl_sync(0xffffffffu, n0, j);
-            kb_j = __shfl_sync(0xffffffffu, kb0, j);
+      // ---- coalesced write-out of round r for the warp's 32 chunks ----
+      // rel0: this round's first symbol inside each chunk; a lane's part of
+      // chunk j is written when it lies inside the chunk and the matrix
+      const int64_t rel0 = (int64_t)r * kRoundSyms;
+      if (MODE == kDecodeExp) {
+        // 8 lanes per chunk, 16 symbols (two rank words) per lane
+        const int m = lane & 7, jq = lane >> 3;
+        const bool in_chunk = rel0 + 16 * m < cs;
+        uint8_t* base = static_cast<uint8_t*>(out) + c0 * cs + rel0 + 16 * m;
+#pragma unroll 4
+        for (int i = 0; i < 8; ++i) {
+          const int j = 4 * i + jq;
+          const int64_t o = (int64_t)j * cs;
+          if (in_chunk && o + rel0 + 16 * m < grp_syms_left) {
+            const uint32_t* sw = stage + j * kStageStride + 2 * m;
+            const uint2 lo = palette8(sw[0], p0, p1, p2, p3);
+            const uint2 hi = palette8(sw[1], p0, p1, p2, p3);
+            *reinterpret_cast<uint4*>(base + o) = make_uint4(lo.x, lo.y, hi.x, hi.y);
           }
-          if (ok) {
-            if (MODE == kDecodeFull) {
-              pre[p] = __ldg(reinterpret_cast<const uint2*>(a.sm + row * 64) + w);
-            } else if (MODE == kDecodePalette) {
-              // (n, kb) of the row from lane j's chunk start, no division
-              int n = n_j;
-              int kb = kb_j + r * (kRoundSyms / 64) + rs;
-              while (kb >= a.kb_per_row) {
-                kb -= a.kb_per_row;
-                ++n;
-              }
-              pre[p].x = (__ldg(a.esc_bits + (int64_t)kb * a.esc_nw + (n >> 5)) >> (n & 31)) & 1u;
+        }
+      } else if (MODE == kDecodeFull) {
+        // 16 lanes per chunk, 8 symbols (one rank word) per lane
+        const int m = lane & 15, jh = lane >> 4;
+        const bool in_chunk = rel0 + 8 * m < cs;
+        const int64_t sym0 = c0 * cs + rel0 + 8 * m;
+        const uint8_t* sbase = a.sm + sym0;
+        uint16_t* obase = static_cast<uint16_t*>(out) + sym0;
+        // eight loads in flight before their first use
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint2 sv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int64_t o = (int64_t)(16 * h + 2 * i + jh) * cs;
+            sv[i] = (in_chunk && o + rel0 + 8 * m < grp_syms_left)
+                        ? __ldg(reinterpret_cast<const uint2*>(sbase + o))
+                        : make_uint2(0u, 0u);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = 16 * h + 2 * i + jh;
+            const int64_t o = (int64_t)j * cs;
+            if (in_chunk && o + rel0 + 8 * m < grp_syms_left) {
+              const uint2 e = palette8(stage[j * kStageStride + m], p0, p1, p2, p3);
+              const uint2 lo = merge4(sv[i].x, e.x), hi = merge4(sv[i].y, e.y);
+              *reinterpret_cast<uint4*>(obase + o) = make_uint4(lo.x, lo.y, hi.x, hi.y);
             }
           }
         }
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const int j = 4 * p + (lane >> 3);
-          if (!((okmask >> p) & 1u)) continue;
-          const int64_t row = (c0 + j) * rows_per_chunk + r * (kRoundSyms / 64) + rs;
-          const uint32_t word = stage[j * kStageStride + rs * 8 + w];
-          if (MODE == kDecodePalette) {
-            reinterpret_cast<uint32_t*>(out)[row * 8 + w] = pre[p].x ? 0u : word;
-          } else {
-            const uint32_t e0 = palette4(word & 0xFFFFu, p0, p1, p2, p3);
-            const uint32_t e1 = palette4(word >> 16, p0, p1, p2, p3);
-            if (MODE == kDecodeExp) {
-              reinterpret_cast<uint2*>(out)[row * 8 + w] = make_uint2(e0, e1);
-            } else {
-              const uint2 lo = merge4(pre[p].x, e0), hi = merge4(pre[p].y, e1);
-              reinterpret_cast<uint4*>(out)[row * 8 + w] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      } else {
+        // 4 lanes per chunk, 32 symbols (four rank words, half a 64-weight
+        // row) per lane; escape rows are written as zeros
+        const int m = lane & 3, jr = lane >> 2;
+        const bool in_chunk = rel0 + 32 * m < cs;
+        const int n_me = row_n, kb_me = row_kb;
+        uint8_t* base = static_cast<uint8_t*>(out) + (c0 * cs + rel0) / 2 + 16 * m;
+#pragma unroll 2
+        for (int i = 0; i < 4; ++i) {
+          const int j = 8 * i + jr;
+          const int n_j = __shfl_sync(0xffffffffu, n_me, j);
+          const int kb_j = __shfl_sync(0xffffffffu, kb_me, j);
+          const int64_t o = (int64_t)j * cs;
+          if (in_chunk && o + rel0 + 32 * m < grp_syms_left) {
+            int n = n_j, kb = kb_j + (m >> 1);
+            while (kb >= a.kb_per_row) {
+              kb -= a.kb_per_row;
+              ++n;
             }
+            const bool esc =
+                (__ldg(a.esc_bits + (int64_t)kb * a.esc_nw + (n >> 5)) >> (n & 31)) & 1u;
+            const uint32_t* sw = stage + j * kStageStride + 4 * m;
+            uint4 v = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+            if (esc) v = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(base + o / 2) = v;
           }
         }
       }
       __syncwarp();
+      if (MODE == kDecodePalette) {  // the next round's first row
+        row_kb += kRoundSyms / 64;
+        while (row_kb >= a.kb_per_row) {
+          row_kb -= a.kb_per_row;
+          ++row_n;
+        }
+      }
 
       // exceptions of this round overwrite the placeholder the bulk write left
       if (MODE != kDecodePalette && nx > 0) {
         const int64_t base = c * cs;
-        const uint32_t lim = (uint32_t)((r + 1) * kRoundSyms);
+        const uint32_t lo = (uint32_t)(r * kRoundSyms), hi = lo + kRoundSyms;
         int keep = 0;
         for (int i = 0; i < nx; ++i) {
           const uint32_t x = exc[i];
           const uint32_t pos = x >> 8;
-          if (pos < lim) {
+          if (pos >= lo && pos < hi) {
             const int64_t o = base + pos;
             if (MODE == kDecodeExp) {
               static_cast<uint8_t*>(out)[o] = (uint8_t)(x & 0xFFu);
             } else {
               const uint32_t s = a.sm[o];
-              const uint32_t ex = x & 0xFFu;
               static_cast<uint16_t*>(out)[o] =
-                  (uint16_t)(((s & 0x80u) << 8) | (ex << 7) | (s & 0x7Fu));
+                  (uint16_t)(((s & 0x80u) << 8) | ((x & 0xFFu) << 7) | (s & 0x7Fu));
             }
           } else {
             exc[keep++] = x;
@@ -346,11 +415,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // a lane whose exception list overflowed replays its chunk symbol by symbol
     if (MODE != kDecodePalette && overflow) {
-      Reader sr;
-      reader_init(sr, src, ng, start);
+      Bits sb;
+      bits_init(sb, words, start);
       const int64_t base = c * cs;
       for (int i = 0; i < nsyms; ++i) {
-        const uint32_t ex = slow_symbol(sr, src, ng, sm.canon);
+        uint32_t len;
+        const uint32_t ex = canon_symbol(sm.canon, bits_peek(sb) >> 20, &len);
+        sb.q += len;
+        bits_slide(sb, words);
         if (MODE == kDecodeExp) {
           static_cast<uint8_t*>(out)[base + i] = (uint8_t)ex;
         } else {
@@ -360,40 +432,83 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-    if (live && (bad || reader_consumed(rd, start) != end - start))
-      atomicOr(a.status, kStatusBadChunk);
+    if (live && (bad || bits_pos(b) != end)) atomicOr(a.status, kStatusBadChunk);
     __syncwarp();
   }
 }
 
+template <typename F>
+cudaError_t set_attrs(F* f, size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the smallest shared-memory split that holds the CTA leaves L1 the rest
+  const int pct = (int)((100 * (smem + 1024) + 228 * 1024 - 1) / (228 * 1024));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
+  return e;
+}
+
 }  // namespace
 
-int decode_ctas_needed(int64_t n_chunks) {
+// Launch shape: one CTA per SM (capped at `sms`) with W warps, a warp decoding
+// 32 chunks per pass.  A pass takes about as long as the SM's warps share its
+// issue slots, so W is chosen in [16, 32] to minimise passes x W (the last
+// pass nearly full); a problem too small to give every SM 16 warps spreads
+// over more SMs with fewer warps instead.
+void decode_launch_shape(int64_t n_chunks, int sms, int* ctas, int* warps) {
   const int64_t groups = (n_chunks + 31) / 32;
-  return (int)((groups + kWarps - 1) / kWarps);
+  if (sms < 1) sms = 1;
+  if (groups <= (int64_t)sms * kMinWarps) {
+    const int64_t w = groups <= sms ? 1 : (groups + sms - 1) / sms;
+    *warps = (int)w;
+    *ctas = (int)((groups + w - 1) / w);
+    return;
+  }
+  int best_w = kMaxWarps;
+  int64_t best_cost = -1;
+  for (int w = kMaxWarps; w >= kMinWarps; --w) {
+    const int64_t per = (int64_t)sms * w;
+    const int64_t cost = (groups + per - 1) / per * w;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_w = w;
+    }
+  }
+  *warps = best_w;
+  *ctas = sms;
+}
+
+int decode_ctas_needed(int64_t n_chunks) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int ctas = 0, warps = 0;
+  decode_launch_shape(n_chunks, sms, &ctas, &warps);
+  return ctas;
 }
 
 cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cudaStream_t s) {
-  const int need = decode_ctas_needed(a.n_chunks);
-  const int grid = (ctas > 0 && ctas < need) ? ctas : need;
-  if (grid <= 0) return cudaSuccess;
-  const size_t smem = sizeof(Smem);
-  cudaError_t e = cudaSuccess;
+  if (a.n_chunks <= 0) return cudaSuccess;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (ctas > 0 && ctas < sms) sms = ctas;  // an SM budget (decoder/GEMM split)
+  int grid = 0, warps = 0;
+  decode_launch_shape(a.n_chunks, sms, &grid, &warps);
+  const size_t smem = smem_bytes(warps);
+  const dim3 block(32 * warps);
   switch (mode) {
     case kDecodeExp:
-      e = cudaFuncSetAttribute(decode_kernel<kDecodeExp>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) decode_kernel<kDecodeExp><<<grid, kThreads, smem, s>>>(a, out);
+      e = set_attrs(decode_kernel<kDecodeExp>, smem);
+      if (e == cudaSuccess) decode_kernel<kDecodeExp><<<grid, block, smem, s>>>(a, out);
       break;
     case kDecodeFull:
-      e = cudaFuncSetAttribute(decode_kernel<kDecodeFull>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) decode_kernel<kDecodeFull><<<grid, kThreads, smem, s>>>(a, out);
+      e = set_attrs(decode_kernel<kDecodeFull>, smem);
+      if (e == cudaSuccess) decode_kernel<kDecodeFull><<<grid, block, smem, s>>>(a, out);
       break;
     case kDecodePalette:
-      e = cudaFuncSetAttribute(decode_kernel<kDecodePalette>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) decode_kernel<kDecodePalette><<<grid, kThreads, smem, s>>>(a, out);
+      e = set_attrs(decode_kernel<kDecodePalette>, smem);
+      if (e == cudaSuccess) decode_kernel<kDecodePalette><<<grid, block, smem, s>>>(a, out);
       break;
     default:
       return cudaErrorInvalidValue;

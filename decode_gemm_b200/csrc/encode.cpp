@@ -138,9 +138,12 @@ bool build_decode_tables(const uint8_t code_len[256], const uint8_t palette[16],
   out->lut.assign(kLutSize, 0);
   for (int v = 0; v < kLutSize; ++v) {
     const int s0 = first_sym[v];
-    if (s0 < 0) continue;  // no code starts this window: entry 0 (invalid)
-    if (rank[s0] < 0) {    // an exponent outside the palette: one raw symbol
-      out->lut[v] = (uint32_t)s0 | kLutRaw | ((uint32_t)first_len[v] << 28);
+    if (s0 < 0) {  // no code starts this window: one placeholder, one bit
+      out->lut[v] = 1u | (4u << 4) | kLutSpecial | kLutInvalid;
+      continue;
+    }
+    if (rank[s0] < 0) {  // an exponent outside the palette: one placeholder
+      out->lut[v] = (uint32_t)first_len[v] | (4u << 4) | kLutSpecial;
       continue;
     }
     uint32_t vals = 0, cnt = 0, pos = 0;
@@ -153,7 +156,7 @@ bool build_decode_tables(const uint8_t code_len[256], const uint8_t palette[16],
       cnt++;
       pos += l;
     }
-    out->lut[v] = vals | (cnt << 24) | (pos << 28);
+    out->lut[v] = pos | ((4 * cnt) << 4) | (vals << 12);
   }
   // canonical tables
   int count[kLutBits + 2] = {0};

@@ -292,7 +292,7 @@ uw_status uw_mlp_tune_split(const uw_mlp_layer* layers, int32_t n_layers, const 
   // (decoder CTAs, GEMM CTAs): no split, then the decoder on a few SMs
   std::vector<std::pair<int, int>> splits = {{0, 0}};
   for (int d : {4, 8, 16, 24})
-    if (d < sms) splits.push_back({2 * d, sms - d});  // 2 decoder CTAs fit on an SM
+    if (d < sms) splits.push_back({d, sms - d});  // one decoder CTA per SM
   cudaStream_t ms = static_cast<cudaStream_t>(stream);
   cudaEvent_t a = nullptr, b = nullptr;
   if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return UW_ERR_CUDA;

@@ -17,15 +17,19 @@ constexpr int kLutSize = 1 << kLutBits;
 // Decode-table entry (one u32 per 12-bit window of the stream).  The table
 // decodes to 4-bit palette ranks; all three preprocessing outputs derive from
 // them (exponent = palette[rank]).
-//   bits  0..23  ranks of the codes that fit in the window, first one lowest,
-//                at most kPalCap of them, stopping before any exponent that is
-//                not in the palette
-//   bits 24..26  number of ranks (0: see bit 27)
-//   bit  27      raw: the window starts with the code of an exponent outside the
-//                palette; bits 0..7 hold that exponent (one symbol)
-//   bits 28..31  stream bits consumed (0: the window starts with no code)
-constexpr int kPalCap = 6;
-constexpr uint32_t kLutRaw = 1u << 27;
+//   bits  0..3   stream bits the entry consumes (1..12)
+//   bits  4..8   4 x the number of ranks it yields (4..4*kPalCap)
+//   bit   9      special: the window starts with the code of an exponent outside
+//                the palette ("raw"), or with no code at all (bit 10 set too);
+//                the entry then yields a single rank 0 placeholder and consumes
+//                the raw code's length (1 bit for a window with no code)
+//   bit   10     no code starts the window (corrupt stream)
+//   bits 12..31  the ranks of the codes that fit in the window, first one
+//                lowest, at most kPalCap of them, stopping before any exponent
+//                that is not in the palette
+constexpr int kPalCap = 5;
+constexpr uint32_t kLutSpecial = 1u << 9;
+constexpr uint32_t kLutInvalid = 1u << 10;
 
 // Canonical-code tables for one-symbol-at-a-time decoding (chunk tails, slow
 // path): limit[l] = first 12-bit window whose first code is longer than l;

@@ -9,9 +9,16 @@ namespace uw {
 
 enum DecodeMode { kDecodeExp = 0, kDecodeFull = 1, kDecodePalette = 2 };
 
+// Zero words that follow the Huffman stream in device memory: a lane decoding
+// a chunk reads at most 12 bits per symbol past the chunk's start plus a
+// four-word window, so every read of a chunk whose start lies inside the
+// stream stays inside the padded buffer.
+inline int64_t stream_pad_words(int64_t chunk_syms) { return 3 * chunk_syms / 8 + 8; }
+
 // Everything a decode/transcode launch reads, as device pointers.
 struct DecodeArgs {
-  const uint32_t* words;      // Huffman stream, n_words (a multiple of 4) words
+  const uint32_t* words;      // Huffman stream: n_words (a multiple of 4) words,
+                              // then stream_pad_words(chunk_syms) zero words
   const uint32_t* chunk_off;  // n_chunks + 1 bit offsets
   const uint32_t* lut;        // 4096-entry rank table (see DecodeTables)
   const uint32_t* canon;      // canonical-code tables (kCanonWords words)
@@ -28,10 +35,13 @@ struct DecodeArgs {
 };
 
 // Decode/transcode every chunk into `out` (layout per mode: BF16 [N*K],
-// exponent bytes [N*K], packed nibbles [N*K/2]).  ctas <= 0: one CTA per 256
-// chunks.  Returns the launch error.
+// exponent bytes [N*K], packed nibbles [N*K/2]).  ctas > 0 caps the SMs the
+// launch may use (one CTA per SM); ctas <= 0: all of them.  Returns the
+// launch error.
 cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cudaStream_t s);
 int decode_ctas_needed(int64_t n_chunks);
+// CTAs and warps per CTA of a decode over n_chunks chunks on `sms` SMs.
+void decode_launch_shape(int64_t n_chunks, int sms, int* ctas, int* warps);
 
 // Device status bits.
 constexpr uint32_t kStatusBadChunk = 1u;

@@ -135,7 +135,7 @@ typedef struct uw_gemm_config {
   int32_t tile_n;        /* tokens per MMA tile: 16..256, multiple of 16 (0=auto)  */
   int32_t stages;        /* shared-memory ring depth, even, 2..12 (0 = auto)       */
   int32_t gemm_ctas;     /* persistent GEMM CTAs (0 = one per SM)                   */
-  int32_t decode_ctas;   /* CTAs of the preprocessing kernel (0 = auto)            */
+  int32_t decode_ctas;   /* SMs (one CTA each) of the preprocessing kernel (0 = all) */
   int32_t reserved[3];
 } uw_gemm_config;
 
@@ -291,8 +291,8 @@ typedef struct uw_mlp_opts {
                            ("hard": 1-3) are preprocessed on side_stream one hard
                            projection ahead, into two alternating workspace slots,
                            while the main stream runs the GEMMs                     */
-  int32_t decode_ctas;  /* SM split, decoder share: CTAs of each side-stream
-                           preprocessing kernel (0 = as many as it needs)            */
+  int32_t decode_ctas;  /* SM split, decoder share: SMs (one CTA each) of each
+                           side-stream preprocessing kernel (0 = all of them)        */
   int32_t gemm_ctas;    /* SM split, GEMM share: CTAs of each GEMM while the stack
                            runs (0 = one per SM); a profile's own value wins         */
   int32_t reserved;
