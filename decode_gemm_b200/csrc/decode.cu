@@ -70,18 +70,6 @@ size_t smem_bytes(int warps) {
   return sizeof(SmemHead) + (size_t)warps * kWarpSmemWords * 4;
 }
 
-__device__ __forceinline__ void st_shared_if(uint32_t addr, uint32_t v, bool p) {
-  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.shared.u32 [%0], %1;\n\t}"
-               :: "r"(addr), "r"(v), "r"((uint32_t)p) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_global_if(const uint32_t* ptr, uint32_t old, bool p) {
-  uint32_t v = old;
-  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q ld.global.nc.u32 %0, [%1];\n\t}"
-      : "+r"(v) : "l"(ptr), "r"((uint32_t)p));
-  return v;
-}
-
 // Four consecutive stream words; bit q (MSB first) of w0 is the next bit.
 struct Bits {
   uint32_t w0, w1, w2, w3;
@@ -104,18 +92,22 @@ __device__ __forceinline__ uint32_t bits_peek(const Bits& b) {
   return __funnelshift_l(b.w1, b.w0, b.q);
 }
 
-// Slide the window by one word once q has passed 32 (q < 64).  Reads stay in
-// the padded stream buffer: a lane never reads more than 12 bits per symbol
-// past its chunk's start, plus the window.
+// Slide the window by one word once q has passed 32 (q < 64): predicated
+// moves and load, no branch.  Reads stay in the padded stream buffer: a lane
+// never reads more than 12 bits per symbol past its chunk's start, plus the
+// window.
 __device__ __forceinline__ void bits_slide(Bits& b, const uint32_t* words) {
-  const bool s = b.q >= 32u;
-  const uint32_t nw = ld_global_if(words + b.nxt, b.w3, s);
-  b.w0 = s ? b.w1 : b.w0;
-  b.w1 = s ? b.w2 : b.w1;
-  b.w2 = s ? b.w3 : b.w2;
-  b.w3 = nw;
-  b.nxt += s ? 1u : 0u;
-  b.q &= 31u;
+  const uint32_t* p = words + b.nxt;
+  asm("{\n\t.reg .pred s;\n\t"
+      "setp.gt.u32 s, %4, 31;\n\t"
+      "@s mov.b32 %0, %1;\n\t"
+      "@s mov.b32 %1, %2;\n\t"
+      "@s mov.b32 %2, %3;\n\t"
+      "@s ld.global.nc.u32 %3, [%6];\n\t"
+      "@s add.u32 %5, %5, 1;\n\t"
+      "and.b32 %4, %4, 31;\n\t}"
+      : "+r"(b.w0), "+r"(b.w1), "+r"(b.w2), "+r"(b.w3), "+r"(b.q), "+r"(b.nxt)
+      : "l"(p));
 }
 
 // Stream bit position of the next bit.
@@ -145,17 +137,23 @@ struct Packer {
   uint32_t sp;
 };
 
-__device__ __forceinline__ void pack(Packer& pk, uint32_t e) {
-  const uint32_t v = e >> 12;
-  const uint32_t c4 = (e >> 4) & 31u;
-  const uint32_t lo = pk.a_lo | (v << pk.ab);
-  const uint32_t hi = __funnelshift_l(v, 0u, pk.ab);  // bits of v past bit 31
-  const uint32_t ab = pk.ab + c4;
-  const bool full = ab >= 32u;
-  st_shared_if(pk.sp, lo, full);
-  pk.sp += full ? 4u : 0u;
-  pk.a_lo = full ? hi : lo;
-  pk.ab = ab & 31u;
+// Append the entry's ranks (c4 = 4 x their count); a completed word is stored
+// with a predicated shared store.
+__device__ __forceinline__ void pack(Packer& pk, uint32_t e, uint32_t c4) {
+  asm("{\n\t.reg .pred f;\n\t.reg .b32 v, lo, hi;\n\t"
+      "shr.b32 v, %3, 12;\n\t"
+      "shl.b32 lo, v, %1;\n\t"
+      "or.b32 lo, lo, %0;\n\t"
+      "shf.l.wrap.b32 hi, v, 0, %1;\n\t"
+      "add.u32 %1, %1, %4;\n\t"
+      "setp.gt.u32 f, %1, 31;\n\t"
+      "@f st.shared.u32 [%2], lo;\n\t"
+      "@f add.u32 %2, %2, 4;\n\t"
+      "selp.b32 %0, hi, lo, f;\n\t"
+      "and.b32 %1, %1, 31;\n\t}"
+      : "+r"(pk.a_lo), "+r"(pk.ab), "+r"(pk.sp)
+      : "r"(e), "r"(c4)
+      : "memory");
 }
 
 template <int MODE>
@@ -262,9 +260,10 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         if (e2 & kLutSpecial) special(e2, win2, left4 - (int)((e1 >> 4) & 31u));
       }
       b.q = q1 + (e2 & 15u);
-      left4 -= (int)(((e1 >> 4) & 31u) + ((e2 >> 4) & 31u));
-      pack(pk, e1);
-      pack(pk, e2);
+      const uint32_t c1 = (e1 >> 4) & 31u, c2 = (e2 >> 4) & 31u;
+      left4 -= (int)(c1 + c2);
+      pack(pk, e1, c1);
+      pack(pk, e2, c2);
       bits_slide(b, words);
     };
     // One lookup; TAIL: fewer than kPalCap symbols may be left, so an entry
@@ -277,8 +276,9 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         e = (e & 0xF000u) | (4u << 4) | first_code_len(sm.canon, win >> 20);
       if (e & kLutSpecial) special(e, win, left4);
       b.q += e & 15u;
-      left4 -= (int)((e >> 4) & 31u);
-      pack(pk, e);
+      const uint32_t c = (e >> 4) & 31u;
+      left4 -= (int)c;
+      pack(pk, e, c);
       bits_slide(b, words);
     };
 
