@@ -64,6 +64,7 @@ GemmArgs base_gemm_args(const uw_handle_s* h) {
   std::memcpy(a.palette, h->palette, 16);
   a.sm_count = h->sm_count;
   a.status = h->d_status;
+  a.sync = h->d_sync;
   return a;
 }
 
@@ -312,6 +313,7 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   const size_t o_eoff = place((size_t)(f->n_esc_groups + 1) * 4);
   const size_t o_eexp = place((size_t)std::max<int64_t>(f->n_esc_rows, 1) * kRow);
   const size_t o_stat = place(256);
+  const size_t o_sync = place(kGemmSyncWords * 4);
   const size_t o_pidx = o.prepare_direct ? place(T / 2) : 0;
   cudaError_t e = cudaMalloc(&h->d_block, off);
   if (e != cudaSuccess) {
@@ -328,6 +330,7 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   h->d_esc_off = reinterpret_cast<uint32_t*>(base + o_eoff);
   h->d_esc_exp = base + o_eexp;
   h->d_status = reinterpret_cast<uint32_t*>(base + o_stat);
+  h->d_sync = reinterpret_cast<uint32_t*>(base + o_sync);
   h->d_pal_idx = o.prepare_direct ? base + o_pidx : nullptr;
   cudaStream_t s = h->stream;
   const Part parts[] = {
@@ -348,6 +351,7 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   if (e == cudaSuccess)
     e = cudaMemsetAsync(h->d_words + f->n_words, 0, (size_t)pad_words * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->d_status, 0, 256, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->d_sync, 0, kGemmSyncWords * 4, s);
   if (e == cudaSuccess && h->d_pal_idx) {
     // load-time transcode: the resident palette form of pipeline 4
     DecodeArgs a = decode_args(h);

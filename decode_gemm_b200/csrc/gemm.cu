@@ -22,8 +22,13 @@
 //     per 4 weights; the escape decision is taken once per 64-weight row from a
 //     16-byte bitmap staged with the tile.
 //   * Persistent CTAs split the flattened (output tile, K block) space evenly
-//     (stream-K); tiles shared by two CTAs are finished by a small fix-up kernel
-//     that adds the partial sums in K order, so results are deterministic.
+//     (stream-K).  A tile shared by several CTAs is finished inside the kernel
+//     by the CTA holding its first K block: that tile is the last it works on,
+//     so by then the others have usually handed over their partial sums
+//     (written to the workspace, then a ready flag tagged with the launch's
+//     epoch); it adds them in K order, so results are deterministic.  The
+//     epoch lives on the device (the last CTA to exit advances it), so stale
+//     flags from earlier launches, aborted ones or graph replays never match.
 //   * Every mbarrier wait is bounded in wall time; on expiry the kernel records
 //     a timeout in the status word, drains its MMAs and copies, frees TMEM and
 //     returns.
@@ -75,6 +80,7 @@ struct GemmParams {
   void* Y;
   float* partials;
   uint32_t* status;
+  uint32_t* sync;     // [0] epoch, [1] exited CTAs, [2 + cta] ready flags
   int64_t M, N, K;
   int64_t units;      // output tiles * K blocks
   int32_t tile_n, stages, wslots, n_mma, NT, MT, KB, esc_nwp, out_f32, tmem_cols;
@@ -129,12 +135,54 @@ __device__ __forceinline__ void set_abort(volatile int* abort, uint32_t* status)
   }
 }
 
+// The four epilogue warps synchronise among themselves on named barrier 1;
+// the OR-reduction gives all 128 threads the same decision.
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("barrier.cta.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *flag == tag, giving up after limit_ns or when *abort is raised.
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t tag, volatile int* abort,
+                                          uint64_t limit_ns) {
+  if (ld_acquire(flag) == tag) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(64);
+    if (ld_acquire(flag) == tag) return true;
+    if (*abort || globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(threads_for(MODE), 1)
     gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 1024-byte aligned, by an offset into the shared array (the accesses stay
+  // shared-window loads and stores)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const StageLayout L = stage_layout(MODE, p.tile_n);
   const int S = p.stages;
   const int WS = MODE == kGemmBf16 ? 0 : p.wslots;
@@ -148,6 +196,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             b_tfull = 2 * S + 2 * WS, b_tempty = b_tfull + 2, b_drain = b_tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + b_drain + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* tag_slot = tmem_slot + 2;  // this launch's hand-off tag (epoch + 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -168,6 +217,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       mbar_init(bar(b_drain + a), 1);
     }
     *abort = 0;
+    *tag_slot = __ldcg(p.sync) + 1u;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -355,14 +405,16 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     // ------------------------------------------------------------ epilogue --
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
+    const bool leader = warp == kEpiWarp0 && lane == 0;
+    const uint32_t tag = *tag_slot;
+    const int64_t part_stride = (int64_t)p.tile_n * kBM;
     int seg = 0;
     int64_t qa = 0;  // index (among this CTA's units) of the segment's first unit
     for (int64_t u = u0; u < u1; ++seg) {
       const int64_t t = u / KB;
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
-      const bool full = kb0 == 0 && kb1 == KB;
-      const int slot = (u == u0) ? 0 : 1;
+      const bool split = !(kb0 == 0 && kb1 == KB);
       const int acc = seg & 1;
       const uint32_t acc_phase = (uint32_t)(seg >> 1) & 1u;
       // every lane observes the accumulator barrier before reading TMEM; the
@@ -370,8 +422,26 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const bool got =
           mbar_wait_bounded(bar(b_tfull + acc), acc_phase, abort, p.wait_ns, kEpiSleepNs);
       if (!got) set_abort(abort, p.status);
-      if (__any_sync(0xffffffffu, !got)) break;
+      if (epi_any(!got)) break;
       tc_fence_after();
+      // a split tile's owner (the CTA with its first K block) collects the
+      // partial sums of CTAs blockIdx.x+1 .. last
+      bool owner = false;
+      int64_t last = 0;
+      if (split) {
+        const int64_t ua = t * KB;
+        owner = unit_owner(ua, p.units, G) == (int64_t)blockIdx.x;
+        last = unit_owner(ua + KB - 1, p.units, G);
+        if (owner) {
+          bool ok = true;
+          if (leader) {
+            for (int64_t q = blockIdx.x + 1; q <= last && ok; ++q)
+              ok = wait_flag(p.sync + 2 + q, tag, abort, p.wait_ns);
+            if (!ok) set_abort(abort, p.status);
+          }
+          if (epi_any(!ok)) break;
+        }
+      }
       const int64_t nt = t / p.MT, mt = t - nt * p.MT;
       const int64_t n = nt * kBM + row;
       const int64_t m0 = mt * p.tile_n;
@@ -382,30 +452,53 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const uint32_t lanebase = (uint32_t)(quad * 32) << 16;
       const uint32_t t0 = tmem_base + lanebase + (uint32_t)((acc * NM + 0) * p.tile_n);
       const uint32_t t1 = tmem_base + lanebase + (uint32_t)((acc * NM + 1) * p.tile_n);
-      float* part = p.partials + ((int64_t)blockIdx.x * 2 + slot) * (int64_t)p.tile_n * kBM;
+      float* part = p.partials + (int64_t)blockIdx.x * part_stride;
       for (int c = 0; c < cols; c += 16) {
         uint32_t r0[16], r1[16];
         if (has0) tmem_ld16(t0 + (uint32_t)c, r0);
         if (has1) tmem_ld16(t1 + (uint32_t)c, r1);
         tmem_ld_wait();
+        float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          if (c + j < cols) {
-            float v = has0 ? __uint_as_float(r0[j]) : 0.f;
-            if (has1) v += __uint_as_float(r1[j]);
-            if (full) {
-              if (n < p.N) {
-                const int64_t o = (m0 + c + j) * p.N + n;
-                if (p.out_f32)
-                  static_cast<float*>(p.Y)[o] = v;
-                else
-                  static_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(v);
-              }
-            } else {
-              part[(int64_t)(c + j) * kBM + row] = v;
+          v[j] = has0 ? __uint_as_float(r0[j]) : 0.f;
+          if (has1) v[j] += __uint_as_float(r1[j]);
+        }
+        if (split && !owner) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c + j < cols) part[(int64_t)(c + j) * kBM + row] = v[j];
+          continue;
+        }
+        if (split) {
+          // the other CTAs' sums, in K order; a contributor's 16 loads are all
+          // in flight before the first add
+          for (int64_t q = blockIdx.x + 1; q <= last; ++q) {
+            const float* src = p.partials + q * part_stride + (int64_t)c * kBM + row;
+            float pv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pv[j] = c + j < cols ? __ldcg(src + j * kBM) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += pv[j];
+          }
+        }
+        if (n < p.N) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (c + j < cols) {
+              const int64_t o = (m0 + c + j) * p.N + n;
+              if (p.out_f32)
+                static_cast<float*>(p.Y)[o] = v[j];
+              else
+                static_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(v[j]);
             }
           }
         }
+      }
+      if (split && !owner) {  // hand the partial sum over
+        __threadfence();
+        epi_sync();
+        if (leader) st_release(p.sync + 2 + blockIdx.x, tag);
       }
       tc_fence_before();
       __syncwarp();
@@ -465,27 +558,31 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           else
             v4[i] = *reinterpret_cast<const uint32_t*>(st + L.w1 + r * 32 + c * 4);
         }
+        // thread rows r_i = gt/8 + 16 i: row r_i's escape bit is bit gt/8 + 16 (i & 1)
+        // of bitmap word i / 2; most warps see no escape row in a tile and skip
+        // the per-row test
         uint32_t eb[4] = {0u, 0u, 0u, 0u};
+        uint32_t emask = 0;
         if (MODE == kGemmPalette) {
           const uint4 w4 = *reinterpret_cast<const uint4*>(st + L.ebits);
           eb[0] = w4.x;
           eb[1] = w4.y;
           eb[2] = w4.z;
           eb[3] = w4.w;
+          const uint32_t sh = (uint32_t)gt >> 3;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) emask |= ((eb[i >> 1] >> (sh + 16 * (i & 1))) & 1u) << i;
         }
+        const bool any_esc = MODE == kGemmPalette && __any_sync(0xffffffffu, emask != 0);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int c8 = gt + 128 * i;
           const int r = c8 >> 3, c = c8 & 7;
           if (MODE == kGemmPalette) {
-            e8[i].x = palette4(v4[i] & 0xFFFFu, p.palette[0], p.palette[1], p.palette[2],
-                               p.palette[3]);
-            e8[i].y = palette4(v4[i] >> 16, p.palette[0], p.palette[1], p.palette[2],
-                               p.palette[3]);
-            // row r = 32*(i/2) + ... : its escape bit, decided once for the row
-            const uint32_t word = eb[r >> 5];
-            if ((word >> (r & 31)) & 1u) {
-              uint32_t slot = (uint32_t)__popc(word & ((1u << (r & 31)) - 1u));
+            e8[i] = palette8(v4[i], p.palette[0], p.palette[1], p.palette[2], p.palette[3]);
+            if (any_esc && ((emask >> i) & 1u)) {
+              // an escape row: its verbatim exponents, slot = escape rows before it
+              uint32_t slot = (uint32_t)__popc(eb[r >> 5] & ((1u << (r & 31)) - 1u));
               for (int w = 0; w < (r >> 5); ++w) slot += (uint32_t)__popc(eb[w]);
               if (slot < (uint32_t)kEscCap) {
                 e8[i] = *reinterpret_cast<const uint2*>(st + L.erows + slot * 64 + c * 8);
@@ -518,55 +615,14 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
   }
-}
-
-// Finish tiles whose K range was split between CTAs: add the partial sums in
-// K order (CTA order) and write Y.  One block per output tile, one thread per
-// W row of the tile; the contributing CTAs' slots are resolved once per block.
-constexpr int kMaxSplit = 256;  // a tile spans at most gridDim CTAs (<= SM count)
-constexpr int kFixCols = 16;    // output columns (tokens) per fix-up block
-
-__global__ void __launch_bounds__(128) splitk_fixup_kernel(const __grid_constant__ GemmParams p,
-                                                           int64_t G) {
-  __shared__ int64_t base[kMaxSplit];
-  const int64_t t = blockIdx.x;
-  const int64_t ua = t * p.KB, ub = ua + p.KB - 1;
-  const int64_t i0 = unit_owner(ua, p.units, G), i1 = unit_owner(ub, p.units, G);
-  if (i0 == i1) return;  // written by the GEMM itself
-  const int nsplit = (int)(i1 - i0 + 1);
-  for (int q = threadIdx.x; q < nsplit && q < kMaxSplit; q += blockDim.x) {
-    const int64_t i = i0 + q;
-    const int64_t s = unit_begin(i, p.units, G), e = unit_begin(i + 1, p.units, G);
-    // first segment of CTA i lives in slot 0, its last in slot 1
-    base[q] = (s == e) ? -1 : (i * 2 + ((s / p.KB == t) ? 0 : 1)) * (int64_t)p.tile_n * kBM;
-  }
-  __syncthreads();
-  const int row = threadIdx.x;
-  const int64_t nt = t / p.MT, mt = t - nt * p.MT;
-  const int64_t n = nt * kBM + row;
-  const int64_t m0 = mt * p.tile_n;
-  const int cols = (int)imin64(p.tile_n, p.M - m0);
-  const int j0 = blockIdx.y * kFixCols;  // this block's columns (tokens)
-  if (n >= p.N || j0 >= cols) return;
-  const int ns = nsplit < kMaxSplit ? nsplit : kMaxSplit;
-  float acc[kFixCols];
-#pragma unroll
-  for (int jj = 0; jj < kFixCols; ++jj) acc[jj] = 0.f;
-  for (int q = 0; q < ns; ++q) {
-    if (base[q] < 0) continue;
-    const float* src = p.partials + base[q] + (int64_t)j0 * kBM + row;
-#pragma unroll
-    for (int jj = 0; jj < kFixCols; ++jj)  // independent loads in flight
-      if (j0 + jj < cols) acc[jj] += src[(int64_t)jj * kBM];
-  }
-#pragma unroll
-  for (int jj = 0; jj < kFixCols; ++jj) {
-    if (j0 + jj >= cols) break;
-    const int64_t o = (m0 + j0 + jj) * p.N + n;
-    if (p.out_f32)
-      static_cast<float*>(p.Y)[o] = acc[jj];
-    else
-      static_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(acc[jj]);
+  // the last CTA to leave advances the epoch for the next launch
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sync + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sync + 1, 0u);
+      __threadfence();
+      atomicAdd(p.sync, 1u);
+    }
   }
 }
 
@@ -676,12 +732,15 @@ bool gemm_resolve(GemmArgs* a) {
   const int64_t units = NT * MT * (a->K / kBK);
   int ctas = a->ctas > 0 ? a->ctas : a->sm_count;
   if ((int64_t)ctas > units) ctas = (int)units;
+  if (ctas > kGemmMaxCtas) ctas = kGemmMaxCtas;
   a->ctas = ctas;
   return true;
 }
 
+// One partial-sum tile per CTA: a CTA hands over at most one (the split tile
+// its range starts in, when it does not hold that tile's first K block).
 size_t gemm_partials_bytes(const GemmArgs& a) {
-  return (size_t)a.ctas * 2 * (size_t)a.tile_n * kBM * sizeof(float);
+  return (size_t)a.ctas * (size_t)a.tile_n * kBM * sizeof(float);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* hooks) {
@@ -712,6 +771,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.Y = a.Y;
   p.partials = a.partials;
   p.status = a.status;
+  p.sync = a.sync;
+  if (!p.sync) return cudaErrorInvalidValue;
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
@@ -737,7 +798,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   auto end = [&](int slot) {
     if (hooks && hooks->end) hooks->end(hooks->ctx, slot);
   };
-  // kinds: 3 bf16, 4 exponent, 5 palette GEMM; 6 fix-up
+  // kinds: 3 bf16, 4 exponent, 5 palette GEMM
   const int slot = begin(3 + a.mode);
   switch (a.mode) {
     case kGemmBf16:
@@ -756,16 +817,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
       return cudaErrorInvalidValue;
   }
   end(slot);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // tiles split between CTAs get their sum here (only when some tile is split)
-  if (p.units % G != 0 || (p.units / G) % KB != 0) {
-    const int fs = begin(6);
-    const dim3 fgrid((unsigned)(p.NT * p.MT), (unsigned)((a.tile_n + kFixCols - 1) / kFixCols));
-    splitk_fixup_kernel<<<fgrid, kBM, 0, s>>>(p, G);
-    end(fs);
-    e = cudaGetLastError();
-  }
-  return e;
+  return cudaGetLastError();
 }
 
 }  // namespace uw

@@ -33,6 +33,7 @@ struct uw_handle_s {
   uint32_t* d_esc_off = nullptr;
   uint8_t* d_esc_exp = nullptr;
   uint32_t* d_status = nullptr;
+  uint32_t* d_sync = nullptr;    // GEMM split-K hand-off (kGemmSyncWords, zeroed at upload)
   uint8_t* d_pal_idx = nullptr;  // resident palette indices (pipeline 4), may be null
 
   // workspace for pipelines 1-3 and split-K partial sums

@@ -8,7 +8,7 @@
 // array compiled into the library, so a call allocates nothing.
 //
 // Cost of the convenience: every GPU on which the library's device code is
-// loaded holds the array (kScratchFloats floats, 10 MiB) until the process
+// loaded holds the array (kScratchFloats floats, 5 MiB) until the process
 // exits, and all calls share it.
 #include <cuda_runtime.h>
 
@@ -19,10 +19,10 @@
 
 namespace {
 
-// Split-K partial sums: up to kMaxCtas CTAs x 2 segments x 64 tokens x 128 rows.
+// Split-K partial sums: up to kMaxCtas CTAs x 64 tokens x 128 rows.
 constexpr int kMaxCtas = 160;
 constexpr int kMaxM = 64;
-constexpr size_t kScratchFloats = (size_t)kMaxCtas * 2 * kMaxM * 128;
+constexpr size_t kScratchFloats = (size_t)kMaxCtas * kMaxM * 128;
 
 static __device__ __align__(256) float g_gemm_scratch[kScratchFloats];
 
@@ -81,11 +81,13 @@ uw_status uw_gemm_palette_noalloc(uw_handle_t h, const uint16_t* X_dev, void* Y_
   a.out_f32 = out_f32 ? 1 : 0;
   a.sm_count = h->sm_count < kMaxCtas ? h->sm_count : kMaxCtas;
   a.status = h->d_status;
+  a.sync = h->d_sync;
   if (!uw::gemm_resolve(&a)) return UW_ERR_UNSUPPORTED;
   a.partials_bytes = uw::gemm_partials_bytes(a);
   if (a.partials_bytes > kScratchFloats * sizeof(float)) return UW_ERR_SHAPE;
-  // Nothing in the scratch has to start at zero: every partial sum the
-  // fix-up reads is written earlier in the same call.
+  // Nothing in the scratch has to start at zero: every partial sum a tile's
+  // owner reads is written earlier in the same call (the hand-off flags live
+  // in the handle's own zeroed block).
   a.partials = scratch;
   const cudaError_t e = uw::launch_gemm(a, h->stream, nullptr);
   return e == cudaSuccess ? UW_OK : UW_ERR_CUDA;

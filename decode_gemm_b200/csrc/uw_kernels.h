@@ -54,6 +54,12 @@ namespace uw {
 // Reconstructive / plain GEMM: Y[M, N] = X[M, K] * W^T.
 enum GemmMode { kGemmBf16 = 0, kGemmExp = 1, kGemmPalette = 2 };
 
+// Most persistent CTAs a GEMM launch may use, and the words of the per-handle
+// split-K hand-off block: [0] launch epoch, [1] CTAs that have exited, then
+// one ready flag per CTA (see launch_gemm).  The block starts zeroed.
+constexpr int kGemmMaxCtas = 1024;
+constexpr int kGemmSyncWords = 2 + kGemmMaxCtas;
+
 struct GemmArgs {
   int mode = kGemmBf16;
   int64_t M = 0, N = 0, K = 0;
@@ -71,6 +77,7 @@ struct GemmArgs {
   int out_f32 = 0;
   float* partials = nullptr;     // workspace for split partial sums
   size_t partials_bytes = 0;
+  uint32_t* sync = nullptr;      // kGemmSyncWords words, zeroed before first use
   int tile_n = 0;                // tokens per tile (0 = auto)
   int stages = 0;                // load ring depth (0 = auto)
   int wslots = 0;                // rebuilt-W ring depth (0 = auto)

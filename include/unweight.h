@@ -191,7 +191,11 @@ UW_API uw_status uw_stats(uw_handle_t h, uw_stats_t* out);
  * uw_set_workspace registers caller-owned device memory (kept by pointer until
  * replaced or the handle is freed; ptr NULL unregisters); uw_alloc_workspace
  * makes the handle allocate and own one of `bytes` bytes.  Calls that need
- * more workspace than registered return UW_ERR_WORKSPACE and launch nothing. */
+ * more workspace than registered return UW_ERR_WORKSPACE and launch nothing.
+ * A tile whose K range is split between CTAs is summed inside the GEMM
+ * kernel, through the workspace and a small hand-off block the handle owns;
+ * so a handle's calls must be ordered (one stream, or synchronised streams):
+ * two of its GEMMs running at the same time race. */
 UW_API uw_status uw_workspace_bytes(uw_handle_t h, int32_t pipeline, int64_t M, size_t* bytes);
 UW_API uw_status uw_set_workspace(uw_handle_t h, void* ws_dev, size_t bytes);
 UW_API uw_status uw_alloc_workspace(uw_handle_t h, size_t bytes);
@@ -232,7 +236,7 @@ UW_API uw_status uw_gemm_ex(uw_handle_t h, const uint16_t* X_dev, void* Y_dev, i
  *   - Computes Y[M, N] = X W^T like uw_gemm(..., UW_PIPE_PALETTE_DIRECT);
  *     Y is float* when out_f32 is nonzero, else BF16.  Needs a handle
  *     uploaded with prepare_direct (UW_ERR_UNSUPPORTED otherwise).
- *   - Limit: M <= 64 (UW_ERR_SHAPE above that).  The array is 10 MiB and is
+ *   - Limit: M <= 64 (UW_ERR_SHAPE above that).  The array is 5 MiB and is
  *     held on every GPU where the library's device code is loaded, until the
  *     process exits.
  *   - The handle's device must be current (UW_ERR_ARG otherwise).  The first
@@ -273,7 +277,7 @@ UW_API uw_status uw_get_choice(uw_handle_t h, int64_t M, uw_gemm_config* cfg);
 typedef enum uw_kernel_kind {
   UW_KERNEL_DECODE_FULL = 0, UW_KERNEL_DECODE_EXP = 1, UW_KERNEL_TRANSCODE = 2,
   UW_KERNEL_GEMM_BF16 = 3, UW_KERNEL_GEMM_EXP = 4, UW_KERNEL_GEMM_PALETTE = 5,
-  UW_KERNEL_SPLITK_FIXUP = 6
+  UW_KERNEL_SPLITK_FIXUP = 6  /* reserved: split tiles are summed inside the GEMM */
 } uw_kernel_kind;
 UW_API uw_status uw_trace_enable(uw_handle_t h, int32_t enable);
 UW_API uw_status uw_trace_read(uw_handle_t h, int32_t* kinds, float* ms, int32_t capacity,
