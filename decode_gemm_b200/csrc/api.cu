@@ -178,7 +178,7 @@ uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg) {
   if (!valid_pipeline(cfg.pipeline)) return UW_ERR_ARG;
   if (cfg.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) return UW_ERR_UNSUPPORTED;
   if (cfg.tile_n < 0 || cfg.tile_n > 256 || cfg.tile_n % 16) return UW_ERR_ARG;
-  if (cfg.stages < 0 || cfg.stages > 12 || (cfg.stages & 1)) return UW_ERR_ARG;
+  if (cfg.stages < 0 || cfg.stages > 16 || (cfg.stages & 1)) return UW_ERR_ARG;
   if (cfg.gemm_ctas < 0 || cfg.decode_ctas < 0) return UW_ERR_ARG;
   return UW_OK;
 }

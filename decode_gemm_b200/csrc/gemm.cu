@@ -54,8 +54,10 @@ using namespace sm100;
 constexpr int kBM = 128;           // W rows per tile (MMA M)
 constexpr int kBK = 64;            // K per stage: one 128-byte swizzle row of BF16
 constexpr int kWTileBytes = kBM * kBK * 2;
-constexpr int kEscCap = 32;        // escape rows staged per stage (more: read from global)
+constexpr int kEscCap = 14;        // escape rows staged per stage (more: read from global);
+                                   // 14 makes a 16-token palette stage exactly 15 KB
 constexpr int kMaxWSlots = 8;      // rebuilt-W ring depth (runtime, <= this)
+constexpr int kMaxStages = 16;     // load ring depth (runtime, <= this)
 constexpr int kNumEpiWarps = 4;
 constexpr int kNumRebuildWarps = 8;  // two groups of 4, alternating stages
 constexpr int kGroupWarps = kNumRebuildWarps / 2;
@@ -707,8 +709,10 @@ bool gemm_resolve(GemmArgs* a) {
   if (a->tile_n < 16 || a->tile_n > 256 || a->tile_n % 16) return false;
   // Ring depths are even: consumers alternate units, so an even depth keeps
   // every slot with one consumer (see the MMA issuers in the kernel).
-  const int max_stages = a->mode == kGemmBf16 ? 12 : 8;
-  // rebuilt-W ring: 4 slots, 2 when shared memory is short
+  // As many load stages as fit (up to kMaxStages) beside four rebuilt-W slots
+  // (two per rebuild group: with one, a group's next rebuild waits for its
+  // last tile's MMA).
+  const int max_stages = a->mode == kGemmBf16 ? 12 : kMaxStages;
   if (a->wslots == 0) a->wslots = a->mode == kGemmBf16 ? 0 : 4;
   if (a->mode != kGemmBf16 &&
       (a->wslots < 2 || a->wslots > kMaxWSlots || (a->wslots & 1)))

@@ -133,7 +133,7 @@ typedef struct uw_stats_t {
 typedef struct uw_gemm_config {
   int32_t pipeline;      /* uw_pipeline, not AUTO                                  */
   int32_t tile_n;        /* tokens per MMA tile: 16..256, multiple of 16 (0=auto)  */
-  int32_t stages;        /* shared-memory ring depth, even, 2..12 (0 = auto)       */
+  int32_t stages;        /* shared-memory ring depth, even, 2..16 (0 = auto)       */
   int32_t gemm_ctas;     /* persistent GEMM CTAs (0 = one per SM)                   */
   int32_t decode_ctas;   /* SMs (one CTA each) of the preprocessing kernel (0 = all) */
   int32_t reserved[3];
