@@ -55,10 +55,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum; profiles/*.md), valid only while the kernel source
 # (src_sha, see _kernel_src_sha) is unchanged.
 TRAFFIC = {
-    "gemm_palette": {"bytes_per_launch": 90.173952e6 + 3.2064e6, "src_sha": "42f5962f3a4e66ea",
+    "gemm_palette": {"bytes_per_launch": 90.58176e6 + 3.479552e6, "src_sha": "2a73685f6de8ccf6",
                      "capture": "profiles/gemm_palette_gate_14336x4096_M1.md (M = 1 launch)"},
-    "transcode": {"bytes_per_launch": 19.4304e6 + 0.097024e6, "src_sha": "42f5962f3a4e66ea",
+    "decode_full": {"bytes_per_launch": 88.303104e6 + 68.056576e6, "src_sha": "2a73685f6de8ccf6",
+                    "capture": "profiles/decode_full_gate_14336x4096.md (output partly still in L2)"},
+    "transcode": {"bytes_per_launch": 20.110336e6 + 4.608e6, "src_sha": "2a73685f6de8ccf6",
                   "capture": "profiles/transcode_gate_14336x4096.md (output still in L2)"},
+    "gemm_bf16": {"bytes_per_launch": 118.631168e6 + 3.966976e6, "src_sha": "2a73685f6de8ccf6",
+                  "capture": "profiles/gemm_bf16_gate_14336x4096_M1.md (M = 1 launch)"},
 }
 
 
@@ -70,6 +74,10 @@ def _args():
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # single-kernel runs for profilers: three launches of one kernel, nothing timed
+    ap.add_argument("--only", choices=("decode_full", "decode_exp", "transcode", "gemm_bf16",
+                                       "gemm_exp", "gemm_palette"))
+    ap.add_argument("--m", type=int, default=1, help="tokens for --only gemm_*")
     return ap.parse_args()
 
 
@@ -99,7 +107,6 @@ def _alg_bytes(kind, st, M, N, K, x_frac=1.0):
         "gemm_bf16": 2 * T + xy,
         "gemm_exp": 2 * T + xy,
         "gemm_palette": T + T // 2 + esc + xy,
-        "splitk_fixup": 0,
     }[kind]
 
 
@@ -373,7 +380,7 @@ def run_ours(args):
             pre, gemm = _run_kernels(p)
             st = stats[idx]
             rec = {}
-            for kind in ([pre] if pre else []) + [gemm, "splitk_fixup"]:
+            for kind in ([pre] if pre else []) + [gemm]:
                 c = cursor[idx]
                 if c < len(tr) and tr[c][0] == kind:
                     rec[kind] = tr[c][1]
@@ -386,18 +393,6 @@ def run_ours(args):
                     if kind.startswith("gemm"):
                         agg["flops"] += 2 * m * N * K
             per_run.setdefault((m, p), []).append(rec)
-    # the split-K fix-up finishes its GEMM's output: charge its time to that GEMM
-    gemm_kinds = [k for k in per_kind if k.startswith("gemm")]
-    fix = per_kind.pop("splitk_fixup", None)
-    if fix and gemm_kinds:
-        fix_by_gemm = {}
-        for (m, p), recs in per_run.items():
-            g = _run_kernels(p)[1]
-            fix_by_gemm[g] = fix_by_gemm.get(g, 0.0) + sum(r.get("splitk_fixup", 0.0) for r in recs)
-        for g, t in fix_by_gemm.items():
-            if g in per_kind:
-                per_kind[g]["ms"] += t
-                per_kind[g]["fixup_ms"] = t
     dominant = max(per_kind, key=lambda k: per_kind[k]["ms"])
     peaks, peak_src = _peaks()
     d = per_kind[dominant]
@@ -411,7 +406,6 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": d["bytes"] / d["n"],
                 "avg_launch_us": 1e3 * d["ms"] / d["n"], "peak_source": peak_src}
     kernels = {k: {"launches": v["n"], "total_ms": v["ms"], "share": v["ms"] / elapsed_ms,
-                   "fixup_ms": v.get("fixup_ms", 0.0),
                    "GBps": v["bytes"] / (v["ms"] * 1e-3) / 1e9 if v["ms"] > 0 else None,
                    "frac_hbm": (v["bytes"] / (v["ms"] * 1e-3) / 1e9) / peaks["hbm_gbs"]
                    if v["ms"] > 0 else None}
@@ -423,11 +417,10 @@ def run_ours(args):
             return 1e3 * statistics.median(xs) if xs else None
         pre, gemm = _run_kernels(p)
         g = med(gemm) or 0.0
-        fx = med("splitk_fixup") or 0.0
         pr = med(pre) if pre else 0.0
-        pipelines[f"{p}/M{m}"] = {"preprocess_us": pr, "gemm_us": g + fx, "total_us": pr + g + fx,
-                                  "gemm_tflops": 2 * m * N * K / ((g + fx) * 1e-6) / 1e12
-                                  if g + fx > 0 else None}
+        pipelines[f"{p}/M{m}"] = {"preprocess_us": pr, "gemm_us": g, "total_us": pr + g,
+                                  "gemm_tflops": 2 * m * N * K / (g * 1e-6) / 1e12
+                                  if g > 0 else None}
 
     # ---- BF16 torch.matmul on the same box (context only)
     wbf = []
@@ -516,8 +509,48 @@ def run_ours(args):
     return 0
 
 
+def run_only(args):
+    """Three launches of one kernel on the bench workload (first set of weights),
+    for a profiler to capture (select by kernel name: decode_kernel<0|1|2> is
+    exponent / full / transcode, gemm_kernel<0|1|2> bf16 / exponent / palette).
+    The handle is uploaded without the load-time transcode unless the palette
+    GEMM needs it (that launch comes first)."""
+    import numpy as np
+    import torch
+    import decode_gemm_b200 as uw
+    import synthdata
+
+    w = synthdata.workload(args.workload)
+    N, K = w.shape
+    h = uw.uw_encode(w, uw.default_opts(prepare_direct=1 if args.only == "gemm_palette" else 0))
+    out = torch.empty(2 * N * K, dtype=torch.uint8, device="cuda")
+    pipe = {"gemm_bf16": 1, "gemm_exp": 2, "gemm_palette": 4}.get(args.only)
+    if pipe:
+        M = args.m
+        X = torch.from_numpy(synthdata.activations(M, K, seed=11 + M).view(np.int16)).cuda()
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(uw.uw_workspace_bytes(h, pipe, M), dtype=torch.uint8, device="cuda")
+        uw.uw_set_workspace(h, ws)
+    for _ in range(3):
+        if args.only == "decode_full":
+            uw.uw_decode_full(h, out)
+        elif args.only == "decode_exp":
+            uw.uw_decode_exp(h, out)
+        elif args.only == "transcode":
+            uw.uw_transcode_palette(h, out)
+        else:  # pipelines 1 and 2 run their decode first (select the GEMM by name)
+            uw.uw_gemm(h, X, Y, M, pipe)
+    torch.cuda.synchronize()
+    if uw.uw_last_device_status(h) != uw.UW_OK:
+        raise SystemExit("device status not OK")
+    print(json.dumps({"only": args.only, "m": args.m if pipe else None, "launches": 3}))
+    return 0
+
+
 def main():
     args = _args()
+    if args.only:
+        return run_only(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
