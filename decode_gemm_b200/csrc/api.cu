@@ -60,6 +60,7 @@ GemmArgs base_gemm_args(const uw_handle_s* h) {
   a.esc_bits = h->d_esc_bits;
   a.esc_off = h->d_esc_off;
   a.esc_exp = h->d_esc_exp;
+  a.esc_pack = h->d_esc_pack;
   a.esc_nw = (int32_t)(4 * ((h->N + kEscGroupRows - 1) / kEscGroupRows));
   std::memcpy(a.palette, h->palette, 16);
   a.sm_count = h->sm_count;
@@ -312,6 +313,8 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   const size_t o_ebits = place((size_t)std::max<int64_t>(f->n_esc_words, 1) * 4);
   const size_t o_eoff = place((size_t)(f->n_esc_groups + 1) * 4);
   const size_t o_eexp = place((size_t)std::max<int64_t>(f->n_esc_rows, 1) * kRow);
+  const size_t pack_bytes = (size_t)f->n_esc_groups * 16 + (size_t)f->n_esc_rows * kRow;
+  const size_t o_epack = place(std::max<size_t>(pack_bytes, 16));
   const size_t o_stat = place(256);
   const size_t o_sync = place(kGemmSyncWords * 4);
   const size_t o_pidx = o.prepare_direct ? place(T / 2) : 0;
@@ -329,6 +332,19 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   h->d_esc_bits = reinterpret_cast<uint32_t*>(base + o_ebits);
   h->d_esc_off = reinterpret_cast<uint32_t*>(base + o_eoff);
   h->d_esc_exp = base + o_eexp;
+  h->d_esc_pack = base + o_epack;
+  // escape groups packed for the GEMM: bitmap of the group's 128 rows, then its rows
+  std::vector<uint8_t> pack(pack_bytes);
+  {
+    const int64_t KB = f->K / kRow, nwp = 4 * ((f->N + kEscGroupRows - 1) / kEscGroupRows);
+    for (int64_t g = 0; g < f->n_esc_groups; ++g) {
+      const int64_t nt = g / KB, kb = g % KB;
+      uint8_t* dst = pack.data() + 16 * g + (size_t)f->esc_off[g] * kRow;
+      std::memcpy(dst, f->esc_bits + kb * nwp + nt * 4, 16);
+      std::memcpy(dst + 16, f->esc_exp + (size_t)f->esc_off[g] * kRow,
+                  (size_t)(f->esc_off[g + 1] - f->esc_off[g]) * kRow);
+    }
+  }
   h->d_status = reinterpret_cast<uint32_t*>(base + o_stat);
   h->d_sync = reinterpret_cast<uint32_t*>(base + o_sync);
   h->d_pal_idx = o.prepare_direct ? base + o_pidx : nullptr;
@@ -342,6 +358,7 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
       {(void**)&h->d_esc_bits, f->esc_bits, (size_t)f->n_esc_words * 4},
       {(void**)&h->d_esc_off, f->esc_off, (size_t)(f->n_esc_groups + 1) * 4},
       {(void**)&h->d_esc_exp, f->esc_exp, (size_t)f->n_esc_rows * kRow},
+      {(void**)&h->d_esc_pack, pack.data(), pack_bytes},
   };
   for (const Part& p : parts) {
     if (p.bytes == 0) continue;

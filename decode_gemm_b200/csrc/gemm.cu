@@ -54,13 +54,16 @@ using namespace sm100;
 constexpr int kBM = 128;           // W rows per tile (MMA M)
 constexpr int kBK = 64;            // K per stage: one 128-byte swizzle row of BF16
 constexpr int kWTileBytes = kBM * kBK * 2;
-constexpr int kEscCap = 14;        // escape rows staged per stage (more: read from global);
-                                   // 14 makes a 16-token palette stage exactly 15 KB
+constexpr int kEscCap = 15;        // escape rows staged per stage (more: read from global);
+                                   // 15 keeps a 16-token palette stage at 15 KB
 constexpr int kMaxWSlots = 8;      // rebuilt-W ring depth (runtime, <= this)
 constexpr int kMaxStages = 16;     // load ring depth (runtime, <= this)
 constexpr int kNumEpiWarps = 4;
 constexpr int kNumRebuildWarps = 8;  // two groups of 4, alternating stages
 constexpr int kGroupWarps = kNumRebuildWarps / 2;
+constexpr int kGroupThreads = kGroupWarps * 32;
+constexpr int kRebuildItems = kBM * kBK / 8 / kGroupThreads;  // 8-weight items per thread
+static_assert(kRebuildItems == 8, "escape-bit mapping assumes rows gt/8 + 16 i");
 constexpr int kMmaWarp0 = 1;         // MMA issuers: warps 1 and 2
 constexpr int kNumMmaWarps = 2;
 constexpr int kEpiWarp0 = kMmaWarp0 + kNumMmaWarps;  // warps 3..6 (quadrants 3,0,1,2)
@@ -79,6 +82,7 @@ struct GemmParams {
   const uint32_t* esc_bits;
   const uint32_t* esc_off;
   const uint8_t* esc_exp;
+  const uint8_t* esc_pack;  // per group (tile, K block): 16-byte bitmap, then its escape rows
   void* Y;
   float* partials;
   uint32_t* status;
@@ -110,9 +114,9 @@ __host__ __device__ inline StageLayout stage_layout(int mode, int tile_n) {
     L.bytes = xb + 16384;
   } else {
     L.w1 = xb + 8192;
-    L.ebits = xb + 12288;
-    L.erows = xb + 12288 + 128;
-    L.bytes = xb + 12288 + 128 + kEscCap * 64;
+    L.ebits = xb + 12288;        // bitmap and escape rows arrive in one copy
+    L.erows = xb + 12288 + 16;
+    L.bytes = xb + 12288 + 16 + kEscCap * 64;
   }
   L.bytes = (L.bytes + 1023) / 1024 * 1024;
   return L;
@@ -284,7 +288,13 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             if (MODE == kGemmExp) bytes += 16384;
             if (MODE == kGemmPalette) {
               nesc = min(c1 - c0, (uint32_t)kEscCap);
-              bytes += 8192 + 4096 + 16 + nesc * 64;
+              bytes += 8192 + 4096 + (c1 > c0 ? 16 + nesc * 64 : 0);
+              // a group with no escape row needs no copy: its bitmap is zero
+              if (c1 == c0) {
+                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(smem_u32(st + L.ebits)),
+                             "r"(0u)
+                             : "memory");
+              }
             }
             mbar_expect_tx(fb, bytes);
             tma_load_2d(smem_u32(st + L.x), &p.tm_x, fb, kb * kBK, m0);
@@ -292,10 +302,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             if (MODE == kGemmExp) tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kb * kBK, n0);
             if (MODE == kGemmPalette) {
               tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kb * (kBK / 2), n0);
-              bulk_load(smem_u32(st + L.ebits), p.esc_bits + (int64_t)kb * p.esc_nwp + nt * 4, 16,
-                        fb);
-              if (nesc)
-                bulk_load(smem_u32(st + L.erows), p.esc_exp + (int64_t)c0 * 64, nesc * 64, fb);
+              if (c1 > c0)  // group gi's bitmap and first nesc rows
+                bulk_load(smem_u32(st + L.ebits),
+                          p.esc_pack + 16 * (nt * KB + kb) + (int64_t)c0 * 64, 16 + nesc * 64, fb);
             }
             ++issued;
           }
@@ -560,45 +569,59 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           else
             v4[i] = *reinterpret_cast<const uint32_t*>(st + L.w1 + r * 32 + c * 4);
         }
-        // thread rows r_i = gt/8 + 16 i: row r_i's escape bit is bit gt/8 + 16 (i & 1)
-        // of bitmap word i / 2; most warps see no escape row in a tile and skip
-        // the per-row test
-        uint32_t eb[4] = {0u, 0u, 0u, 0u};
-        uint32_t emask = 0;
-        if (MODE == kGemmPalette) {
-          const uint4 w4 = *reinterpret_cast<const uint4*>(st + L.ebits);
-          eb[0] = w4.x;
-          eb[1] = w4.y;
-          eb[2] = w4.z;
-          eb[3] = w4.w;
-          const uint32_t sh = (uint32_t)gt >> 3;
+        // every item as if no row were an escape row (no branch in the loop, so
+        // the items' dependency chains interleave) ...
 #pragma unroll
-          for (int i = 0; i < 8; ++i) emask |= ((eb[i >> 1] >> (sh + 16 * (i & 1))) & 1u) << i;
-        }
-        const bool any_esc = MODE == kGemmPalette && __any_sync(0xffffffffu, emask != 0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c8 = gt + 128 * i;
+        for (int i = 0; i < kRebuildItems; ++i) {
+          const int c8 = gt + kGroupThreads * i;
           const int r = c8 >> 3, c = c8 & 7;
-          if (MODE == kGemmPalette) {
+          if (MODE == kGemmPalette)
             e8[i] = palette8(v4[i], p.palette[0], p.palette[1], p.palette[2], p.palette[3]);
-            if (any_esc && ((emask >> i) & 1u)) {
-              // an escape row: its verbatim exponents, slot = escape rows before it
-              uint32_t slot = (uint32_t)__popc(eb[r >> 5] & ((1u << (r & 31)) - 1u));
-              for (int w = 0; w < (r >> 5); ++w) slot += (uint32_t)__popc(eb[w]);
-              if (slot < (uint32_t)kEscCap) {
-                e8[i] = *reinterpret_cast<const uint2*>(st + L.erows + slot * 64 + c * 8);
-              } else {
-                const uint32_t first = __ldg(p.esc_off + nt * KB + kb);
-                e8[i] = __ldg(reinterpret_cast<const uint2*>(p.esc_exp +
-                                                             (int64_t)(first + slot) * 64 + c * 8));
-              }
-            }
-          }
           const uint2 lo = merge4(s8[i].x, e8[i].x);
           const uint2 hi = merge4(s8[i].y, e8[i].y);
           *reinterpret_cast<uint4*>(wt + r * 128 + ((c ^ (r & 7)) << 4)) =
               make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+        // ... then the escape rows.  Thread rows r_i = gt/8 + 16 i, so a warp's
+        // 32 rows are bits 4w..4w+3 and 16+4w..16+4w+3 (w = warp in the group) of
+        // each 32-row bitmap word: one masked OR tells the whole warp whether
+        // any of its rows is an escape row.  Those rows' verbatim exponents (slot
+        // = escape rows before the row in the tile) overwrite the 16-byte pieces
+        // just written.
+        uint4 eb4 = make_uint4(0u, 0u, 0u, 0u);
+        if (MODE == kGemmPalette) eb4 = *reinterpret_cast<const uint4*>(st + L.ebits);
+        const uint32_t warp_rows = 0x000F000Fu << (4 * (gt >> 5));
+        if (MODE == kGemmPalette && ((eb4.x | eb4.y | eb4.z | eb4.w) & warp_rows)) {
+          const uint32_t eb[4] = {eb4.x, eb4.y, eb4.z, eb4.w};
+          const uint32_t sh = (uint32_t)gt >> 3;
+          uint32_t emask = 0;
+#pragma unroll
+          for (int i = 0; i < kRebuildItems; ++i)
+            emask |= ((eb[i >> 1] >> (sh + 16 * (i & 1))) & 1u) << i;
+          const uint32_t pc1 = __popc(eb[0]), pc2 = pc1 + __popc(eb[1]),
+                         pc3 = pc2 + __popc(eb[2]);
+#pragma unroll
+          for (int i = 0; i < kRebuildItems; ++i) {
+            if (!((emask >> i) & 1u)) continue;
+            const int c8 = gt + kGroupThreads * i;
+            const int r = c8 >> 3, c = c8 & 7;
+            const int w = r >> 5;
+            const uint32_t word = w == 0 ? eb[0] : w == 1 ? eb[1] : w == 2 ? eb[2] : eb[3];
+            const uint32_t before = w == 0 ? 0u : w == 1 ? pc1 : w == 2 ? pc2 : pc3;
+            const uint32_t slot = before + (uint32_t)__popc(word & ((1u << (r & 31)) - 1u));
+            uint2 ex;
+            if (slot < (uint32_t)kEscCap) {
+              ex = *reinterpret_cast<const uint2*>(st + L.erows + slot * 64 + c * 8);
+            } else {
+              const uint32_t first = __ldg(p.esc_off + nt * KB + kb);
+              ex = __ldg(reinterpret_cast<const uint2*>(p.esc_exp + (int64_t)(first + slot) * 64 +
+                                                        c * 8));
+            }
+            const uint2 lo = merge4(s8[i].x, ex.x);
+            const uint2 hi = merge4(s8[i].y, ex.y);
+            *reinterpret_cast<uint4*>(wt + r * 128 + ((c ^ (r & 7)) << 4)) =
+                make_uint4(lo.x, lo.y, hi.x, hi.y);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -772,6 +795,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.esc_bits = a.esc_bits;
   p.esc_off = a.esc_off;
   p.esc_exp = a.esc_exp;
+  p.esc_pack = a.esc_pack;
   p.Y = a.Y;
   p.partials = a.partials;
   p.status = a.status;

@@ -32,6 +32,9 @@ struct uw_handle_s {
   uint32_t* d_esc_bits = nullptr;
   uint32_t* d_esc_off = nullptr;
   uint8_t* d_esc_exp = nullptr;
+  // per escape group g = (n/128, kb): its 16-byte row bitmap, then its escape
+  // rows (64 bytes each), at byte 16 g + 64 esc_off[g] (one copy per GEMM unit)
+  uint8_t* d_esc_pack = nullptr;
   uint32_t* d_status = nullptr;
   uint32_t* d_sync = nullptr;    // GEMM split-K hand-off (kGemmSyncWords, zeroed at upload)
   uint8_t* d_pal_idx = nullptr;  // resident palette indices (pipeline 4), may be null

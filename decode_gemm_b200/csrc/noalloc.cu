@@ -75,6 +75,7 @@ uw_status uw_gemm_palette_noalloc(uw_handle_t h, const uint16_t* X_dev, void* Y_
   a.esc_bits = h->d_esc_bits;
   a.esc_off = h->d_esc_off;
   a.esc_exp = h->d_esc_exp;
+  a.esc_pack = h->d_esc_pack;
   a.esc_nw = (int32_t)(4 * ((h->N + uw::kEscGroupRows - 1) / uw::kEscGroupRows));
   std::memcpy(a.palette, h->palette, 16);
   a.Y = Y_dev;

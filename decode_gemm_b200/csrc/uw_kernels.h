@@ -71,6 +71,7 @@ struct GemmArgs {
   const uint32_t* esc_bits = nullptr;
   const uint32_t* esc_off = nullptr;
   const uint8_t* esc_exp = nullptr;
+  const uint8_t* esc_pack = nullptr;   // per group: bitmap then rows (see handle)
   int32_t esc_nw = 0;
   uint8_t palette[16] = {0};
   void* Y = nullptr;             // [M, N] bf16 or f32
