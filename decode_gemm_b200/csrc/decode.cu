@@ -110,6 +110,33 @@ __device__ __forceinline__ void bits_slide(Bits& b, const uint32_t* words) {
       : "l"(p));
 }
 
+// Predicated global accesses: the write-out computes every piece and only
+// stores (or, for inputs that may lie past the arrays, loads) under the
+// predicate, so its loops carry no branch and their iterations interleave.
+__device__ __forceinline__ void st_v4_if(void* p, uint4 v, bool pred) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %5, 0;\n\t"
+               "@q st.global.v4.u32 [%0], {%1, %2, %3, %4};\n\t}"
+               ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"((uint32_t)pred)
+               : "memory");
+}
+
+__device__ __forceinline__ uint2 ld_v2_if(const void* p, bool pred) {
+  uint2 v = make_uint2(0u, 0u);
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %3, 0;\n\t"
+      "@q ld.global.nc.v2.u32 {%0, %1}, [%2];\n\t}"
+      : "+r"(v.x), "+r"(v.y)
+      : "l"(p), "r"((uint32_t)pred));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_u32_if(const uint32_t* p, bool pred) {
+  uint32_t v = 0u;
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q ld.global.nc.u32 %0, [%1];\n\t}"
+      : "+r"(v)
+      : "l"(p), "r"((uint32_t)pred));
+  return v;
+}
+
 // Stream bit position of the next bit.
 __device__ __forceinline__ uint32_t bits_pos(const Bits& b) { return (b.nxt - 4u) * 32u + b.q; }
 
@@ -314,12 +341,11 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         for (int i = 0; i < 8; ++i) {
           const int j = 4 * i + jq;
           const int64_t o = (int64_t)j * cs;
-          if (in_chunk && o + rel0 + 16 * m < grp_syms_left) {
-            const uint32_t* sw = stage + j * kStageStride + 2 * m;
-            const uint2 lo = palette8(sw[0], p0, p1, p2, p3);
-            const uint2 hi = palette8(sw[1], p0, p1, p2, p3);
-            *reinterpret_cast<uint4*>(base + o) = make_uint4(lo.x, lo.y, hi.x, hi.y);
-          }
+          const uint32_t* sw = stage + j * kStageStride + 2 * m;
+          const uint2 lo = palette8(sw[0], p0, p1, p2, p3);
+          const uint2 hi = palette8(sw[1], p0, p1, p2, p3);
+          st_v4_if(base + o, make_uint4(lo.x, lo.y, hi.x, hi.y),
+                   in_chunk && o + rel0 + 16 * m < grp_syms_left);
         }
       } else if (MODE == kDecodeFull) {
         // 16 lanes per chunk, 8 symbols (one rank word) per lane
@@ -335,19 +361,16 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int64_t o = (int64_t)(16 * h + 2 * i + jh) * cs;
-            sv[i] = (in_chunk && o + rel0 + 8 * m < grp_syms_left)
-                        ? __ldg(reinterpret_cast<const uint2*>(sbase + o))
-                        : make_uint2(0u, 0u);
+            sv[i] = ld_v2_if(sbase + o, in_chunk && o + rel0 + 8 * m < grp_syms_left);
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int j = 16 * h + 2 * i + jh;
             const int64_t o = (int64_t)j * cs;
-            if (in_chunk && o + rel0 + 8 * m < grp_syms_left) {
-              const uint2 e = palette8(stage[j * kStageStride + m], p0, p1, p2, p3);
-              const uint2 lo = merge4(sv[i].x, e.x), hi = merge4(sv[i].y, e.y);
-              *reinterpret_cast<uint4*>(obase + o) = make_uint4(lo.x, lo.y, hi.x, hi.y);
-            }
+            const uint2 e = palette8(stage[j * kStageStride + m], p0, p1, p2, p3);
+            const uint2 lo = merge4(sv[i].x, e.x), hi = merge4(sv[i].y, e.y);
+            st_v4_if(obase + o, make_uint4(lo.x, lo.y, hi.x, hi.y),
+                     in_chunk && o + rel0 + 8 * m < grp_syms_left);
           }
         }
       } else {
@@ -363,19 +386,17 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
           const int n_j = __shfl_sync(0xffffffffu, n_me, j);
           const int kb_j = __shfl_sync(0xffffffffu, kb_me, j);
           const int64_t o = (int64_t)j * cs;
-          if (in_chunk && o + rel0 + 32 * m < grp_syms_left) {
-            int n = n_j, kb = kb_j + (m >> 1);
-            while (kb >= a.kb_per_row) {
-              kb -= a.kb_per_row;
-              ++n;
-            }
-            const bool esc =
-                (__ldg(a.esc_bits + (int64_t)kb * a.esc_nw + (n >> 5)) >> (n & 31)) & 1u;
-            const uint32_t* sw = stage + j * kStageStride + 4 * m;
-            uint4 v = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-            if (esc) v = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(base + o / 2) = v;
+          const bool valid = in_chunk && o + rel0 + 32 * m < grp_syms_left;
+          int n = n_j, kb = kb_j + (m >> 1);
+          while (kb >= a.kb_per_row) {  // a row of 64 weights past the end of row n
+            kb -= a.kb_per_row;
+            ++n;
           }
+          const bool esc =
+              (ld_u32_if(a.esc_bits + (int64_t)kb * a.esc_nw + (n >> 5), valid) >> (n & 31)) & 1u;
+          const uint32_t* sw = stage + j * kStageStride + 4 * m;
+          const uint4 v = esc ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(sw[0], sw[1], sw[2], sw[3]);
+          st_v4_if(base + o / 2, v, valid);
         }
       }
       __syncwarp();
