@@ -160,6 +160,7 @@ uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
   a.out_f32 = out_f32;
   a.tile_n = cfg.tile_n;
   a.stages = cfg.stages;
+  a.halves = cfg.halves;
   a.ctas = cfg.gemm_ctas;
   switch (cfg.pipeline) {
     case UW_PIPE_FULL: a.mode = kGemmBf16; break;
@@ -179,7 +180,9 @@ uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg) {
   if (!valid_pipeline(cfg.pipeline)) return UW_ERR_ARG;
   if (cfg.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) return UW_ERR_UNSUPPORTED;
   if (cfg.tile_n < 0 || cfg.tile_n > 256 || cfg.tile_n % 16) return UW_ERR_ARG;
-  if (cfg.stages < 0 || cfg.stages > 16 || (cfg.stages & 1)) return UW_ERR_ARG;
+  if (cfg.halves < 0 || cfg.halves > 2) return UW_ERR_ARG;
+  if (cfg.stages < 0 || cfg.stages > 16 || (cfg.halves != 2 && (cfg.stages & 1)))
+    return UW_ERR_ARG;
   if (cfg.gemm_ctas < 0 || cfg.decode_ctas < 0) return UW_ERR_ARG;
   return UW_OK;
 }
@@ -446,18 +449,21 @@ uw_status uw_workspace_bytes(uw_handle_t h, int32_t pipeline, int64_t M, size_t*
     *bytes = 0;
     return UW_OK;
   }
-  // enough for any variant: every token tile (16..256) and up to one CTA per SM
+  // enough for any variant: every token tile (16..256), both unit shapes and
+  // up to one CTA per SM
   size_t worst = 0;
-  for (int tn = 16; tn <= 256; tn += 16) {
-    uw_gemm_config v = c;
-    v.tile_n = tn;
-    v.stages = 2;
-    v.gemm_ctas = h->sm_count;
-    GemmArgs a;
-    size_t need = 0, pre = 0;
-    if (plan_gemm(h, nullptr, nullptr, M, v, 1, &a, &need, &pre) == UW_OK)
-      worst = std::max(worst, need);
-  }
+  for (int hv = 1; hv <= 2; ++hv)
+    for (int tn = 16; tn <= 256; tn += 16) {
+      uw_gemm_config v = c;
+      v.tile_n = tn;
+      v.stages = 2;
+      v.halves = hv;
+      v.gemm_ctas = h->sm_count;
+      GemmArgs a;
+      size_t need = 0, pre = 0;
+      if (plan_gemm(h, nullptr, nullptr, M, v, 1, &a, &need, &pre) == UW_OK)
+        worst = std::max(worst, need);
+    }
   if (!worst) return UW_ERR_UNSUPPORTED;
   *bytes = worst;
   return UW_OK;

@@ -51,14 +51,19 @@ std::vector<uw_gemm_config> candidates(const uw_handle_s* h, int64_t M) {
   for (int p = UW_PIPE_FULL; p <= UW_PIPE_PALETTE_DIRECT; ++p) {
     if (p == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) continue;
     for (int t : tiles)
-      for (int st : {0, 4}) {
-        uw_gemm_config c;
-        std::memset(&c, 0, sizeof(c));
-        c.pipeline = p;
-        c.tile_n = t;
-        c.stages = st;
-        out.push_back(c);
-      }
+      for (int st : {0, 4})
+        for (int hv : {0, 1, 2}) {
+          // the wide shape only pays from a few token tiles on
+          if (hv == 2 && M < 256) continue;
+          if (hv == 1 && M < 512) continue;  // already the automatic choice
+          uw_gemm_config c;
+          std::memset(&c, 0, sizeof(c));
+          c.pipeline = p;
+          c.tile_n = t;
+          c.stages = st;
+          c.halves = hv;
+          out.push_back(c);
+        }
   }
   return out;
 }
@@ -322,9 +327,10 @@ uw_status uw_autotune(uw_handle_t* hs_in, int32_t n_handles, const int64_t* Ms, 
         const auto& c = chosen[i][j].second;
         std::fprintf(f,
                      "      {\"M\": %lld, \"pipeline\": %d, \"tile_n\": %d, \"stages\": %d, "
-                     "\"gemm_ctas\": %d, \"decode_ctas\": %d, \"us\": %.2f}%s\n",
+                     "\"gemm_ctas\": %d, \"decode_ctas\": %d, \"halves\": %d, \"us\": %.2f}%s\n",
                      (long long)chosen[i][j].first, c.pipeline, c.tile_n, c.stages, c.gemm_ctas,
-                     c.decode_ctas, 1e3 * chosen_ms[i][j], j + 1 < chosen[i].size() ? "," : "");
+                     c.decode_ctas, c.halves, 1e3 * chosen_ms[i][j],
+                     j + 1 < chosen[i].size() ? "," : "");
       }
       std::fprintf(f, "    ]}%s\n", i + 1 < hs.size() ? "," : "");
     }
@@ -360,13 +366,14 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
     const JVal* ch = hv.get("choices");
     if (!ch || ch->kind != JVal::Arr) return UW_ERR_FORMAT;
     for (const JVal& c : ch->arr) {
-      int64_t M = 0, pl = 0, tn = 0, sg = 0, gc = 0, dc = 0;
+      int64_t M = 0, pl = 0, tn = 0, sg = 0, gc = 0, dc = 0, hv2 = 0;
       if (c.kind != JVal::Obj || !num_field(c, "M", &M) || !num_field(c, "pipeline", &pl))
         return UW_ERR_FORMAT;
       num_field(c, "tile_n", &tn);
       num_field(c, "stages", &sg);
       num_field(c, "gemm_ctas", &gc);
       num_field(c, "decode_ctas", &dc);
+      num_field(c, "halves", &hv2);
       uw_gemm_config cfg;
       std::memset(&cfg, 0, sizeof(cfg));
       cfg.pipeline = (int32_t)pl;
@@ -374,6 +381,7 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
       cfg.stages = (int32_t)sg;
       cfg.gemm_ctas = (int32_t)gc;
       cfg.decode_ctas = (int32_t)dc;
+      cfg.halves = (int32_t)hv2;
       if (M <= 0 || check_config(hs[i], cfg) != UW_OK) return UW_ERR_FORMAT;
       parsed[i][M] = cfg;
     }

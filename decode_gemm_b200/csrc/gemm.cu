@@ -58,6 +58,7 @@ constexpr int kEscCap = 15;        // escape rows staged per stage (more: read f
                                    // 15 keeps a 16-token palette stage at 15 KB
 constexpr int kMaxWSlots = 8;      // rebuilt-W ring depth (runtime, <= this)
 constexpr int kMaxStages = 16;     // load ring depth (runtime, <= this)
+constexpr int64_t kWideMinM = 512;  // tokens from which units span 256 W rows
 constexpr int kNumEpiWarps = 4;
 constexpr int kNumRebuildWarps = 8;  // two groups of 4, alternating stages
 constexpr int kGroupWarps = kNumRebuildWarps / 2;
@@ -90,6 +91,9 @@ struct GemmParams {
   int64_t M, N, K;
   int64_t units;      // output tiles * K blocks
   int32_t tile_n, stages, wslots, n_mma, NT, MT, KB, esc_nwp, out_f32, tmem_cols;
+  int32_t halves;    // 128-row halves per unit: 1, or 2 for the wide (large-M) shape
+  int32_t acc_bufs;  // TMEM accumulator sets (2: epilogue overlaps the next tile)
+  int32_t NG;        // 128-row groups of W (escape groups per K block)
   uint32_t palette[4];
   uint32_t stage_bytes, x_bytes;
   uint64_t wait_ns;
@@ -100,23 +104,29 @@ struct StageLayout {
   uint32_t x, w0, w1, ebits, erows, bytes;
 };
 
-__host__ __device__ inline StageLayout stage_layout(int mode, int tile_n) {
+// A unit's H 128-row halves lie back to back in each region (the TMA boxes
+// cover all H*128 rows at once); palette escape data is per half: a 16-byte
+// bitmap, then up to kEscCap rows (kEscArea bytes).
+constexpr uint32_t kEscArea = 16 + kEscCap * 64;
+
+__host__ __device__ inline StageLayout stage_layout(int mode, int tile_n, int halves) {
   StageLayout L;
   L.x = 0;
   const uint32_t xb = (uint32_t)tile_n * kBK * 2;  // multiple of 2048 for tile_n % 16 == 0
+  const uint32_t H = (uint32_t)halves;
   L.w0 = xb;
   if (mode == kGemmBf16) {
-    L.w1 = L.ebits = L.erows = xb + kWTileBytes;
-    L.bytes = xb + kWTileBytes;
+    L.w1 = L.ebits = L.erows = xb + H * kWTileBytes;
+    L.bytes = xb + H * kWTileBytes;
   } else if (mode == kGemmExp) {
-    L.w1 = xb + 8192;
-    L.ebits = L.erows = xb + 16384;
-    L.bytes = xb + 16384;
+    L.w1 = xb + H * 8192;
+    L.ebits = L.erows = xb + H * 16384;
+    L.bytes = xb + H * 16384;
   } else {
-    L.w1 = xb + 8192;
-    L.ebits = xb + 12288;        // bitmap and escape rows arrive in one copy
-    L.erows = xb + 12288 + 16;
-    L.bytes = xb + 12288 + 16 + kEscCap * 64;
+    L.w1 = xb + H * 8192;
+    L.ebits = xb + H * 12288;  // half h: bitmap at ebits + h*kEscArea, rows 16 bytes on
+    L.erows = L.ebits + 16;
+    L.bytes = L.ebits + H * kEscArea;
   }
   L.bytes = (L.bytes + 1023) / 1024 * 1024;
   return L;
@@ -189,10 +199,16 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   // 1024-byte aligned, by an offset into the shared array (the accesses stay
   // shared-window loads and stores)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const StageLayout L = stage_layout(MODE, p.tile_n);
+  const StageLayout L = stage_layout(MODE, p.tile_n, p.halves);
   const int S = p.stages;
   const int WS = MODE == kGemmBf16 ? 0 : p.wslots;
-  const int NM = p.n_mma;  // MMA-issuing warps (K blocks split by parity)
+  // MMA-issuing warps: with one half per unit they split the units by parity
+  // (NM = 2) or one takes all (NM = 1); in the wide shape warp h takes half h
+  // of every unit, and rebuild group h rebuilds it
+  const int NM = p.n_mma;
+  const int H = p.halves;
+  const bool wide = H == 2;
+  const int RU = kBM * H;  // W rows per unit
   uint8_t* ring = smem;
   uint8_t* wring = ring + (size_t)S * L.bytes;  // rebuilt W tiles (reconstructive modes)
   uint8_t* tail = wring + (size_t)WS * kWTileBytes;
@@ -211,7 +227,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(bar(b_full + s), 1);
-      mbar_init(bar(b_empty + s), 1 + (MODE == kGemmBf16 ? 0 : kGroupWarps));
+      // released by each half's MMA commit and, reconstructive modes, its
+      // rebuild group's warps
+      mbar_init(bar(b_empty + s), (uint32_t)H * (1 + (MODE == kGemmBf16 ? 0 : kGroupWarps)));
     }
     for (int w = 0; w < WS; ++w) {
       mbar_init(bar(b_wfull + w), kGroupWarps);
@@ -256,25 +274,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
       const int64_t nt = t / p.MT, mt = t - nt * p.MT;
-      const int32_t n0 = (int32_t)(nt * kBM), m0 = (int32_t)(mt * p.tile_n);
-      // escape-row offsets of this tile's groups, 31 at a time in lanes
-      int win0 = kb0;
-      uint32_t eoff = 0;
-      if (MODE == kGemmPalette) {
-        const int64_t gi = nt * KB + win0 + lane;
-        eoff = gi <= (int64_t)p.NT * KB ? __ldg(p.esc_off + gi) : 0u;
-      }
+      const int32_t n0 = (int32_t)(nt * RU), m0 = (int32_t)(mt * p.tile_n);
       for (int kb = kb0; kb < kb1; ++kb) {
-        uint32_t c0 = 0, c1 = 0;
-        if (MODE == kGemmPalette) {
-          if (kb - win0 + 1 > 31) {
-            win0 = kb;
-            const int64_t gi = nt * KB + win0 + lane;
-            eoff = gi <= (int64_t)p.NT * KB ? __ldg(p.esc_off + gi) : 0u;
-          }
-          c0 = __shfl_sync(0xffffffffu, eoff, kb - win0);
-          c1 = __shfl_sync(0xffffffffu, eoff, kb - win0 + 1);
-        }
         if (lane == 0) {
           if (!mbar_wait_bounded(bar(b_empty + stage), phase ^ 1u, abort, p.wait_ns)) {
             set_abort(abort, p.status);
@@ -283,17 +284,33 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             uint8_t* st = ring + (size_t)stage * L.bytes;
             const uint32_t fb = bar(b_full + stage);
             uint32_t bytes = p.x_bytes;
-            uint32_t nesc = 0;
-            if (MODE == kGemmBf16) bytes += kWTileBytes;
-            if (MODE == kGemmExp) bytes += 16384;
+            if (MODE == kGemmBf16) bytes += H * kWTileBytes;
+            if (MODE == kGemmExp) bytes += H * 16384;
+            // escape rows of each half's group (128 rows, this K block): one
+            // copy of its bitmap and first rows, or none and a zero bitmap
+            uint32_t c0[2] = {0u, 0u}, nesc[2] = {0u, 0u};
+            bool has[2] = {false, false};
             if (MODE == kGemmPalette) {
-              nesc = min(c1 - c0, (uint32_t)kEscCap);
-              bytes += 8192 + 4096 + (c1 > c0 ? 16 + nesc * 64 : 0);
-              // a group with no escape row needs no copy: its bitmap is zero
-              if (c1 == c0) {
-                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(smem_u32(st + L.ebits)),
-                             "r"(0u)
-                             : "memory");
+              bytes += H * 12288;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                if (h >= H) break;
+                const int64_t grow = nt * H + h;  // 128-row group
+                if (grow < p.NG) {
+                  const int64_t gi = grow * KB + kb;
+                  c0[h] = __ldg(p.esc_off + gi);
+                  const uint32_t c1 = __ldg(p.esc_off + gi + 1);
+                  has[h] = c1 > c0[h];
+                  nesc[h] = min(c1 - c0[h], (uint32_t)kEscCap);
+                }
+                if (has[h]) {
+                  bytes += 16 + nesc[h] * 64;
+                } else {
+                  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
+                                   smem_u32(st + L.ebits + h * kEscArea)),
+                               "r"(0u)
+                               : "memory");
+                }
               }
             }
             mbar_expect_tx(fb, bytes);
@@ -302,9 +319,12 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             if (MODE == kGemmExp) tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kb * kBK, n0);
             if (MODE == kGemmPalette) {
               tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kb * (kBK / 2), n0);
-              if (c1 > c0)  // group gi's bitmap and first nesc rows
-                bulk_load(smem_u32(st + L.ebits),
-                          p.esc_pack + 16 * (nt * KB + kb) + (int64_t)c0 * 64, 16 + nesc * 64, fb);
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                if (h < H && has[h])
+                  bulk_load(smem_u32(st + L.ebits + h * kEscArea),
+                            p.esc_pack + 16 * ((nt * H + h) * KB + kb) + (int64_t)c0[h] * 64,
+                            16 + nesc[h] * 64, fb);
             }
             ++issued;
           }
@@ -334,15 +354,18 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     }
   } else if (warp < kMmaWarp0 + kNumMmaWarps) {
     // ---------------------------------------------------------- MMA issuers --
-    // Warp kMmaWarp0 + par takes the CTA's units q with q % 2 == par (all of
-    // them when NM == 1) and accumulates into its own TMEM columns.  The ring
-    // depths are even, so a stage or W slot is always consumed by the same
-    // warp, in order: a parity wait can then never see a stale phase.
+    // One half per unit: warp kMmaWarp0 + par takes the CTA's units q with
+    // q % 2 == par (all of them when NM == 1) and accumulates into its own
+    // TMEM columns.  The ring depths are then even, so a stage or W slot is
+    // always consumed by the same warp, in order: a parity wait can never see
+    // a stale phase.  Wide shape: warp par takes half par of every unit (W
+    // slots go in pairs, slot 2 j + par for pair j) into its own columns.
     const int par = warp - kMmaWarp0;
     if (par < NM) {
       const uint32_t idesc = idesc_bf16(kBM, p.tile_n);
+      const int WP = wide ? WS / 2 : WS;  // W slot positions this warp cycles through
       // ring positions of the current unit, advanced for every unit of the CTA
-      int stage = 0, wslot = 0;
+      int stage = 0, wpos = 0;
       uint32_t phase = 0, wphase = 0;
       int q = 0;  // index of the unit among this CTA's units
       int seg = 0;
@@ -351,8 +374,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         const int64_t t = u / KB;
         const int kb0 = (int)(u - t * KB);
         const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
-        const int acc = seg & 1;
-        const uint32_t acc_phase = (uint32_t)(seg >> 1) & 1u;
+        const int acc = p.acc_bufs == 2 ? (seg & 1) : 0;
+        const uint32_t acc_phase = (uint32_t)(p.acc_bufs == 2 ? (seg >> 1) : seg) & 1u;
         if (lane == 0 &&
             !mbar_wait_bounded(bar(b_tempty + acc), acc_phase ^ 1u, abort, p.wait_ns)) {
           set_abort(abort, p.status);
@@ -364,7 +387,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         const uint32_t d_tmem = tmem_base + (uint32_t)((acc * NM + par) * p.tile_n);
         bool first = true;
         for (int kb = kb0; kb < kb1; ++kb, ++q) {
-          const bool mine = NM == 1 || (q & 1) == par;
+          const bool mine = wide || NM == 1 || (q & 1) == par;
+          const int wslot = wide ? 2 * wpos + par : wpos;
           if (mine && lane == 0) {
             bool got = mbar_wait_bounded(bar(b_full + stage), phase, abort, p.wait_ns);
             if (got && MODE != kGemmBf16)
@@ -375,9 +399,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             } else {
               tc_fence_after();
               uint8_t* st = ring + (size_t)stage * L.bytes;
-              const uint32_t a_addr = MODE == kGemmBf16
-                                          ? smem_u32(st + L.w0)
-                                          : smem_u32(wring + (size_t)wslot * kWTileBytes);
+              const uint32_t a_addr =
+                  MODE == kGemmBf16 ? smem_u32(st + L.w0 + (wide ? par * kWTileBytes : 0))
+                                    : smem_u32(wring + (size_t)wslot * kWTileBytes);
               const uint64_t a_desc = smem_desc_sw128(a_addr);
               const uint64_t b_desc = smem_desc_sw128(smem_u32(st + L.x));
 #pragma unroll
@@ -395,8 +419,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             stage = 0;
             phase ^= 1u;
           }
-          if (WS && ++wslot == WS) {
-            wslot = 0;
+          if (WP && ++wpos == WP) {
+            wpos = 0;
             wphase ^= 1u;
           }
         }
@@ -418,7 +442,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     const int row = quad * 32 + lane;
     const bool leader = warp == kEpiWarp0 && lane == 0;
     const uint32_t tag = *tag_slot;
-    const int64_t part_stride = (int64_t)p.tile_n * kBM;
+    const int64_t part_stride = (int64_t)p.tile_n * RU;  // a CTA's partial-sum tile
     int seg = 0;
     int64_t qa = 0;  // index (among this CTA's units) of the segment's first unit
     for (int64_t u = u0; u < u1; ++seg) {
@@ -426,8 +450,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
       const bool split = !(kb0 == 0 && kb1 == KB);
-      const int acc = seg & 1;
-      const uint32_t acc_phase = (uint32_t)(seg >> 1) & 1u;
+      const int acc = p.acc_bufs == 2 ? (seg & 1) : 0;
+      const uint32_t acc_phase = (uint32_t)(p.acc_bufs == 2 ? (seg >> 1) : seg) & 1u;
       // every lane observes the accumulator barrier before reading TMEM; the
       // wait is long (a whole segment), so it sleeps between polls
       const bool got =
@@ -454,54 +478,60 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         }
       }
       const int64_t nt = t / p.MT, mt = t - nt * p.MT;
-      const int64_t n = nt * kBM + row;
       const int64_t m0 = mt * p.tile_n;
       const int cols = (int)imin64(p.tile_n, p.M - m0);
-      // which parity accumulators received MMAs in this segment
+      // which parity accumulators received MMAs in this segment (one half
+      // per unit; in the wide shape each half has its own accumulator)
       const bool has0 = NM == 1 || (kb1 - kb0 >= 2) || ((qa & 1) == 0);
       const bool has1 = NM == 2 && ((kb1 - kb0 >= 2) || ((qa & 1) == 1));
       const uint32_t lanebase = (uint32_t)(quad * 32) << 16;
-      const uint32_t t0 = tmem_base + lanebase + (uint32_t)((acc * NM + 0) * p.tile_n);
-      const uint32_t t1 = tmem_base + lanebase + (uint32_t)((acc * NM + 1) * p.tile_n);
-      float* part = p.partials + (int64_t)blockIdx.x * part_stride;
-      for (int c = 0; c < cols; c += 16) {
-        uint32_t r0[16], r1[16];
-        if (has0) tmem_ld16(t0 + (uint32_t)c, r0);
-        if (has1) tmem_ld16(t1 + (uint32_t)c, r1);
-        tmem_ld_wait();
-        float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v[j] = has0 ? __uint_as_float(r0[j]) : 0.f;
-          if (has1) v[j] += __uint_as_float(r1[j]);
-        }
-        if (split && !owner) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c + j < cols) part[(int64_t)(c + j) * kBM + row] = v[j];
-          continue;
-        }
-        if (split) {
-          // the other CTAs' sums, in K order; a contributor's 16 loads are all
-          // in flight before the first add
-          for (int64_t q = blockIdx.x + 1; q <= last; ++q) {
-            const float* src = p.partials + q * part_stride + (int64_t)c * kBM + row;
-            float pv[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) pv[j] = c + j < cols ? __ldcg(src + j * kBM) : 0.f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += pv[j];
-          }
-        }
-        if (n < p.N) {
+      for (int h = 0; h < H; ++h) {
+        const bool use0 = wide || has0, use1 = !wide && has1;
+        const uint32_t t0 =
+            tmem_base + lanebase + (uint32_t)((acc * NM + (wide ? h : 0)) * p.tile_n);
+        const uint32_t t1 = tmem_base + lanebase + (uint32_t)((acc * NM + 1) * p.tile_n);
+        const int64_t n = nt * RU + h * kBM + row;
+        const int64_t hoff = (int64_t)h * kBM * p.tile_n;  // the half's place in a partial tile
+        float* part = p.partials + (int64_t)blockIdx.x * part_stride + hoff;
+        for (int c = 0; c < cols; c += 16) {
+          uint32_t r0[16], r1[16];
+          if (use0) tmem_ld16(t0 + (uint32_t)c, r0);
+          if (use1) tmem_ld16(t1 + (uint32_t)c, r1);
+          tmem_ld_wait();
+          float v[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            if (c + j < cols) {
-              const int64_t o = (m0 + c + j) * p.N + n;
-              if (p.out_f32)
-                static_cast<float*>(p.Y)[o] = v[j];
-              else
-                static_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(v[j]);
+            v[j] = use0 ? __uint_as_float(r0[j]) : 0.f;
+            if (use1) v[j] += __uint_as_float(r1[j]);
+          }
+          if (split && !owner) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c + j < cols) part[(int64_t)(c + j) * kBM + row] = v[j];
+            continue;
+          }
+          if (split) {
+            // the other CTAs' sums, in K order; a contributor's 16 loads are all
+            // in flight before the first add
+            for (int64_t q = blockIdx.x + 1; q <= last; ++q) {
+              const float* src = p.partials + q * part_stride + hoff + (int64_t)c * kBM + row;
+              float pv[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pv[j] = c + j < cols ? __ldcg(src + j * kBM) : 0.f;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] += pv[j];
+            }
+          }
+          if (n < p.N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (c + j < cols) {
+                const int64_t o = (m0 + c + j) * p.N + n;
+                if (p.out_f32)
+                  static_cast<float*>(p.Y)[o] = v[j];
+                else
+                  static_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(v[j]);
+              }
             }
           }
         }
@@ -521,13 +551,15 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     // ------------------------------------------------------------- rebuild --
     // Two groups of 4 warps take alternate stages (unit q of this CTA goes to
     // group q % 2), so two tiles are rebuilt while the tensor core consumes.
+    // Wide shape: group h rebuilds half h of every unit (W slot 2 j + h).
     const int rt = threadIdx.x - kRebuildWarp0 * 32;  // 0..255
     const int grp = rt >> 7;                           // 0 or 1
     const int gt = rt & 127;                           // thread within the group
+    const int WP = wide ? WS / 2 : WS;
     bool ok = true;
     int q = 0;  // index of the unit among this CTA's units
     // ring positions of unit q, advanced for every unit of the CTA
-    int stage = 0, wslot = 0;
+    int stage = 0, wpos = 0;
     uint32_t phase = 0, wphase = 0;
     for (int64_t u = u0; u < u1 && ok;) {
       const int64_t t = u / KB;
@@ -535,17 +567,17 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
       const int64_t nt = t / p.MT;
       for (int kb = kb0; kb < kb1; ++kb, ++q) {
-        const int cur_stage = stage, cur_wslot = wslot;
+        const int cur_stage = stage, cur_wslot = wide ? 2 * wpos + grp : wpos;
         const uint32_t cur_phase = phase, cur_wphase = wphase;
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
-        if (++wslot == WS) {
-          wslot = 0;
+        if (++wpos == WP) {
+          wpos = 0;
           wphase ^= 1u;
         }
-        if ((q & 1) != grp) continue;
+        if (!wide && (q & 1) != grp) continue;
         // every thread observes the stage's TMA completion before reading it
         const bool got = mbar_wait_bounded(bar(b_full + cur_stage), cur_phase, abort, p.wait_ns) &&
                          mbar_wait_bounded(bar(b_wfree + cur_wslot), cur_wphase ^ 1u, abort, p.wait_ns);
@@ -553,6 +585,13 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         ok = !__any_sync(0xffffffffu, !got);
         if (!ok) break;
         const uint8_t* st = ring + (size_t)cur_stage * L.bytes;
+        // this group's half of the stage: sign+mantissa, exponents or indices,
+        // escape bitmap and rows; its 128-row escape group
+        const int hh = wide ? grp : 0;
+        const uint8_t* sS = st + L.w0 + hh * 8192;
+        const uint8_t* sW1 = st + L.w1 + hh * (MODE == kGemmExp ? 8192 : 4096);
+        const uint8_t* sEsc = st + L.ebits + hh * kEscArea;
+        const int64_t grow = nt * H + hh;
         uint8_t* wt = wring + (size_t)cur_wslot * kWTileBytes;
         // all inputs first (the stores below may alias nothing they read, but
         // the compiler cannot know that), then rebuild and store
@@ -563,11 +602,11 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         for (int i = 0; i < 8; ++i) {
           const int c8 = gt + 128 * i;
           const int r = c8 >> 3, c = c8 & 7;
-          s8[i] = *reinterpret_cast<const uint2*>(st + L.w0 + r * 64 + c * 8);
+          s8[i] = *reinterpret_cast<const uint2*>(sS + r * 64 + c * 8);
           if (MODE == kGemmExp)
-            e8[i] = *reinterpret_cast<const uint2*>(st + L.w1 + r * 64 + c * 8);
+            e8[i] = *reinterpret_cast<const uint2*>(sW1 + r * 64 + c * 8);
           else
-            v4[i] = *reinterpret_cast<const uint32_t*>(st + L.w1 + r * 32 + c * 4);
+            v4[i] = *reinterpret_cast<const uint32_t*>(sW1 + r * 32 + c * 4);
         }
         // every item as if no row were an escape row (no branch in the loop, so
         // the items' dependency chains interleave) ...
@@ -589,7 +628,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         // = escape rows before the row in the tile) overwrite the 16-byte pieces
         // just written.
         uint4 eb4 = make_uint4(0u, 0u, 0u, 0u);
-        if (MODE == kGemmPalette) eb4 = *reinterpret_cast<const uint4*>(st + L.ebits);
+        if (MODE == kGemmPalette) eb4 = *reinterpret_cast<const uint4*>(sEsc);
         const uint32_t warp_rows = 0x000F000Fu << (4 * (gt >> 5));
         if (MODE == kGemmPalette && ((eb4.x | eb4.y | eb4.z | eb4.w) & warp_rows)) {
           const uint32_t eb[4] = {eb4.x, eb4.y, eb4.z, eb4.w};
@@ -611,9 +650,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             const uint32_t slot = before + (uint32_t)__popc(word & ((1u << (r & 31)) - 1u));
             uint2 ex;
             if (slot < (uint32_t)kEscCap) {
-              ex = *reinterpret_cast<const uint2*>(st + L.erows + slot * 64 + c * 8);
+              ex = *reinterpret_cast<const uint2*>(sEsc + 16 + slot * 64 + c * 8);
             } else {
-              const uint32_t first = __ldg(p.esc_off + nt * KB + kb);
+              const uint32_t first = __ldg(p.esc_off + grow * KB + kb);
               ex = __ldg(reinterpret_cast<const uint2*>(p.esc_exp + (int64_t)(first + slot) * 64 +
                                                         c * 8));
             }
@@ -704,8 +743,8 @@ int tmem_cols_for(int tile_n) {
   return c;
 }
 
-size_t smem_bytes(int mode, int tile_n, int stages, int wslots) {
-  const StageLayout L = stage_layout(mode, tile_n);
+size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves) {
+  const StageLayout L = stage_layout(mode, tile_n, halves);
   const int ws = mode == kGemmBf16 ? 0 : wslots;
   size_t b = 1024 /* alignment slack */ + (size_t)stages * L.bytes;
   b += (size_t)ws * kWTileBytes;
@@ -724,18 +763,32 @@ cudaError_t set_smem_attr() {
 
 bool gemm_resolve(GemmArgs* a) {
   if (a->M <= 0 || a->N <= 0 || a->K <= 0 || a->K % kBK) return false;
+  // Wide shape (256 W rows per unit, one 128-row half per rebuild group and
+  // MMA warp) from M = 512 on: X is then read once per 256 rows instead of
+  // 128.  Token tiles: all of M up to 128 tokens, 128 above (measured on
+  // 14336x4096: at M = 256 128-token tiles beat one 256-token tile by 13-16%;
+  // 256-token wide tiles fill TMEM, so an epilogue stalls the next tile).
+  // (The plain BF16 GEMM rebuilds nothing, so for it the wide shape only
+  // trades X traffic for TMEM room: it keeps 128-row units, with one 256-token
+  // tile from M = 512.)
+  if (a->halves == 0) a->halves = (a->mode != kGemmBf16 && a->M >= kWideMinM) ? 2 : 1;
+  if (a->halves != 1 && a->halves != 2) return false;
+  const bool wide = a->halves == 2;
   if (a->tile_n == 0) {
-    const int64_t mt = (a->M + 255) / 256;
-    const int64_t per = (a->M + mt - 1) / mt;
-    a->tile_n = (int)((per + 15) / 16 * 16);
+    if (a->M <= 128)
+      a->tile_n = (int)((a->M + 15) / 16 * 16);
+    else
+      a->tile_n = (a->mode == kGemmBf16 && a->M >= kWideMinM) ? 256 : 128;
   }
   if (a->tile_n < 16 || a->tile_n > 256 || a->tile_n % 16) return false;
-  // Ring depths are even: consumers alternate units, so an even depth keeps
-  // every slot with one consumer (see the MMA issuers in the kernel).
+  // One half per unit: ring depths are even, consumers alternate units, so an
+  // even depth keeps every slot with one consumer (see the MMA issuers).  Wide:
+  // every consumer takes every stage, any depth works; W slots go in pairs.
   // As many load stages as fit (up to kMaxStages) beside four rebuilt-W slots
   // (two per rebuild group: with one, a group's next rebuild waits for its
   // last tile's MMA).
   const int max_stages = a->mode == kGemmBf16 ? 12 : kMaxStages;
+  const int step = wide ? 1 : 2;
   if (a->wslots == 0) a->wslots = a->mode == kGemmBf16 ? 0 : 4;
   if (a->mode != kGemmBf16 &&
       (a->wslots < 2 || a->wslots > kMaxWSlots || (a->wslots & 1)))
@@ -743,18 +796,21 @@ bool gemm_resolve(GemmArgs* a) {
   if (a->stages == 0) {
     for (;;) {
       int s = max_stages;
-      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots) > (size_t)kSmemLimit) s -= 2;
-      if (smem_bytes(a->mode, a->tile_n, s, a->wslots) <= (size_t)kSmemLimit || a->wslots <= 2) {
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves) > (size_t)kSmemLimit)
+        s -= step;
+      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves) <= (size_t)kSmemLimit ||
+          a->wslots <= 2 || wide) {
         a->stages = s;
         break;
       }
       a->wslots -= 2;
     }
   }
-  if (a->stages < 2 || (a->stages & 1) ||
-      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots) > (size_t)kSmemLimit)
+  if (a->stages < 2 || (!wide && (a->stages & 1)) ||
+      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves) > (size_t)kSmemLimit)
     return false;
-  const int64_t NT = (a->N + kBM - 1) / kBM;
+  const int64_t RU = (int64_t)kBM * a->halves;
+  const int64_t NT = (a->N + RU - 1) / RU;
   const int64_t MT = (a->M + a->tile_n - 1) / a->tile_n;
   const int64_t units = NT * MT * (a->K / kBK);
   int ctas = a->ctas > 0 ? a->ctas : a->sm_count;
@@ -767,29 +823,31 @@ bool gemm_resolve(GemmArgs* a) {
 // One partial-sum tile per CTA: a CTA hands over at most one (the split tile
 // its range starts in, when it does not hold that tile's first K block).
 size_t gemm_partials_bytes(const GemmArgs& a) {
-  return (size_t)a.ctas * (size_t)a.tile_n * kBM * sizeof(float);
+  return (size_t)a.ctas * (size_t)a.tile_n * kBM * (a.halves == 2 ? 2 : 1) * sizeof(float);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* hooks) {
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int64_t KB = a.K / kBK;
+  const bool wide = a.halves == 2;
+  const uint32_t RU = (uint32_t)kBM * (wide ? 2 : 1);
   if (!make_map_2d(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.K,
                    (uint64_t)a.M, kBK, (uint32_t)a.tile_n, true))
     return cudaErrorInvalidValue;
   bool ok = true;
   if (a.mode == kGemmBf16) {
     ok = make_map_2d(&p.tm_w0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.W, (uint64_t)a.K,
-                     (uint64_t)a.N, kBK, kBM, true);
+                     (uint64_t)a.N, kBK, RU, true);
   } else {
     ok = make_map_2d(&p.tm_w0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.S, (uint64_t)a.K,
-                     (uint64_t)a.N, kBK, kBM, false);
+                     (uint64_t)a.N, kBK, RU, false);
     if (ok && a.mode == kGemmExp)
       ok = make_map_2d(&p.tm_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.E, (uint64_t)a.K,
-                       (uint64_t)a.N, kBK, kBM, false);
+                       (uint64_t)a.N, kBK, RU, false);
     if (ok && a.mode == kGemmPalette)
       ok = make_map_2d(&p.tm_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.I, (uint64_t)a.K / 2,
-                       (uint64_t)a.N, kBK / 2, kBM, false);
+                       (uint64_t)a.N, kBK / 2, RU, false);
   }
   if (!ok) return cudaErrorInvalidValue;
   p.esc_bits = a.esc_bits;
@@ -807,19 +865,22 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.tile_n = a.tile_n;
   p.stages = a.stages;
   p.wslots = a.wslots;
-  p.NT = (int32_t)((a.N + kBM - 1) / kBM);
+  p.NT = (int32_t)((a.N + RU - 1) / RU);
+  p.NG = (int32_t)((a.N + kBM - 1) / kBM);
+  p.halves = wide ? 2 : 1;
   p.MT = (int32_t)((a.M + a.tile_n - 1) / a.tile_n);
   p.KB = (int32_t)KB;
   p.units = (int64_t)p.NT * p.MT * KB;
   p.esc_nwp = a.esc_nw;
   p.out_f32 = a.out_f32;
-  p.n_mma = mma_warps_for(a.tile_n);
-  p.tmem_cols = tmem_cols_for(a.tile_n);
+  p.n_mma = wide ? 2 : mma_warps_for(a.tile_n);
+  p.tmem_cols = wide ? 512 : tmem_cols_for(a.tile_n);
+  p.acc_bufs = (!wide || 4 * a.tile_n <= 512) ? 2 : 1;  // TMEM: bufs x NM x tile_n columns
   std::memcpy(p.palette, a.palette, 16);
   p.x_bytes = (uint32_t)a.tile_n * kBK * 2;
-  p.stage_bytes = stage_layout(a.mode, a.tile_n).bytes;
+  p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves).bytes;
   p.wait_ns = wait_limit_ns();
-  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots);
+  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves);
   const int G = a.ctas;
   cudaError_t e = cudaSuccess;
   auto begin = [&](int kind) { return hooks && hooks->begin ? hooks->begin(hooks->ctx, kind) : -1; };

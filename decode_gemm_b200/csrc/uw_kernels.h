@@ -80,6 +80,7 @@ struct GemmArgs {
   size_t partials_bytes = 0;
   uint32_t* sync = nullptr;      // kGemmSyncWords words, zeroed before first use
   int tile_n = 0;                // tokens per tile (0 = auto)
+  int halves = 0;                // W rows per unit / 128: 1, 2 (wide), 0 = auto by M
   int stages = 0;                // load ring depth (0 = auto)
   int wslots = 0;                // rebuilt-W ring depth (0 = auto)
   int ctas = 0;                  // persistent CTAs (0 = SM count)

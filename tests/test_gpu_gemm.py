@@ -239,3 +239,28 @@ def test_odd_ring_depth_rejected(uw):
         assert uw.lib.uw_gemm_ex(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 4,
                                  C.byref(cfg), 0) == uw.UW_ERR_ARG
     h.free()
+
+
+WIDE_SHAPES = [
+    # (M, N, K, weight maker): units of 256 W rows, one 128-row half per rebuild
+    # group and MMA warp
+    (1, 512, 512, "normal"),
+    (17, 200, 192, "student_t"),    # N < 256: the second half partly past N
+    (40, 128, 256, "student_t"),    # the second half entirely past N
+    (130, 640, 640, "normal"),      # two token tiles, ragged N
+]
+
+
+@pytest.mark.parametrize("M,N,K,kind", WIDE_SHAPES)
+@pytest.mark.parametrize("pipe", PIPES)
+@pytest.mark.parametrize("tile_n", [0, 256])
+def test_wide_units_match_fp64(uw, M, N, K, kind, pipe, tile_n):
+    """The 256-row unit shape (automatic from M = 512) on small shapes."""
+    w = _weights(kind, N, K, seed=80 + M)
+    x = synthdata.activations(M, K, seed=81 + N)
+    h = _upload(uw, w, chunk=128)
+    ws = _workspace(uw, h, M)
+    for ctas in (0, 7):  # one CTA per SM, or a few so tiles split between CTAs
+        y = _gemm(uw, h, x, pipe, halves=2, tile_n=tile_n, gemm_ctas=ctas)
+        _check(y, x, w)
+    h.free()
