@@ -94,6 +94,8 @@ struct GemmParams {
   int32_t halves;    // 128-row halves per unit: 1, or 2 for the wide (large-M) shape
   int32_t acc_bufs;  // TMEM accumulator sets (2: epilogue overlaps the next tile)
   int32_t NG;        // 128-row groups of W (escape groups per K block)
+  int32_t tmem_w;    // W slots in TMEM (MMA A from TMEM) rather than shared memory
+  uint32_t wcol0;    // first TMEM column of the W slots
   uint32_t palette[4];
   uint32_t stage_bytes, x_bytes;
   uint64_t wait_ns;
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   const int RU = kBM * H;  // W rows per unit
   uint8_t* ring = smem;
   uint8_t* wring = ring + (size_t)S * L.bytes;  // rebuilt W tiles (reconstructive modes)
-  uint8_t* tail = wring + (size_t)WS * kWTileBytes;
+  uint8_t* tail = wring + (size_t)(p.tmem_w ? 0 : WS) * kWTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   // barrier indices
   const int b_full = 0, b_empty = S, b_wfull = 2 * S, b_wfree = 2 * S + WS,
@@ -269,13 +271,43 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
+    // palette escape offsets of the next 32 units, one unit per lane, loaded
+    // together (a load per stage would put its latency on the issue path)
+    uint32_t lc0[2] = {0u, 0u}, lc1[2] = {0u, 0u};
+    int qi = 0;  // index of the unit among this CTA's units
     for (int64_t u = u0; u < u1 && ok;) {
       const int64_t t = u / KB;
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
       const int64_t nt = t / p.MT, mt = t - nt * p.MT;
       const int32_t n0 = (int32_t)(nt * RU), m0 = (int32_t)(mt * p.tile_n);
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb, ++qi) {
+        uint32_t c0[2] = {0u, 0u}, c1[2] = {0u, 0u};
+        if (MODE == kGemmPalette) {
+          if ((qi & 31) == 0) {
+            const int64_t uu = u0 + qi + lane;
+            lc0[0] = lc0[1] = lc1[0] = lc1[1] = 0u;
+            if (uu < u1) {
+              const int64_t tt = uu / KB;
+              const int64_t kk = uu - tt * KB;
+              const int64_t g0 = (tt / p.MT) * H;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                if (h >= H) break;
+                if (g0 + h < p.NG) {
+                  const int64_t gi = (g0 + h) * KB + kk;
+                  lc0[h] = __ldg(p.esc_off + gi);
+                  lc1[h] = __ldg(p.esc_off + gi + 1);
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            c0[h] = __shfl_sync(0xffffffffu, lc0[h], qi & 31);
+            c1[h] = __shfl_sync(0xffffffffu, lc1[h], qi & 31);
+          }
+        }
         if (lane == 0) {
           if (!mbar_wait_bounded(bar(b_empty + stage), phase ^ 1u, abort, p.wait_ns)) {
             set_abort(abort, p.status);
@@ -288,21 +320,16 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             if (MODE == kGemmExp) bytes += H * 16384;
             // escape rows of each half's group (128 rows, this K block): one
             // copy of its bitmap and first rows, or none and a zero bitmap
-            uint32_t c0[2] = {0u, 0u}, nesc[2] = {0u, 0u};
+            uint32_t nesc[2] = {0u, 0u};
             bool has[2] = {false, false};
             if (MODE == kGemmPalette) {
               bytes += H * 12288;
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 if (h >= H) break;
-                const int64_t grow = nt * H + h;  // 128-row group
-                if (grow < p.NG) {
-                  const int64_t gi = grow * KB + kb;
-                  c0[h] = __ldg(p.esc_off + gi);
-                  const uint32_t c1 = __ldg(p.esc_off + gi + 1);
-                  has[h] = c1 > c0[h];
-                  nesc[h] = min(c1 - c0[h], (uint32_t)kEscCap);
-                }
+                // 128-row group nt * H + h (past the last group: no escapes)
+                has[h] = c1[h] > c0[h];
+                nesc[h] = min(c1[h] - c0[h], (uint32_t)kEscCap);
                 if (has[h]) {
                   bytes += 16 + nesc[h] * 64;
                 } else {
@@ -399,15 +426,24 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             } else {
               tc_fence_after();
               uint8_t* st = ring + (size_t)stage * L.bytes;
-              const uint32_t a_addr =
-                  MODE == kGemmBf16 ? smem_u32(st + L.w0 + (wide ? par * kWTileBytes : 0))
-                                    : smem_u32(wring + (size_t)wslot * kWTileBytes);
-              const uint64_t a_desc = smem_desc_sw128(a_addr);
               const uint64_t b_desc = smem_desc_sw128(smem_u32(st + L.x));
+              if (MODE != kGemmBf16 && p.tmem_w) {
+                // A: 32 columns of the slot, 8 per 16-wide K step
+                const uint32_t a_tmem = tmem_base + p.wcol0 + (uint32_t)(wslot * 32);
 #pragma unroll
-              for (int k = 0; k < kBK / 16; ++k)
-                mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
-                         (!first || k > 0) ? 1u : 0u);
+                for (int k = 0; k < kBK / 16; ++k)
+                  mma_bf16_tmem_a(d_tmem, a_tmem + 8 * k, b_desc + 2 * k, idesc,
+                                  (!first || k > 0) ? 1u : 0u);
+              } else {
+                const uint32_t a_addr =
+                    MODE == kGemmBf16 ? smem_u32(st + L.w0 + (wide ? par * kWTileBytes : 0))
+                                      : smem_u32(wring + (size_t)wslot * kWTileBytes);
+                const uint64_t a_desc = smem_desc_sw128(a_addr);
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                  mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
+                           (!first || k > 0) ? 1u : 0u);
+              }
               mma_commit(bar(b_empty + stage));
               if (MODE != kGemmBf16) mma_commit(bar(b_wfree + wslot));
             }
@@ -592,6 +628,78 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         const uint8_t* sW1 = st + L.w1 + hh * (MODE == kGemmExp ? 8192 : 4096);
         const uint8_t* sEsc = st + L.ebits + hh * kEscArea;
         const int64_t grow = nt * H + hh;
+        if (p.tmem_w) {
+          // One W row per thread: row r (TMEM lane r, the warp's quadrant)
+          // gets the K block's 64 weights in 32 columns of the slot.  S and E
+          // rows were staged with the 64-byte swizzle, I rows with the 32-byte
+          // one, so a quarter-warp's 16-byte reads hit distinct banks.
+          const int r = 32 * (warp & 3) + lane;
+          uint4 sv[4], ev[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            sv[k] = *reinterpret_cast<const uint4*>(sS + r * 64 + ((k ^ ((r >> 1) & 3)) << 4));
+          if (MODE == kGemmExp) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              ev[k] = *reinterpret_cast<const uint4*>(sW1 + r * 64 + ((k ^ ((r >> 1) & 3)) << 4));
+          } else {
+            const uint4 i0 = *reinterpret_cast<const uint4*>(sW1 + r * 32 + ((0 ^ ((r >> 2) & 1)) << 4));
+            const uint4 i1 = *reinterpret_cast<const uint4*>(sW1 + r * 32 + ((1 ^ ((r >> 2) & 1)) << 4));
+            const uint32_t iw[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+            uint32_t ew[16];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint2 e = palette8(iw[j], p.palette[0], p.palette[1], p.palette[2], p.palette[3]);
+              ew[2 * j] = e.x;
+              ew[2 * j + 1] = e.y;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              ev[k] = make_uint4(ew[4 * k], ew[4 * k + 1], ew[4 * k + 2], ew[4 * k + 3]);
+            // escape rows take their verbatim exponents (slot = escape rows
+            // before the row in the 128-row group); the warp's 32 rows are one
+            // word of the bitmap
+            const uint4 eb4 = *reinterpret_cast<const uint4*>(sEsc);
+            const int wq = warp & 3;
+            const uint32_t word = wq == 0 ? eb4.x : wq == 1 ? eb4.y : wq == 2 ? eb4.z : eb4.w;
+            if ((word >> lane) & 1u) {
+              const uint32_t before = (wq > 0 ? __popc(eb4.x) : 0) + (wq > 1 ? __popc(eb4.y) : 0) +
+                                      (wq > 2 ? __popc(eb4.z) : 0);
+              const uint32_t slot = before + (uint32_t)__popc(word & ((1u << lane) - 1u));
+              const uint4* src;
+              if (slot < (uint32_t)kEscCap) {
+                src = reinterpret_cast<const uint4*>(sEsc + 16 + slot * 64);
+              } else {
+                const uint32_t first = __ldg(p.esc_off + grow * KB + kb);
+                src = reinterpret_cast<const uint4*>(p.esc_exp + (int64_t)(first + slot) * 64);
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) ev[k] = src[k];
+            }
+          }
+          // the stage's inputs are in registers: release it
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(b_empty + cur_stage));
+          const uint32_t* s32 = reinterpret_cast<const uint32_t*>(sv);
+          const uint32_t* e32 = reinterpret_cast<const uint32_t*>(ev);
+          uint32_t wv[32];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const uint2 m = merge4(s32[j], e32[j]);
+            wv[2 * j] = m.x;
+            wv[2 * j + 1] = m.y;
+          }
+          // after the slot's previous MMAs (observed through its free barrier)
+          tc_fence_after();
+          tmem_st32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + p.wcol0 +
+                        (uint32_t)(cur_wslot * 32),
+                    wv);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(b_wfull + cur_wslot));
+          continue;
+        }
         uint8_t* wt = wring + (size_t)cur_wslot * kWTileBytes;
         // all inputs first (the stores below may alias nothing they read, but
         // the compiler cannot know that), then rebuild and store
@@ -713,7 +821,7 @@ EncodeTiledFn encode_fn() {
 
 bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base,
                  uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
-                 bool swizzle128) {
+                 CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -721,8 +829,7 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const v
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -737,14 +844,24 @@ uint64_t wait_limit_ns() {
 
 int mma_warps_for(int tile_n) { return tile_n <= 128 ? 2 : 1; }
 
-int tmem_cols_for(int tile_n) {
+// TMEM columns: two accumulator sets, then (TMEM path) 32 columns per W slot.
+int tmem_cols_for(int tile_n, int wslots_in_tmem) {
   int c = 32;
-  while (c < 2 * mma_warps_for(tile_n) * tile_n) c *= 2;
+  while (c < 2 * mma_warps_for(tile_n) * tile_n + 32 * wslots_in_tmem) c *= 2;
   return c;
 }
 
-size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves) {
+// Reconstructive modes with one half per unit and token tiles up to 64 rebuild
+// W into TMEM (the MMA reads A from there): it frees the shared-memory W ring
+// for load stages.
+bool tmem_w_for(const GemmArgs& a) {
+  return a.mode != kGemmBf16 && a.halves == 1 &&
+         2 * mma_warps_for(a.tile_n) * a.tile_n + 32 * a.wslots <= 512;
+}
+
+size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool tmem_w) {
   const StageLayout L = stage_layout(mode, tile_n, halves);
+  if (tmem_w) wslots = 0;  // the W slots live in TMEM
   const int ws = mode == kGemmBf16 ? 0 : wslots;
   size_t b = 1024 /* alignment slack */ + (size_t)stages * L.bytes;
   b += (size_t)ws * kWTileBytes;
@@ -796,9 +913,9 @@ bool gemm_resolve(GemmArgs* a) {
   if (a->stages == 0) {
     for (;;) {
       int s = max_stages;
-      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves) > (size_t)kSmemLimit)
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, tmem_w_for(*a)) > (size_t)kSmemLimit)
         s -= step;
-      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves) <= (size_t)kSmemLimit ||
+      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, tmem_w_for(*a)) <= (size_t)kSmemLimit ||
           a->wslots <= 2 || wide) {
         a->stages = s;
         break;
@@ -807,7 +924,7 @@ bool gemm_resolve(GemmArgs* a) {
     }
   }
   if (a->stages < 2 || (!wide && (a->stages & 1)) ||
-      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves) > (size_t)kSmemLimit)
+      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, tmem_w_for(*a)) > (size_t)kSmemLimit)
     return false;
   const int64_t RU = (int64_t)kBM * a->halves;
   const int64_t NT = (a->N + RU - 1) / RU;
@@ -832,22 +949,27 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   const int64_t KB = a.K / kBK;
   const bool wide = a.halves == 2;
   const uint32_t RU = (uint32_t)kBM * (wide ? 2 : 1);
+  const bool tw = tmem_w_for(a);
   if (!make_map_2d(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.K,
-                   (uint64_t)a.M, kBK, (uint32_t)a.tile_n, true))
+                   (uint64_t)a.M, kBK, (uint32_t)a.tile_n, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   bool ok = true;
   if (a.mode == kGemmBf16) {
     ok = make_map_2d(&p.tm_w0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.W, (uint64_t)a.K,
-                     (uint64_t)a.N, kBK, RU, true);
+                     (uint64_t)a.N, kBK, RU, CU_TENSOR_MAP_SWIZZLE_128B);
   } else {
+    // rows rebuilt one per thread (TMEM path) are read 16 bytes at a time
+    // along the row: 64- and 32-byte swizzles spread a warp's rows over the banks
+    const CUtensorMapSwizzle sw64 = tw ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const CUtensorMapSwizzle sw32 = tw ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
     ok = make_map_2d(&p.tm_w0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.S, (uint64_t)a.K,
-                     (uint64_t)a.N, kBK, RU, false);
+                     (uint64_t)a.N, kBK, RU, sw64);
     if (ok && a.mode == kGemmExp)
       ok = make_map_2d(&p.tm_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.E, (uint64_t)a.K,
-                       (uint64_t)a.N, kBK, RU, false);
+                       (uint64_t)a.N, kBK, RU, sw64);
     if (ok && a.mode == kGemmPalette)
       ok = make_map_2d(&p.tm_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.I, (uint64_t)a.K / 2,
-                       (uint64_t)a.N, kBK / 2, RU, false);
+                       (uint64_t)a.N, kBK / 2, RU, sw32);
   }
   if (!ok) return cudaErrorInvalidValue;
   p.esc_bits = a.esc_bits;
@@ -874,13 +996,15 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.esc_nwp = a.esc_nw;
   p.out_f32 = a.out_f32;
   p.n_mma = wide ? 2 : mma_warps_for(a.tile_n);
-  p.tmem_cols = wide ? 512 : tmem_cols_for(a.tile_n);
+  p.tmem_cols = wide ? 512 : tmem_cols_for(a.tile_n, tw ? a.wslots : 0);
+  p.tmem_w = tw ? 1 : 0;
+  p.wcol0 = (uint32_t)(2 * mma_warps_for(a.tile_n) * a.tile_n);
   p.acc_bufs = (!wide || 4 * a.tile_n <= 512) ? 2 : 1;  // TMEM: bufs x NM x tile_n columns
   std::memcpy(p.palette, a.palette, 16);
   p.x_bytes = (uint32_t)a.tile_n * kBK * 2;
   p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves).bytes;
   p.wait_ns = wait_limit_ns();
-  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves);
+  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw);
   const int G = a.ctas;
   cudaError_t e = cudaSuccess;
   auto begin = [&](int kind) { return hooks && hooks->begin ? hooks->begin(hooks->ctx, kind) : -1; };
