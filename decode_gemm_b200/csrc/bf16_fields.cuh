@@ -35,4 +35,50 @@ __device__ __forceinline__ uint2 palette8(uint32_t v, uint32_t p0, uint32_t p1, 
   return make_uint2(__byte_perm(lo0, hi0, pick), __byte_perm(lo1, hi1, pick >> 16));
 }
 
+// PTX prmt in its default mode: a selector nibble with bit 3 set fills the
+// byte with the sign bit of the byte it selects (the CUDA intrinsic
+// __byte_perm ignores that bit).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Packed-index word order.  The decoder's stage holds 8 indices per word in
+// element order (nibble t = element t); the stored form interleaves them:
+// element 2t at bits 4t, element 2t+1 at bits 16+4t, so each 16-bit half holds
+// one index of every BF16 pair, in the pair's own lane.
+__device__ __forceinline__ uint32_t nibbles_interleave(uint32_t v) {
+  const uint32_t ev = v & 0x0F0F0F0Fu, od = (v >> 4) & 0x0F0F0F0Fu;
+  // byte 0 of (x | x >> 4) = nibbles 0 and 2 of the group, byte 2 = 4 and 6
+  return __byte_perm(ev | (ev >> 4), od | (od >> 4), 0x6420);
+}
+
+// Eight BF16 weights (four pair words, element order) from one interleaved
+// index word v and their sign+mantissa bytes (s0: elements 0-3, s1: 4-7),
+// for a palette that is the run base..base+15: the exponent is base + index,
+// so a pair's exponent fields are (index << 7) + bias, bias = base * 128 in
+// both halves.  The sign moves from bit 7 to bit 15 of each half by prmt's
+// sign replication.
+__device__ __forceinline__ uint4 rebuild8_run(uint32_t v, uint32_t s0, uint32_t s1,
+                                              uint32_t bias) {
+  const uint32_t m = 0x807F807Fu;  // sign and mantissa bits of a pair
+  const uint32_t x0 = (v & 0x000F000Fu) * 128u + bias;
+  const uint32_t x1 = (v & 0x00F000F0u) * 8u + bias;
+  const uint32_t x2 = __umulhi(v & 0x0F000F00u, 0x80000000u) + bias;  // >> 1
+  const uint32_t x3 = __umulhi(v & 0xF000F000u, 0x08000000u) + bias;  // >> 5
+  return make_uint4(x0 | (prmt(s0, 0u, 0x9180u) & m), x1 | (prmt(s0, 0u, 0xB3A2u) & m),
+                    x2 | (prmt(s1, 0u, 0x9180u) & m), x3 | (prmt(s1, 0u, 0xB3A2u) & m));
+}
+
+// The same for any palette (p0..p3: entries 0..15 in byte order): exponents
+// by lookup, put back in element order, then merged.
+__device__ __forceinline__ uint4 rebuild8_lut(uint32_t v, uint32_t s0, uint32_t s1, uint32_t p0,
+                                              uint32_t p1, uint32_t p2, uint32_t p3) {
+  const uint2 e = palette8(v, p0, p1, p2, p3);  // exponents of elements 0 2 4 6 | 1 3 5 7
+  const uint2 lo = merge4(s0, __byte_perm(e.x, e.y, 0x5140));
+  const uint2 hi = merge4(s1, __byte_perm(e.x, e.y, 0x7362));
+  return make_uint4(lo.x, lo.y, hi.x, hi.y);
+}
+
 }  // namespace uw

@@ -395,7 +395,10 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
           const bool esc =
               (ld_u32_if(a.esc_bits + (int64_t)kb * a.esc_nw + (n >> 5), valid) >> (n & 31)) & 1u;
           const uint32_t* sw = stage + j * kStageStride + 4 * m;
-          const uint4 v = esc ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(sw[0], sw[1], sw[2], sw[3]);
+          // stored word order: element 2t at bits 4t, 2t+1 at bits 16+4t
+          const uint4 v = esc ? make_uint4(0u, 0u, 0u, 0u)
+                              : make_uint4(nibbles_interleave(sw[0]), nibbles_interleave(sw[1]),
+                                           nibbles_interleave(sw[2]), nibbles_interleave(sw[3]));
           st_v4_if(base + o / 2, v, valid);
         }
       }

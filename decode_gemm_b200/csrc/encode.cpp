@@ -16,7 +16,10 @@
 //   * stream = codes of E in row-major order, MSB first, bit p in bit 31-p%32 of
 //     32-bit word p/32, zero padded to 16 bytes; chunk c starts at chunk_off[c];
 //   * palette = top 16 by (count desc, value asc), padded with the smallest
-//     absent byte values; escape rows grouped by (n/128, kb).
+//     absent byte values, then sorted ascending (a run b..b+15 then has index
+//     e - b); escape rows grouped by (n/128, kb);
+//   * packed indices: 8 per little-endian 32-bit word, element 2t at bits 4t,
+//     element 2t+1 at bits 16+4t (each half-word feeds one lane of a BF16 pair).
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -300,7 +303,8 @@ uw_status encode_host(const uint16_t* w, int64_t N, int64_t K, const uw_encode_o
       if (nb > 0) or_word(&words[wi], (uint32_t)(buf << (32 - nb)));
     });
 
-    // palette: count descending, value ascending; pad with the smallest absent values
+    // palette: the first 16 by count descending, value ascending; pad with the
+    // smallest absent values; stored ascending
     std::vector<int> order;
     for (int s = 0; s < 256; ++s)
       if (e.hist[s] > 0) order.push_back(s);
@@ -315,6 +319,7 @@ uw_status encode_host(const uint16_t* w, int64_t N, int64_t K, const uw_encode_o
         order.push_back(v);
         used[v] = true;
       }
+    std::sort(order.begin(), order.end());
     for (int i = 0; i < 16; ++i) e.palette[i] = (uint8_t)order[i];
     bool in_pal[256] = {false};
     for (int i = 0; i < 16; ++i) in_pal[e.palette[i]] = true;

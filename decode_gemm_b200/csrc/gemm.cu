@@ -90,12 +90,17 @@ struct GemmParams {
   uint32_t* sync;     // [0] epoch, [1] exited CTAs, [2 + cta] ready flags
   int64_t M, N, K;
   int64_t units;      // output tiles * K blocks
-  int32_t tile_n, stages, wslots, n_mma, NT, MT, KB, esc_nwp, out_f32, tmem_cols;
+  int32_t tile_n, stages, wslots, n_mma, NT, MT, esc_nwp, out_f32, tmem_cols;
+  int32_t KB;        // units along K (K blocks / ks)
+  int32_t KBK;       // 64-wide K blocks
+  int32_t ks;        // K blocks per unit (stage): 1, or 2 on the TMEM path
   int32_t halves;    // 128-row halves per unit: 1, or 2 for the wide (large-M) shape
   int32_t acc_bufs;  // TMEM accumulator sets (2: epilogue overlaps the next tile)
   int32_t NG;        // 128-row groups of W (escape groups per K block)
   int32_t tmem_w;    // W slots in TMEM (MMA A from TMEM) rather than shared memory
   uint32_t wcol0;    // first TMEM column of the W slots
+  int32_t pal_run;   // palette is the run base..base+15 (index = exponent - base)
+  uint32_t pal_bias; // base * 128 in both 16-bit halves
   uint32_t palette[4];
   uint32_t stage_bytes, x_bytes;
   uint64_t wait_ns;
@@ -106,29 +111,31 @@ struct StageLayout {
   uint32_t x, w0, w1, ebits, erows, bytes;
 };
 
-// A unit's H 128-row halves lie back to back in each region (the TMA boxes
-// cover all H*128 rows at once); palette escape data is per half: a 16-byte
+// A stage holds ks X tiles (one per K block), then the unit's W data: the TMA
+// boxes cover all H*128 rows and ks K blocks at once (row-major inside a box,
+// 64*ks sign+mantissa or exponent bytes, 32*ks index bytes per row).  Palette
+// escape data has one area per (half, K block) part (H * ks <= 2): a 16-byte
 // bitmap, then up to kEscCap rows (kEscArea bytes).
 constexpr uint32_t kEscArea = 16 + kEscCap * 64;
 
-__host__ __device__ inline StageLayout stage_layout(int mode, int tile_n, int halves) {
+__host__ __device__ inline StageLayout stage_layout(int mode, int tile_n, int halves, int ks) {
   StageLayout L;
   L.x = 0;
   const uint32_t xb = (uint32_t)tile_n * kBK * 2;  // multiple of 2048 for tile_n % 16 == 0
-  const uint32_t H = (uint32_t)halves;
-  L.w0 = xb;
+  const uint32_t HK = (uint32_t)(halves * ks);      // 128x64 W blocks per stage
+  L.w0 = (uint32_t)ks * xb;
   if (mode == kGemmBf16) {
-    L.w1 = L.ebits = L.erows = xb + H * kWTileBytes;
-    L.bytes = xb + H * kWTileBytes;
+    L.w1 = L.ebits = L.erows = L.w0 + HK * kWTileBytes;
+    L.bytes = L.w0 + HK * kWTileBytes;
   } else if (mode == kGemmExp) {
-    L.w1 = xb + H * 8192;
-    L.ebits = L.erows = xb + H * 16384;
-    L.bytes = xb + H * 16384;
+    L.w1 = L.w0 + HK * 8192;
+    L.ebits = L.erows = L.w0 + HK * 16384;
+    L.bytes = L.w0 + HK * 16384;
   } else {
-    L.w1 = xb + H * 8192;
-    L.ebits = xb + H * 12288;  // half h: bitmap at ebits + h*kEscArea, rows 16 bytes on
+    L.w1 = L.w0 + HK * 8192;
+    L.ebits = L.w0 + HK * 12288;  // part p: bitmap at ebits + p*kEscArea, rows 16 bytes on
     L.erows = L.ebits + 16;
-    L.bytes = L.ebits + H * kEscArea;
+    L.bytes = L.ebits + HK * kEscArea;
   }
   L.bytes = (L.bytes + 1023) / 1024 * 1024;
   return L;
@@ -194,14 +201,16 @@ __device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t tag, vo
   }
 }
 
-template <int MODE>
+// KS_: K blocks per unit (compile time, so the per-block loops unroll); it
+// equals p.ks.
+template <int MODE, int KS_>
 __global__ void __launch_bounds__(threads_for(MODE), 1)
     gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned, by an offset into the shared array (the accesses stay
   // shared-window loads and stores)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const StageLayout L = stage_layout(MODE, p.tile_n, p.halves);
+  const StageLayout L = stage_layout(MODE, p.tile_n, p.halves, p.ks);
   const int S = p.stages;
   const int WS = MODE == kGemmBf16 ? 0 : p.wslots;
   // MMA-issuing warps: with one half per unit they split the units by parity
@@ -263,7 +272,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   const int64_t G = gridDim.x;
   const int64_t u0 = unit_begin(blockIdx.x, p.units, G);
   const int64_t u1 = unit_begin(blockIdx.x + 1, p.units, G);
-  const int KB = p.KB;
+  const int KB = p.KB;    // units along K
+  constexpr int KS = KS_;  // K blocks per unit
+  const int NP = H * KS;  // escape parts per stage: (half, K block) pairs, at most 2
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
@@ -292,12 +303,14 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
               const int64_t kk = uu - tt * KB;
               const int64_t g0 = (tt / p.MT) * H;
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                if (h >= H) break;
-                if (g0 + h < p.NG) {
-                  const int64_t gi = (g0 + h) * KB + kk;
-                  lc0[h] = __ldg(p.esc_off + gi);
-                  lc1[h] = __ldg(p.esc_off + gi + 1);
+              for (int q = 0; q < 2; ++q) {
+                if (q >= NP) break;
+                // part q: half q / KS, K block kk * KS + q % KS
+                const int64_t g = g0 + q / KS;
+                if (g < p.NG) {
+                  const int64_t gi = g * p.KBK + kk * KS + q % KS;
+                  lc0[q] = __ldg(p.esc_off + gi);
+                  lc1[q] = __ldg(p.esc_off + gi + 1);
                 }
               }
             }
@@ -315,43 +328,47 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           } else {
             uint8_t* st = ring + (size_t)stage * L.bytes;
             const uint32_t fb = bar(b_full + stage);
-            uint32_t bytes = p.x_bytes;
-            if (MODE == kGemmBf16) bytes += H * kWTileBytes;
-            if (MODE == kGemmExp) bytes += H * 16384;
-            // escape rows of each half's group (128 rows, this K block): one
-            // copy of its bitmap and first rows, or none and a zero bitmap
+            uint32_t bytes = p.x_bytes * KS;
+            if (MODE == kGemmBf16) bytes += NP * kWTileBytes;
+            if (MODE == kGemmExp) bytes += NP * 16384;
+            // escape rows of each part's 128-row group and K block: one copy of
+            // its bitmap and first rows, or none and a zero bitmap
             uint32_t nesc[2] = {0u, 0u};
             bool has[2] = {false, false};
             if (MODE == kGemmPalette) {
-              bytes += H * 12288;
+              bytes += NP * 12288;
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                if (h >= H) break;
-                // 128-row group nt * H + h (past the last group: no escapes)
-                has[h] = c1[h] > c0[h];
-                nesc[h] = min(c1[h] - c0[h], (uint32_t)kEscCap);
-                if (has[h]) {
-                  bytes += 16 + nesc[h] * 64;
+              for (int q = 0; q < 2; ++q) {
+                if (q >= NP) break;
+                // (past the last group: no escapes)
+                has[q] = c1[q] > c0[q];
+                nesc[q] = min(c1[q] - c0[q], (uint32_t)kEscCap);
+                if (has[q]) {
+                  bytes += 16 + nesc[q] * 64;
                 } else {
                   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
-                                   smem_u32(st + L.ebits + h * kEscArea)),
+                                   smem_u32(st + L.ebits + q * kEscArea)),
                                "r"(0u)
                                : "memory");
                 }
               }
             }
             mbar_expect_tx(fb, bytes);
-            tma_load_2d(smem_u32(st + L.x), &p.tm_x, fb, kb * kBK, m0);
-            tma_load_2d(smem_u32(st + L.w0), &p.tm_w0, fb, kb * kBK, n0);
-            if (MODE == kGemmExp) tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kb * kBK, n0);
-            if (MODE == kGemmPalette) {
-              tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kb * (kBK / 2), n0);
+            const int kbk = kb * KS;  // first K block of the unit
 #pragma unroll
-              for (int h = 0; h < 2; ++h)
-                if (h < H && has[h])
-                  bulk_load(smem_u32(st + L.ebits + h * kEscArea),
-                            p.esc_pack + 16 * ((nt * H + h) * KB + kb) + (int64_t)c0[h] * 64,
-                            16 + nesc[h] * 64, fb);
+            for (int j = 0; j < KS; ++j)
+              tma_load_2d(smem_u32(st + L.x + j * p.x_bytes), &p.tm_x, fb, (kbk + j) * kBK, m0);
+            tma_load_2d(smem_u32(st + L.w0), &p.tm_w0, fb, kbk * kBK, n0);
+            if (MODE == kGemmExp) tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kbk * kBK, n0);
+            if (MODE == kGemmPalette) {
+              tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kbk * (kBK / 2), n0);
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                if (q < NP && has[q])
+                  bulk_load(smem_u32(st + L.ebits + q * kEscArea),
+                            p.esc_pack + 16 * ((nt * H + q / KS) * p.KBK + kbk + q % KS) +
+                                (int64_t)c0[q] * 64,
+                            16 + nesc[q] * 64, fb);
             }
             ++issued;
           }
@@ -428,12 +445,17 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
               uint8_t* st = ring + (size_t)stage * L.bytes;
               const uint64_t b_desc = smem_desc_sw128(smem_u32(st + L.x));
               if (MODE != kGemmBf16 && p.tmem_w) {
-                // A: 32 columns of the slot, 8 per 16-wide K step
-                const uint32_t a_tmem = tmem_base + p.wcol0 + (uint32_t)(wslot * 32);
+                // A: 32 columns of the slot per K block, 8 per 16-wide K step;
+                // B: the K block's X tile
+                const uint32_t a_tmem = tmem_base + p.wcol0 + (uint32_t)(wslot * 32 * KS);
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                  mma_bf16_tmem_a(d_tmem, a_tmem + 8 * k, b_desc + 2 * k, idesc,
-                                  (!first || k > 0) ? 1u : 0u);
+                for (int j = 0; j < KS; ++j) {
+                  const uint64_t bj = smem_desc_sw128(smem_u32(st + L.x + j * p.x_bytes));
+#pragma unroll
+                  for (int k = 0; k < kBK / 16; ++k)
+                    mma_bf16_tmem_a(d_tmem, a_tmem + 32 * j + 8 * k, bj + 2 * k, idesc,
+                                    (!first || j > 0 || k > 0) ? 1u : 0u);
+                }
               } else {
                 const uint32_t a_addr =
                     MODE == kGemmBf16 ? smem_u32(st + L.w0 + (wide ? par * kWTileBytes : 0))
@@ -629,72 +651,102 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         const uint8_t* sEsc = st + L.ebits + hh * kEscArea;
         const int64_t grow = nt * H + hh;
         if (p.tmem_w) {
-          // One W row per thread: row r (TMEM lane r, the warp's quadrant)
-          // gets the K block's 64 weights in 32 columns of the slot.  S and E
-          // rows were staged with the 64-byte swizzle, I rows with the 32-byte
-          // one, so a quarter-warp's 16-byte reads hit distinct banks.
+          // One W row per thread: row r (TMEM lane r, the warp's quadrant) gets
+          // K block j's 64 weights in columns 32 j .. 32 j + 31 of the slot.
+          // Rows were staged with the TMA swizzle of their width (128, 64 or 32
+          // bytes: 16-byte chunk c of row r sits at chunk c ^ (bits 7.. of the
+          // row's offset)), so a quarter-warp's 16-byte reads hit distinct banks.
           const int r = 32 * (warp & 3) + lane;
-          uint4 sv[4], ev[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            sv[k] = *reinterpret_cast<const uint4*>(sS + r * 64 + ((k ^ ((r >> 1) & 3)) << 4));
-          if (MODE == kGemmExp) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              ev[k] = *reinterpret_cast<const uint4*>(sW1 + r * 64 + ((k ^ ((r >> 1) & 3)) << 4));
-          } else {
-            const uint4 i0 = *reinterpret_cast<const uint4*>(sW1 + r * 32 + ((0 ^ ((r >> 2) & 1)) << 4));
-            const uint4 i1 = *reinterpret_cast<const uint4*>(sW1 + r * 32 + ((1 ^ ((r >> 2) & 1)) << 4));
-            const uint32_t iw[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-            uint32_t ew[16];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint2 e = palette8(iw[j], p.palette[0], p.palette[1], p.palette[2], p.palette[3]);
-              ew[2 * j] = e.x;
-              ew[2 * j + 1] = e.y;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              ev[k] = make_uint4(ew[4 * k], ew[4 * k + 1], ew[4 * k + 2], ew[4 * k + 3]);
-            // escape rows take their verbatim exponents (slot = escape rows
-            // before the row in the 128-row group); the warp's 32 rows are one
-            // word of the bitmap
-            const uint4 eb4 = *reinterpret_cast<const uint4*>(sEsc);
-            const int wq = warp & 3;
-            const uint32_t word = wq == 0 ? eb4.x : wq == 1 ? eb4.y : wq == 2 ? eb4.z : eb4.w;
-            if ((word >> lane) & 1u) {
-              const uint32_t before = (wq > 0 ? __popc(eb4.x) : 0) + (wq > 1 ? __popc(eb4.y) : 0) +
-                                      (wq > 2 ? __popc(eb4.z) : 0);
-              const uint32_t slot = before + (uint32_t)__popc(word & ((1u << lane) - 1u));
-              const uint4* src;
-              if (slot < (uint32_t)kEscCap) {
-                src = reinterpret_cast<const uint4*>(sEsc + 16 + slot * 64);
-              } else {
-                const uint32_t first = __ldg(p.esc_off + grow * KB + kb);
-                src = reinterpret_cast<const uint4*>(p.esc_exp + (int64_t)(first + slot) * 64);
-              }
-#pragma unroll
-              for (int k = 0; k < 4; ++k) ev[k] = src[k];
-            }
-          }
-          // the stage's inputs are in registers: release it
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(b_empty + cur_stage));
-          const uint32_t* s32 = reinterpret_cast<const uint32_t*>(sv);
-          const uint32_t* e32 = reinterpret_cast<const uint32_t*>(ev);
-          uint32_t wv[32];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const uint2 m = merge4(s32[j], e32[j]);
-            wv[2 * j] = m.x;
-            wv[2 * j + 1] = m.y;
-          }
+          const int wq = warp & 3;
+          const uint32_t sw_rb = 64u * KS;                  // S / E row bytes
+          const uint32_t sw_m = sw_rb / 16u - 1u;           // chunk-index swizzle mask
+          const uint32_t sw_x = ((uint32_t)r * sw_rb >> 7) & sw_m;
+          const uint32_t iw_rb = 32u * KS;                  // index row bytes
+          const uint32_t iw_x = ((uint32_t)r * iw_rb >> 7) & (iw_rb / 16u - 1u);
+          const uint32_t tcol = tmem_base + ((uint32_t)(32 * wq) << 16) + p.wcol0 +
+                                (uint32_t)(cur_wslot * 32 * KS);
           // after the slot's previous MMAs (observed through its free barrier)
           tc_fence_after();
-          tmem_st32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + p.wcol0 +
-                        (uint32_t)(cur_wslot * 32),
-                    wv);
-          tmem_st_wait();
+#pragma unroll
+          for (int j = 0; j < KS; ++j) {
+            uint4 sv[4], ev[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              sv[k] = *reinterpret_cast<const uint4*>(sS + r * sw_rb +
+                                                      (((uint32_t)(4 * j + k) ^ sw_x) << 4));
+            const uint32_t* s32 = reinterpret_cast<const uint32_t*>(sv);
+            uint32_t wv[32];
+            bool verbatim = MODE == kGemmExp;  // exponents in ev[] (else W built from indices)
+            if (MODE == kGemmExp) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                ev[k] = *reinterpret_cast<const uint4*>(sW1 + r * sw_rb +
+                                                        (((uint32_t)(4 * j + k) ^ sw_x) << 4));
+            } else {
+              const uint4 i0 = *reinterpret_cast<const uint4*>(
+                  sW1 + r * iw_rb + (((uint32_t)(2 * j) ^ iw_x) << 4));
+              const uint4 i1 = *reinterpret_cast<const uint4*>(
+                  sW1 + r * iw_rb + (((uint32_t)(2 * j + 1) ^ iw_x) << 4));
+              const uint32_t iw[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+              // W straight from the index words (weights 8 m .. 8 m + 7 per word);
+              // the choice of form is uniform, so it stays outside the loops
+              if (p.pal_run) {
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                  const uint4 w4 = rebuild8_run(iw[m], s32[2 * m], s32[2 * m + 1], p.pal_bias);
+                  wv[4 * m] = w4.x;
+                  wv[4 * m + 1] = w4.y;
+                  wv[4 * m + 2] = w4.z;
+                  wv[4 * m + 3] = w4.w;
+                }
+              } else {
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                  const uint4 w4 = rebuild8_lut(iw[m], s32[2 * m], s32[2 * m + 1], p.palette[0],
+                                                p.palette[1], p.palette[2], p.palette[3]);
+                  wv[4 * m] = w4.x;
+                  wv[4 * m + 1] = w4.y;
+                  wv[4 * m + 2] = w4.z;
+                  wv[4 * m + 3] = w4.w;
+                }
+              }
+              // escape rows take their verbatim exponents (slot = escape rows
+              // before the row in the 128-row group); the warp's 32 rows are one
+              // word of the K block's bitmap
+              const uint8_t* sEj = sEsc + j * kEscArea;
+              const uint4 eb4 = *reinterpret_cast<const uint4*>(sEj);
+              const uint32_t word = wq == 0 ? eb4.x : wq == 1 ? eb4.y : wq == 2 ? eb4.z : eb4.w;
+              if ((word >> lane) & 1u) {
+                verbatim = true;
+                const uint32_t before = (wq > 0 ? __popc(eb4.x) : 0) +
+                                        (wq > 1 ? __popc(eb4.y) : 0) + (wq > 2 ? __popc(eb4.z) : 0);
+                const uint32_t slot = before + (uint32_t)__popc(word & ((1u << lane) - 1u));
+                const uint4* src;
+                if (slot < (uint32_t)kEscCap) {
+                  src = reinterpret_cast<const uint4*>(sEj + 16 + slot * 64);
+                } else {
+                  const uint32_t first = __ldg(p.esc_off + grow * p.KBK + kb * KS + j);
+                  src = reinterpret_cast<const uint4*>(p.esc_exp + (int64_t)(first + slot) * 64);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) ev[k] = src[k];
+              }
+            }
+            if (verbatim) {
+              const uint32_t* e32 = reinterpret_cast<const uint32_t*>(ev);
+#pragma unroll
+              for (int m = 0; m < 16; ++m) {
+                const uint2 w2 = merge4(s32[m], e32[m]);
+                wv[2 * m] = w2.x;
+                wv[2 * m + 1] = w2.y;
+              }
+            }
+            tmem_st32(tcol + (uint32_t)(32 * j), wv);
+            tmem_st_wait();  // wv is reused by the next K block
+          }
+          // the stage's inputs are consumed: release it, then hand the slot over
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(b_empty + cur_stage));
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(b_wfull + cur_wslot));
@@ -718,16 +770,28 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         }
         // every item as if no row were an escape row (no branch in the loop, so
         // the items' dependency chains interleave) ...
-#pragma unroll
-        for (int i = 0; i < kRebuildItems; ++i) {
+        // (the palette form is uniform: one loop per form)
+        auto store_item = [&](int i, uint4 w4) {
           const int c8 = gt + kGroupThreads * i;
           const int r = c8 >> 3, c = c8 & 7;
-          if (MODE == kGemmPalette)
-            e8[i] = palette8(v4[i], p.palette[0], p.palette[1], p.palette[2], p.palette[3]);
-          const uint2 lo = merge4(s8[i].x, e8[i].x);
-          const uint2 hi = merge4(s8[i].y, e8[i].y);
-          *reinterpret_cast<uint4*>(wt + r * 128 + ((c ^ (r & 7)) << 4)) =
-              make_uint4(lo.x, lo.y, hi.x, hi.y);
+          *reinterpret_cast<uint4*>(wt + r * 128 + ((c ^ (r & 7)) << 4)) = w4;
+        };
+        if (MODE == kGemmExp) {
+#pragma unroll
+          for (int i = 0; i < kRebuildItems; ++i) {
+            const uint2 lo = merge4(s8[i].x, e8[i].x);
+            const uint2 hi = merge4(s8[i].y, e8[i].y);
+            store_item(i, make_uint4(lo.x, lo.y, hi.x, hi.y));
+          }
+        } else if (p.pal_run) {
+#pragma unroll
+          for (int i = 0; i < kRebuildItems; ++i)
+            store_item(i, rebuild8_run(v4[i], s8[i].x, s8[i].y, p.pal_bias));
+        } else {
+#pragma unroll
+          for (int i = 0; i < kRebuildItems; ++i)
+            store_item(i, rebuild8_lut(v4[i], s8[i].x, s8[i].y, p.palette[0], p.palette[1],
+                                       p.palette[2], p.palette[3]));
         }
         // ... then the escape rows.  Thread rows r_i = gt/8 + 16 i, so a warp's
         // 32 rows are bits 4w..4w+3 and 16+4w..16+4w+3 (w = warp in the group) of
@@ -760,7 +824,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             if (slot < (uint32_t)kEscCap) {
               ex = *reinterpret_cast<const uint2*>(sEsc + 16 + slot * 64 + c * 8);
             } else {
-              const uint32_t first = __ldg(p.esc_off + grow * KB + kb);
+              const uint32_t first = __ldg(p.esc_off + grow * p.KBK + kb);
               ex = __ldg(reinterpret_cast<const uint2*>(p.esc_exp + (int64_t)(first + slot) * 64 +
                                                         c * 8));
             }
@@ -844,23 +908,30 @@ uint64_t wait_limit_ns() {
 
 int mma_warps_for(int tile_n) { return tile_n <= 128 ? 2 : 1; }
 
-// TMEM columns: two accumulator sets, then (TMEM path) 32 columns per W slot.
-int tmem_cols_for(int tile_n, int wslots_in_tmem) {
+// TMEM columns: two accumulator sets, then (TMEM path) the W slots.
+int tmem_cols_for(int tile_n, int w_cols) {
   int c = 32;
-  while (c < 2 * mma_warps_for(tile_n) * tile_n + 32 * wslots_in_tmem) c *= 2;
+  while (c < 2 * mma_warps_for(tile_n) * tile_n + w_cols) c *= 2;
   return c;
 }
 
-// Reconstructive modes with one half per unit and token tiles up to 64 rebuild
-// W into TMEM (the MMA reads A from there): it frees the shared-memory W ring
-// for load stages.
-bool tmem_w_for(const GemmArgs& a) {
-  return a.mode != kGemmBf16 && a.halves == 1 &&
-         2 * mma_warps_for(a.tile_n) * a.tile_n + 32 * a.wslots <= 512;
+// K blocks per unit when the reconstructive modes rebuild W into TMEM (the MMA
+// then reads A from there, and the shared-memory W ring becomes load stages);
+// 0 when W goes through shared memory.  Needs one half per unit and the slots
+// (32 columns per K block) beside the accumulators.  Two K blocks per unit
+// when K allows: the load time is set by the number of TMA boxes more than by
+// their bytes (pure load streams of the 14336x4096 palette form: 35 us with
+// one K block per stage, 26 us with two).
+int tmem_ks_for(const GemmArgs& a) {
+  if (a.mode == kGemmBf16 || a.halves != 1) return 0;
+  const int acc = 2 * mma_warps_for(a.tile_n) * a.tile_n;
+  if ((a.K / kBK) % 2 == 0 && acc + 64 * a.wslots <= 512) return 2;
+  if (acc + 32 * a.wslots <= 512) return 1;
+  return 0;
 }
 
-size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool tmem_w) {
-  const StageLayout L = stage_layout(mode, tile_n, halves);
+size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool tmem_w, int ks) {
+  const StageLayout L = stage_layout(mode, tile_n, halves, ks);
   if (tmem_w) wslots = 0;  // the W slots live in TMEM
   const int ws = mode == kGemmBf16 ? 0 : wslots;
   size_t b = 1024 /* alignment slack */ + (size_t)stages * L.bytes;
@@ -869,10 +940,10 @@ size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool
   return b;
 }
 
-template <int MODE>
+template <int MODE, int KS>
 cudaError_t set_smem_attr() {
   static cudaError_t e = cudaFuncSetAttribute(
-      gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+      gemm_kernel<MODE, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
   return e;
 }
 
@@ -910,12 +981,15 @@ bool gemm_resolve(GemmArgs* a) {
   if (a->mode != kGemmBf16 &&
       (a->wslots < 2 || a->wslots > kMaxWSlots || (a->wslots & 1)))
     return false;
+  const int tks = tmem_ks_for(*a);
+  a->tmem_w = tks > 0;
+  a->ks = tks > 0 ? tks : 1;
   if (a->stages == 0) {
     for (;;) {
       int s = max_stages;
-      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, tmem_w_for(*a)) > (size_t)kSmemLimit)
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks) > (size_t)kSmemLimit)
         s -= step;
-      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, tmem_w_for(*a)) <= (size_t)kSmemLimit ||
+      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks) <= (size_t)kSmemLimit ||
           a->wslots <= 2 || wide) {
         a->stages = s;
         break;
@@ -924,12 +998,12 @@ bool gemm_resolve(GemmArgs* a) {
     }
   }
   if (a->stages < 2 || (!wide && (a->stages & 1)) ||
-      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, tmem_w_for(*a)) > (size_t)kSmemLimit)
+      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, a->tmem_w, a->ks) > (size_t)kSmemLimit)
     return false;
   const int64_t RU = (int64_t)kBM * a->halves;
   const int64_t NT = (a->N + RU - 1) / RU;
   const int64_t MT = (a->M + a->tile_n - 1) / a->tile_n;
-  const int64_t units = NT * MT * (a->K / kBK);
+  const int64_t units = NT * MT * (a->K / kBK / a->ks);
   int ctas = a->ctas > 0 ? a->ctas : a->sm_count;
   if ((int64_t)ctas > units) ctas = (int)units;
   if (ctas > kGemmMaxCtas) ctas = kGemmMaxCtas;
@@ -946,10 +1020,13 @@ size_t gemm_partials_bytes(const GemmArgs& a) {
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* hooks) {
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
-  const int64_t KB = a.K / kBK;
+  if (a.ks < 1 || a.ks > 2 || (a.K / kBK) % a.ks) return cudaErrorInvalidValue;  // unresolved
+  const int KS = a.ks;
+  const int64_t KBK = a.K / kBK;
   const bool wide = a.halves == 2;
   const uint32_t RU = (uint32_t)kBM * (wide ? 2 : 1);
-  const bool tw = tmem_w_for(a);
+  const bool tw = a.tmem_w != 0;
+  if (KS > 1 && (!tw || a.mode == kGemmBf16)) return cudaErrorInvalidValue;
   if (!make_map_2d(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.K,
                    (uint64_t)a.M, kBK, (uint32_t)a.tile_n, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -959,17 +1036,22 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
                      (uint64_t)a.N, kBK, RU, CU_TENSOR_MAP_SWIZZLE_128B);
   } else {
     // rows rebuilt one per thread (TMEM path) are read 16 bytes at a time
-    // along the row: 64- and 32-byte swizzles spread a warp's rows over the banks
-    const CUtensorMapSwizzle sw64 = tw ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
-    const CUtensorMapSwizzle sw32 = tw ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    // along the row: the swizzle of the row's width (KS K blocks: 64 KS bytes of
+    // S or E, 32 KS of indices) spreads a warp's rows over the banks
+    auto sw_for = [&](int row_bytes) {
+      if (!tw) return CU_TENSOR_MAP_SWIZZLE_NONE;
+      return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+             : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                               : CU_TENSOR_MAP_SWIZZLE_32B;
+    };
     ok = make_map_2d(&p.tm_w0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.S, (uint64_t)a.K,
-                     (uint64_t)a.N, kBK, RU, sw64);
+                     (uint64_t)a.N, kBK * KS, RU, sw_for(kBK * KS));
     if (ok && a.mode == kGemmExp)
       ok = make_map_2d(&p.tm_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.E, (uint64_t)a.K,
-                       (uint64_t)a.N, kBK, RU, sw64);
+                       (uint64_t)a.N, kBK * KS, RU, sw_for(kBK * KS));
     if (ok && a.mode == kGemmPalette)
       ok = make_map_2d(&p.tm_w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.I, (uint64_t)a.K / 2,
-                       (uint64_t)a.N, kBK / 2, RU, sw32);
+                       (uint64_t)a.N, kBK / 2 * KS, RU, sw_for(kBK / 2 * KS));
   }
   if (!ok) return cudaErrorInvalidValue;
   p.esc_bits = a.esc_bits;
@@ -991,20 +1073,26 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.NG = (int32_t)((a.N + kBM - 1) / kBM);
   p.halves = wide ? 2 : 1;
   p.MT = (int32_t)((a.M + a.tile_n - 1) / a.tile_n);
-  p.KB = (int32_t)KB;
-  p.units = (int64_t)p.NT * p.MT * KB;
+  p.KBK = (int32_t)KBK;
+  p.ks = KS;
+  p.KB = (int32_t)(KBK / KS);
+  p.units = (int64_t)p.NT * p.MT * p.KB;
   p.esc_nwp = a.esc_nw;
   p.out_f32 = a.out_f32;
   p.n_mma = wide ? 2 : mma_warps_for(a.tile_n);
-  p.tmem_cols = wide ? 512 : tmem_cols_for(a.tile_n, tw ? a.wslots : 0);
+  p.tmem_cols = wide ? 512 : tmem_cols_for(a.tile_n, tw ? 32 * KS * a.wslots : 0);
   p.tmem_w = tw ? 1 : 0;
   p.wcol0 = (uint32_t)(2 * mma_warps_for(a.tile_n) * a.tile_n);
   p.acc_bufs = (!wide || 4 * a.tile_n <= 512) ? 2 : 1;  // TMEM: bufs x NM x tile_n columns
   std::memcpy(p.palette, a.palette, 16);
+  p.pal_run = 1;
+  for (int i = 1; i < 16; ++i)
+    if (a.palette[i] != a.palette[0] + i) p.pal_run = 0;
+  p.pal_bias = (uint32_t)a.palette[0] * 128u * 65537u;
   p.x_bytes = (uint32_t)a.tile_n * kBK * 2;
-  p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves).bytes;
+  p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves, KS).bytes;
   p.wait_ns = wait_limit_ns();
-  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw);
+  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS);
   const int G = a.ctas;
   cudaError_t e = cudaSuccess;
   auto begin = [&](int kind) { return hooks && hooks->begin ? hooks->begin(hooks->ctx, kind) : -1; };
@@ -1015,16 +1103,26 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   const int slot = begin(3 + a.mode);
   switch (a.mode) {
     case kGemmBf16:
-      if ((e = set_smem_attr<kGemmBf16>()) != cudaSuccess) return e;
-      gemm_kernel<kGemmBf16><<<G, threads_for(kGemmBf16), smem, s>>>(p);
+      if ((e = set_smem_attr<kGemmBf16, 1>()) != cudaSuccess) return e;
+      gemm_kernel<kGemmBf16, 1><<<G, threads_for(kGemmBf16), smem, s>>>(p);
       break;
     case kGemmExp:
-      if ((e = set_smem_attr<kGemmExp>()) != cudaSuccess) return e;
-      gemm_kernel<kGemmExp><<<G, threads_for(kGemmExp), smem, s>>>(p);
+      if (KS == 2) {
+        if ((e = set_smem_attr<kGemmExp, 2>()) != cudaSuccess) return e;
+        gemm_kernel<kGemmExp, 2><<<G, threads_for(kGemmExp), smem, s>>>(p);
+      } else {
+        if ((e = set_smem_attr<kGemmExp, 1>()) != cudaSuccess) return e;
+        gemm_kernel<kGemmExp, 1><<<G, threads_for(kGemmExp), smem, s>>>(p);
+      }
       break;
     case kGemmPalette:
-      if ((e = set_smem_attr<kGemmPalette>()) != cudaSuccess) return e;
-      gemm_kernel<kGemmPalette><<<G, threads_for(kGemmPalette), smem, s>>>(p);
+      if (KS == 2) {
+        if ((e = set_smem_attr<kGemmPalette, 2>()) != cudaSuccess) return e;
+        gemm_kernel<kGemmPalette, 2><<<G, threads_for(kGemmPalette), smem, s>>>(p);
+      } else {
+        if ((e = set_smem_attr<kGemmPalette, 1>()) != cudaSuccess) return e;
+        gemm_kernel<kGemmPalette, 1><<<G, threads_for(kGemmPalette), smem, s>>>(p);
+      }
       break;
     default:
       return cudaErrorInvalidValue;

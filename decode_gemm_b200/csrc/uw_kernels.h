@@ -83,6 +83,8 @@ struct GemmArgs {
   int halves = 0;                // W rows per unit / 128: 1, 2 (wide), 0 = auto by M
   int stages = 0;                // load ring depth (0 = auto)
   int wslots = 0;                // rebuilt-W ring depth (0 = auto)
+  int ks = 0;                    // resolved: 64-wide K blocks per unit (stage)
+  int tmem_w = 0;                // resolved: W rebuilt into TMEM (else shared memory)
   int ctas = 0;                  // persistent CTAs (0 = SM count)
   int sm_count = 148;
   uint32_t* status = nullptr;

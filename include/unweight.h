@@ -96,7 +96,7 @@ typedef struct uw_encode_opts {
  *                        p is bit 31 - p%32 of words[p/32]; n_words % 4 == 0
  *   chunk_off [n_chunks+1] u32  start bit of each chunk of chunk_syms symbols;
  *                        chunk_off[n_chunks] = total bits
- *   palette   [16]   u8  most frequent exponents, most frequent first
+ *   palette   [16]   u8  the 16 most frequent exponents, ascending
  *   esc_bits  [(K/64) * NWp] u32, NWp = 4*ceil(N/128): bit n%32 of word
  *                        [kb*NWp + n/32] set when the 64-weight row (n, kb) is an
  *                        escape row (16 bytes per 128-row block; padding bits 0)
@@ -211,8 +211,11 @@ UW_API uw_status uw_decode_full(uw_handle_t h, uint16_t* w_dev);
 UW_API uw_status uw_decode_exp(uw_handle_t h, uint8_t* e_dev);
 /* Palette transcode (pipeline 3 preprocessing; also the load-time step of
  * pipeline 4): N*K/2 bytes of packed 4-bit indices to idx_dev (16-byte
- * aligned); byte j of row n holds element 2j (low nibble) and 2j+1 (high
- * nibble); all indices of an escape row are 0. */
+ * aligned).  Index i of element (n, k) is the rank of its exponent in the
+ * ascending palette.  Each group of 8 consecutive elements of a row is one
+ * little-endian 32-bit word: element 2t at bits 4t..4t+3, element 2t+1 at bits
+ * 16+4t..16+4t+3 (t = 0..3), so each 16-bit half holds one index of every
+ * BF16 pair in the pair's own lane.  All indices of an escape row are 0. */
 UW_API uw_status uw_transcode_palette(uw_handle_t h, uint8_t* idx_dev);
 
 /* Y[M, N] = X[M, K] W^T with BF16 inputs, FP32 accumulation, BF16 output

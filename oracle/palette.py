@@ -9,16 +9,24 @@ index per weight next to the verbatim sign+mantissa byte.
 
 Readings taken where the post is silent:
 
-* Palette order: exponents ranked by count (descending), ties broken by the
-  exponent value (ascending); index 0 is the most frequent exponent.
+* Palette membership: exponents ranked by count (descending), ties broken by
+  the exponent value (ascending); the first 16 are kept.
 * Fewer than 16 distinct exponents: the palette is padded with the smallest
-  byte values not already present, ascending, so its 16 entries stay distinct.
+  byte values not already present, so its 16 entries stay distinct.
+* Palette order: the 16 entries ascending by value; index i is the rank of the
+  exponent among them.  (Exponent histograms of trained weights are unimodal,
+  so the 16 most frequent usually form one run b..b+15, and then the index is
+  simply e - b.)
 * A "row" is 64 consecutive weights along K inside one output row n:
   ``W[n, 64*kb : 64*kb + 64]``.  K must be a multiple of 64.
 * An escape row keeps its 64 exponent bytes verbatim (with S, that is the raw
   BF16 row).  In the transcoded index array its 64 indices are all 0.
-* Nibble packing: byte j of a row of packed indices holds element 2j in its low
-  nibble and element 2j+1 in its high nibble.
+* Nibble packing, per group of 8 consecutive indices of a row (4 bytes, read
+  as one little-endian 32-bit word): bits 4t..4t+3 hold element 2t and bits
+  16+4t..16+4t+3 hold element 2t+1 (t = 0..3).  So byte 0 holds elements 0
+  (low nibble) and 2, byte 1 elements 4 and 6, byte 2 elements 1 and 3, byte 3
+  elements 5 and 7: each 16-bit half of the word carries one index of each
+  BF16 pair, in the pair's own lane.
 """
 from __future__ import annotations
 
@@ -34,7 +42,7 @@ def exponent_histogram(e: np.ndarray) -> np.ndarray:
 
 
 def build_palette(hist: np.ndarray) -> np.ndarray:
-    """The 16 most frequent exponents, most frequent first (see module readings)."""
+    """The 16 most frequent exponents, ascending (see module readings)."""
     hist = np.asarray(hist, dtype=np.int64)
     present = [v for v in range(256) if hist[v] > 0]
     ranked = sorted(present, key=lambda v: (-int(hist[v]), v))
@@ -42,7 +50,7 @@ def build_palette(hist: np.ndarray) -> np.ndarray:
     filler = (v for v in range(256) if v not in palette)
     while len(palette) < PALETTE_SIZE:
         palette.append(next(filler))
-    return np.array(palette, dtype=np.uint8)
+    return np.array(sorted(palette), dtype=np.uint8)
 
 
 def escape_rows(e: np.ndarray, palette: np.ndarray) -> np.ndarray:
@@ -71,17 +79,26 @@ def transcode(e: np.ndarray, palette: np.ndarray, esc: np.ndarray) -> np.ndarray
 
 
 def pack_nibbles(idx: np.ndarray) -> np.ndarray:
-    """[N, K] indices -> [N, K/2] bytes: element 2j in the low nibble of byte j."""
-    idx = np.asarray(idx, dtype=np.uint8)
-    lo = idx[:, 0::2] & 0xF
-    hi = idx[:, 1::2] & 0xF
-    return (lo | (hi << 4)).astype(np.uint8)
+    """[N, K] indices -> [N, K/2] bytes, 8 indices per 4 bytes (see module readings)."""
+    idx = np.asarray(idx, dtype=np.uint8) & 0xF
+    n, k = idx.shape
+    if k % 8:
+        raise ValueError("K must be a multiple of 8")
+    g = idx.reshape(n, k // 8, 8).astype(np.uint32)
+    word = np.zeros((n, k // 8), dtype=np.uint32)
+    for t in range(4):
+        word |= g[:, :, 2 * t] << (4 * t)
+        word |= g[:, :, 2 * t + 1] << (16 + 4 * t)
+    return word.astype("<u4").view(np.uint8).reshape(n, k // 2)
 
 
 def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
-    packed = np.asarray(packed, dtype=np.uint8)
+    """Inverse of ``pack_nibbles``."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
     n, h = packed.shape
-    out = np.empty((n, 2 * h), dtype=np.uint8)
-    out[:, 0::2] = packed & 0xF
-    out[:, 1::2] = packed >> 4
-    return out
+    word = packed.reshape(n, h // 4, 4).copy().view("<u4").reshape(n, h // 4).astype(np.uint32)
+    out = np.empty((n, h // 4, 8), dtype=np.uint8)
+    for t in range(4):
+        out[:, :, 2 * t] = (word >> (4 * t)) & 0xF
+        out[:, :, 2 * t + 1] = (word >> (16 + 4 * t)) & 0xF
+    return out.reshape(n, 2 * h)

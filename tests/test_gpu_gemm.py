@@ -264,3 +264,33 @@ def test_wide_units_match_fp64(uw, M, N, K, kind, pipe, tile_n):
         y = _gemm(uw, h, x, pipe, halves=2, tile_n=tile_n, gemm_ctas=ctas)
         _check(y, x, w)
     h.free()
+
+
+PALETTE_CASES = [
+    ("lookup", list(range(100, 132, 2)), 0),   # 16 exponents, not a run: palette lookup
+    ("run_base0", list(range(0, 16)), 0),      # the run 0..15 (zero and subnormal weights)
+    ("run_escapes", list(range(110, 126)), 40),  # a run; 40 weights get rare exponents
+]
+
+
+@pytest.mark.parametrize("name,exps,planted", PALETTE_CASES, ids=[c[0] for c in PALETTE_CASES])
+@pytest.mark.parametrize("tile_n,halves", [(16, 1), (128, 1), (128, 2)])
+def test_palette_forms_match_fp64(uw, name, exps, planted, tile_n, halves):
+    """Both exponent rebuilds from indices (base + index for a palette that is
+    one run, lookup otherwise), on the TMEM (tile 16) and shared-memory paths."""
+    w = synthdata.exponent_pattern(384, 512, exps, seed=80 + len(exps))
+    rng = np.random.default_rng(82)
+    for _ in range(planted):  # exponents outside the palette: their rows escape
+        r, k = int(rng.integers(0, 384)), int(rng.integers(0, 512))
+        w[r, k] = (w[r, k] & 0x807F) | (int(rng.choice([90, 140])) << 7)
+    h = _upload(uw, w, chunk=512)
+    M = 40
+    _workspace(uw, h, M)
+    x = synthdata.activations(M, 512, 81)
+    outs = {}
+    for pipe in ("exp", "palette_rt", "palette_direct"):
+        outs[pipe] = _gemm(uw, h, x, pipe, tile_n=tile_n, halves=halves)
+        _check(outs[pipe], x, w)
+    assert np.array_equal(outs["exp"], outs["palette_rt"])
+    assert np.array_equal(outs["exp"], outs["palette_direct"])
+    h.free()

@@ -54,8 +54,18 @@ def _encode_lsb_first(symbols, lengths, codes):
 
 
 def _pack_swapped(idx):
+    # plain byte packing (element 2j low, 2j+1 high) instead of the
+    # per-word interleave
     idx = np.asarray(idx, dtype=np.uint8)
-    return (idx[:, 1::2] | (idx[:, 0::2] << 4)).astype(np.uint8)
+    return (idx[:, 0::2] | (idx[:, 1::2] << 4)).astype(np.uint8)
+
+
+def _pack_halves_swapped(idx):
+    # odd elements in the low half-word
+    idx = np.asarray(idx, dtype=np.uint8)
+    sw = idx.copy()
+    sw[:, 0::2], sw[:, 1::2] = idx[:, 1::2], idx[:, 0::2]
+    return P.pack_nibbles.__wrapped__(sw)
 
 
 def _gemm_no_transpose(x_bits, w_bits):
@@ -66,6 +76,16 @@ def _palette_ties_descending(hist):
     hist = np.asarray(hist, dtype=np.int64)
     present = [v for v in range(256) if hist[v] > 0]
     ranked = sorted(present, key=lambda v: (-int(hist[v]), -v))[:16]
+    filler = (v for v in range(256) if v not in ranked)
+    while len(ranked) < 16:
+        ranked.append(next(filler))
+    return np.array(sorted(ranked), np.uint8)
+
+
+def _palette_frequency_order(hist):
+    hist = np.asarray(hist, dtype=np.int64)
+    present = [v for v in range(256) if hist[v] > 0]
+    ranked = sorted(present, key=lambda v: (-int(hist[v]), v))[:16]
     filler = (v for v in range(256) if v not in ranked)
     while len(ranked) < 16:
         ranked.append(next(filler))
@@ -87,6 +107,10 @@ CASES = [
      pins.test_gemm_matches_fsum_triple_loop),
     ("palette tie order", oracle, "build_palette", _palette_ties_descending,
      pins.test_palette_order_and_padding),
+    ("palette by frequency", oracle, "build_palette", _palette_frequency_order,
+     pins.test_palette_order_and_padding),
+    ("index halves swapped", oracle, "pack_nibbles", _pack_halves_swapped,
+     pins.test_transcode_and_nibble_order),
 ]
 
 

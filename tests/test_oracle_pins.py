@@ -230,10 +230,18 @@ def test_palette_order_and_padding():
     hist = np.zeros(256, np.int64)
     hist[[130, 120, 125, 121]] = [5, 9, 9, 1]
     pal = oracle.build_palette(hist)
-    # count descending, ties by value ascending, then the smallest absent bytes
-    assert list(pal[:4]) == [120, 125, 130, 121]
-    assert list(pal[4:]) == list(range(0, 12))
+    # the four present exponents plus the smallest absent bytes, ascending
+    assert list(pal) == list(range(0, 12)) + [120, 121, 125, 130]
     assert len(set(pal.tolist())) == 16
+    # 17 present exponents: the last slot goes by count, then by the smaller
+    # value (115 and 116 tie; 99 is rarer than both)
+    hist = np.zeros(256, np.int64)
+    hist[100:115] = 50 + np.arange(15)
+    hist[[115, 116, 99]] = [7, 7, 3]
+    assert list(oracle.build_palette(hist)) == list(range(100, 116))
+    # a frequency order would put 114 (the most frequent) first
+    hist[114] = 1000
+    assert list(oracle.build_palette(hist)) == list(range(100, 116))
 
 
 def test_at_most_16_exponents_means_no_escape_rows():
@@ -272,7 +280,13 @@ def test_escape_invariants_on_heavy_tails():
 def test_transcode_and_nibble_order():
     idx = np.array([[1, 2, 3, 4, 15, 0] + [0] * 58], np.uint8)
     packed = oracle.pack_nibbles(idx)
-    assert list(packed[0, :3]) == [0x21, 0x43, 0x0F]
+    # group of 8: byte 0 = elements 0 | 2 << 4, byte 1 = 4 | 6 << 4,
+    # byte 2 = 1 | 3 << 4, byte 3 = 5 | 7 << 4
+    assert list(packed[0, :4]) == [0x31, 0x0F, 0x42, 0x00]
+    # read as a little-endian word, element 2t sits at bits 4t, 2t+1 at 16+4t
+    word = int.from_bytes(bytes(packed[0, :4]), "little")
+    assert [(word >> (4 * t)) & 15 for t in range(4)] == [1, 3, 15, 0]
+    assert [(word >> (16 + 4 * t)) & 15 for t in range(4)] == [2, 4, 0, 0]
     assert np.array_equal(oracle.unpack_nibbles(packed), idx)
     w = synthdata.student_t(128, 512, 3.0, 0.015, seed=14)
     enc = oracle.encode(w, chunk_syms=512)
