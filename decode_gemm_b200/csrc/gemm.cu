@@ -229,7 +229,6 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             b_tfull = 2 * S + 2 * WS, b_tempty = b_tfull + 2, b_drain = b_tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + b_drain + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* tag_slot = tmem_slot + 2;  // this launch's hand-off tag (epoch + 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -252,9 +251,40 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       mbar_init(bar(b_drain + a), 1);
     }
     *abort = 0;
-    *tag_slot = __ldcg(p.sync) + 1u;
     fence_mbar_init();
   }
+  const int64_t G = gridDim.x;
+  const int64_t u0 = unit_begin(blockIdx.x, p.units, G);
+  const int64_t u1 = unit_begin(blockIdx.x + 1, p.units, G);
+  const int KB = p.KB;    // units along K
+  constexpr int KS = KS_;  // K blocks per unit
+  const int NP = H * KS;  // escape parts per stage: (half, K block) pairs, at most 2
+  // Palette escape offsets (first and end row of each part's escape run) of 32
+  // units, one unit per lane, loaded together: a load per stage would put its
+  // latency on the issue path.  The first batch is loaded during setup, later
+  // ones half a batch ahead.
+  uint32_t lc0[2] = {0u, 0u}, lc1[2] = {0u, 0u}, nc0[2] = {0u, 0u}, nc1[2] = {0u, 0u};
+  auto esc_batch = [&](int64_t qfirst, uint32_t (&o0)[2], uint32_t (&o1)[2]) {
+    const int64_t uu = u0 + qfirst + lane;
+    o0[0] = o0[1] = o1[0] = o1[1] = 0u;
+    if (uu < u1) {
+      const int64_t tt = uu / KB;
+      const int64_t kk = uu - tt * KB;
+      const int64_t g0 = (tt / p.MT) * H;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (q >= NP) break;
+        // part q: half q / KS, K block kk * KS + q % KS
+        const int64_t g = g0 + q / KS;
+        if (g < p.NG) {
+          const int64_t gi = g * p.KBK + kk * KS + q % KS;
+          o0[q] = __ldg(p.esc_off + gi);
+          o1[q] = __ldg(p.esc_off + gi + 1);
+        }
+      }
+    }
+  };
+  if (MODE == kGemmPalette && warp == 0) esc_batch(0, lc0, lc1);
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&p.tm_x);
     prefetch_tensormap(&p.tm_w0);
@@ -269,22 +299,12 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int64_t G = gridDim.x;
-  const int64_t u0 = unit_begin(blockIdx.x, p.units, G);
-  const int64_t u1 = unit_begin(blockIdx.x + 1, p.units, G);
-  const int KB = p.KB;    // units along K
-  constexpr int KS = KS_;  // K blocks per unit
-  const int NP = H * KS;  // escape parts per stage: (half, K block) pairs, at most 2
-
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     int stage = 0;
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
-    // palette escape offsets of the next 32 units, one unit per lane, loaded
-    // together (a load per stage would put its latency on the issue path)
-    uint32_t lc0[2] = {0u, 0u}, lc1[2] = {0u, 0u};
     int qi = 0;  // index of the unit among this CTA's units
     for (int64_t u = u0; u < u1 && ok;) {
       const int64_t t = u / KB;
@@ -295,24 +315,12 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       for (int kb = kb0; kb < kb1; ++kb, ++qi) {
         uint32_t c0[2] = {0u, 0u}, c1[2] = {0u, 0u};
         if (MODE == kGemmPalette) {
-          if ((qi & 31) == 0) {
-            const int64_t uu = u0 + qi + lane;
-            lc0[0] = lc0[1] = lc1[0] = lc1[1] = 0u;
-            if (uu < u1) {
-              const int64_t tt = uu / KB;
-              const int64_t kk = uu - tt * KB;
-              const int64_t g0 = (tt / p.MT) * H;
+          if ((qi & 31) == 16) esc_batch(qi + 16, nc0, nc1);
+          if ((qi & 31) == 0 && qi > 0) {
 #pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                if (q >= NP) break;
-                // part q: half q / KS, K block kk * KS + q % KS
-                const int64_t g = g0 + q / KS;
-                if (g < p.NG) {
-                  const int64_t gi = g * p.KBK + kk * KS + q % KS;
-                  lc0[q] = __ldg(p.esc_off + gi);
-                  lc1[q] = __ldg(p.esc_off + gi + 1);
-                }
-              }
+            for (int q = 0; q < 2; ++q) {
+              lc0[q] = nc0[q];
+              lc1[q] = nc1[q];
             }
           }
 #pragma unroll
@@ -499,7 +507,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
     const bool leader = warp == kEpiWarp0 && lane == 0;
-    const uint32_t tag = *tag_slot;
+    // this launch's hand-off tag: the epoch (advanced by the previous launch's
+    // last CTA, constant while this launch runs) plus one
+    const uint32_t tag = __ldcg(p.sync) + 1u;
     const int64_t part_stride = (int64_t)p.tile_n * RU;  // a CTA's partial-sum tile
     int seg = 0;
     int64_t qa = 0;  // index (among this CTA's units) of the segment's first unit
@@ -551,6 +561,15 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         const int64_t n = nt * RU + h * kBM + row;
         const int64_t hoff = (int64_t)h * kBM * p.tile_n;  // the half's place in a partial tile
         float* part = p.partials + (int64_t)blockIdx.x * part_stride + hoff;
+        // an owner reads the first contributor's sums one column block ahead,
+        // so their latency overlaps the TMEM reads and the stores
+        const bool gather = split && owner;
+        const float* part1 = p.partials + (int64_t)(blockIdx.x + 1) * part_stride + hoff + row;
+        float pn[16];
+        if (gather) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pn[j] = j < cols ? __ldcg(part1 + j * kBM) : 0.f;
+        }
         for (int c = 0; c < cols; c += 16) {
           uint32_t r0[16], r1[16];
           if (use0) tmem_ld16(t0 + (uint32_t)c, r0);
@@ -568,10 +587,17 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
               if (c + j < cols) part[(int64_t)(c + j) * kBM + row] = v[j];
             continue;
           }
-          if (split) {
+          if (gather) {
             // the other CTAs' sums, in K order; a contributor's 16 loads are all
             // in flight before the first add
-            for (int64_t q = blockIdx.x + 1; q <= last; ++q) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += pn[j];
+            if (c + 16 < cols) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                pn[j] = c + 16 + j < cols ? __ldcg(part1 + (int64_t)(c + 16 + j) * kBM) : 0.f;
+            }
+            for (int64_t q = blockIdx.x + 2; q <= last; ++q) {
               const float* src = p.partials + q * part_stride + hoff + (int64_t)c * kBM + row;
               float pv[16];
 #pragma unroll
