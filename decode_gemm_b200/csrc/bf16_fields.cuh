@@ -49,9 +49,10 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // element 2t at bits 4t, element 2t+1 at bits 16+4t, so each 16-bit half holds
 // one index of every BF16 pair, in the pair's own lane.
 __device__ __forceinline__ uint32_t nibbles_interleave(uint32_t v) {
-  const uint32_t ev = v & 0x0F0F0F0Fu, od = (v >> 4) & 0x0F0F0F0Fu;
-  // byte 0 of (x | x >> 4) = nibbles 0 and 2 of the group, byte 2 = 4 and 6
-  return __byte_perm(ev | (ev >> 4), od | (od >> 4), 0x6420);
+  // swap nibbles 1 <-> 2 and 5 <-> 6 (a delta swap): the bytes become
+  // (0 2) (1 3) (4 6) (5 7); then bytes 1 and 2 trade places
+  const uint32_t t = (v ^ (v >> 4)) & 0x00F000F0u;
+  return __byte_perm(v ^ t ^ (t << 4), 0u, 0x3120);
 }
 
 // Eight BF16 weights (four pair words, element order) from one interleaved

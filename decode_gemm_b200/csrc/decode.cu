@@ -41,6 +41,7 @@
 #include <type_traits>
 
 #include "bf16_fields.cuh"
+#include "pdl.cuh"
 #include "uw_internal.h"
 #include "uw_kernels.h"
 
@@ -192,6 +193,10 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     reinterpret_cast<uint4*>(sm.lut)[i] = __ldg(reinterpret_cast<const uint4*>(a.lut) + i);
   for (int i = threadIdx.x; i < kCanonWords; i += blockDim.x) sm.canon[i] = __ldg(a.canon + i);
   __syncthreads();
+  // the tables are the handle's own (never written by a kernel); the output
+  // may still be read by the kernel before this one
+  if (threadIdx.x == 0) pdl_release();
+  pdl_wait();
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -524,15 +529,15 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cu
   switch (mode) {
     case kDecodeExp:
       e = set_attrs(decode_kernel<kDecodeExp>, smem);
-      if (e == cudaSuccess) decode_kernel<kDecodeExp><<<grid, block, smem, s>>>(a, out);
+      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodeExp>, grid, block, smem, s, a, out);
       break;
     case kDecodeFull:
       e = set_attrs(decode_kernel<kDecodeFull>, smem);
-      if (e == cudaSuccess) decode_kernel<kDecodeFull><<<grid, block, smem, s>>>(a, out);
+      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodeFull>, grid, block, smem, s, a, out);
       break;
     case kDecodePalette:
       e = set_attrs(decode_kernel<kDecodePalette>, smem);
-      if (e == cudaSuccess) decode_kernel<kDecodePalette><<<grid, block, smem, s>>>(a, out);
+      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodePalette>, grid, block, smem, s, a, out);
       break;
     default:
       return cudaErrorInvalidValue;

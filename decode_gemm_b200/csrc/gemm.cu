@@ -43,6 +43,7 @@
 
 #include "bf16_fields.cuh"
 #include "gemm_sm100.cuh"
+#include "pdl.cuh"
 #include "uw_kernels.h"
 
 namespace uw {
@@ -298,6 +299,11 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // set-up above touched only the handle's immutable arrays; from here on X,
+  // the preprocessed weights, the workspace and the hand-off flags may belong
+  // to the kernel before this one
+  if (threadIdx.x == 0) pdl_release();
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
@@ -410,8 +416,11 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     // q % 2 == par (all of them when NM == 1) and accumulates into its own
     // TMEM columns.  The ring depths are then even, so a stage or W slot is
     // always consumed by the same warp, in order: a parity wait can never see
-    // a stale phase.  Wide shape: warp par takes half par of every unit (W
-    // slots go in pairs, slot 2 j + par for pair j) into its own columns.
+    // a stale phase.  (With an odd depth a stage would alternate between the
+    // warps, and a parity wait cannot tell the fill before last, still
+    // pending, from its own completed fill.)  Wide shape: warp par takes half
+    // par of every unit (W slots go in pairs, slot 2 j + par for pair j) into
+    // its own columns.
     const int par = warp - kMmaWarp0;
     if (par < NM) {
       const uint32_t idesc = idesc_bf16(kBM, p.tile_n);
@@ -1130,30 +1139,31 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   switch (a.mode) {
     case kGemmBf16:
       if ((e = set_smem_attr<kGemmBf16, 1>()) != cudaSuccess) return e;
-      gemm_kernel<kGemmBf16, 1><<<G, threads_for(kGemmBf16), smem, s>>>(p);
+      e = launch_pdl(gemm_kernel<kGemmBf16, 1>, G, threads_for(kGemmBf16), smem, s, p);
       break;
     case kGemmExp:
       if (KS == 2) {
         if ((e = set_smem_attr<kGemmExp, 2>()) != cudaSuccess) return e;
-        gemm_kernel<kGemmExp, 2><<<G, threads_for(kGemmExp), smem, s>>>(p);
+        e = launch_pdl(gemm_kernel<kGemmExp, 2>, G, threads_for(kGemmExp), smem, s, p);
       } else {
         if ((e = set_smem_attr<kGemmExp, 1>()) != cudaSuccess) return e;
-        gemm_kernel<kGemmExp, 1><<<G, threads_for(kGemmExp), smem, s>>>(p);
+        e = launch_pdl(gemm_kernel<kGemmExp, 1>, G, threads_for(kGemmExp), smem, s, p);
       }
       break;
     case kGemmPalette:
       if (KS == 2) {
         if ((e = set_smem_attr<kGemmPalette, 2>()) != cudaSuccess) return e;
-        gemm_kernel<kGemmPalette, 2><<<G, threads_for(kGemmPalette), smem, s>>>(p);
+        e = launch_pdl(gemm_kernel<kGemmPalette, 2>, G, threads_for(kGemmPalette), smem, s, p);
       } else {
         if ((e = set_smem_attr<kGemmPalette, 1>()) != cudaSuccess) return e;
-        gemm_kernel<kGemmPalette, 1><<<G, threads_for(kGemmPalette), smem, s>>>(p);
+        e = launch_pdl(gemm_kernel<kGemmPalette, 1>, G, threads_for(kGemmPalette), smem, s, p);
       }
       break;
     default:
       return cudaErrorInvalidValue;
   }
   end(slot);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

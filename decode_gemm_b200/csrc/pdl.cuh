@@ -1,0 +1,42 @@
+// Programmatic dependent launch: consecutive kernels of the library on one
+// stream overlap one's start-up (barrier set-up, TMEM allocation, table loads,
+// reads of the handle's immutable arrays) with the tail of the kernel before.
+//
+// A kernel launched with launch_pdl must call pdl_wait() before it touches any
+// memory an earlier kernel of the stream may write or read (inputs, workspace,
+// outputs, hand-off flags); it calls pdl_release() once its own CTAs no longer
+// need to hold back the next kernel's start (here: right after set-up, since
+// every kernel of the library is a persistent grid of at most one CTA per SM).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <utility>
+
+namespace uw {
+
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+}  // namespace uw
