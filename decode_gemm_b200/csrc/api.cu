@@ -215,7 +215,10 @@ uw_status run_gemm_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
     case UW_PIPE_FULL: a.W = static_cast<const uint16_t*>(pre); break;
     case UW_PIPE_EXP: a.E = static_cast<const uint8_t*>(pre); break;
     case UW_PIPE_PALETTE_RT: a.I = static_cast<const uint8_t*>(pre); break;
-    default: a.I = h->d_pal_idx; break;
+    default:
+      a.I = h->d_pal_idx;
+      a.w1_resident = 1;
+      break;
   }
   LaunchHooks hooks;
   hooks.ctx = h;

@@ -193,10 +193,12 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     reinterpret_cast<uint4*>(sm.lut)[i] = __ldg(reinterpret_cast<const uint4*>(a.lut) + i);
   for (int i = threadIdx.x; i < kCanonWords; i += blockDim.x) sm.canon[i] = __ldg(a.canon + i);
   __syncthreads();
-  // the tables are the handle's own (never written by a kernel); the output
-  // may still be read by the kernel before this one
+  // the tables, the stream and S are the handle's own (never written by a
+  // kernel); the output may still be read by the kernel before this one, so a
+  // warp waits for that kernel before its first write (its first round is
+  // decoded meanwhile)
   if (threadIdx.x == 0) pdl_release();
-  pdl_wait();
+  bool waited = false;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -332,6 +334,10 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         while (left4 > 0) lookup_one(std::true_type());
       }
       __syncwarp();
+      if (!waited) {
+        pdl_wait();
+        waited = true;
+      }
 
       // ---- coalesced write-out of round r for the warp's 32 chunks ----
       // rel0: this round's first symbol inside each chunk; a lane's part of

@@ -100,6 +100,8 @@ struct GemmParams {
   int32_t NG;        // 128-row groups of W (escape groups per K block)
   int32_t tmem_w;    // W slots in TMEM (MMA A from TMEM) rather than shared memory
   uint32_t wcol0;    // first TMEM column of the W slots
+  const uint8_t* pf_s;   // the handle's sign+mantissa array, for early L2 prefetch
+  const uint8_t* pf_i;   // resident index array (pipeline 4), or null
   int32_t pal_run;   // palette is the run base..base+15 (index = exponent - base)
   uint32_t pal_bias; // base * 128 in both 16-bit halves
   uint32_t palette[4];
@@ -301,8 +303,25 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   const uint32_t tmem_base = *tmem_slot;
   // set-up above touched only the handle's immutable arrays; from here on X,
   // the preprocessed weights, the workspace and the hand-off flags may belong
-  // to the kernel before this one
+  // to the kernel before this one.  Meanwhile the rebuild warps (idle until
+  // the first stage lands) pull the first ring's immutable weight rows into
+  // L2, so the first loads after the wait hit L2.
   if (threadIdx.x == 0) pdl_release();
+  if (MODE != kGemmBf16 && warp >= kRebuildWarp0 && H == 1) {
+    const int64_t n_pf = imin64(u1 - u0, S);
+    const int rt = threadIdx.x - kRebuildWarp0 * 32;
+    for (int64_t i = rt; i < n_pf * kBM; i += kNumRebuildWarps * 32) {
+      const int64_t u = u0 + i / kBM;
+      const int64_t t = u / p.KB;
+      const int64_t nt = t / p.MT;
+      const int64_t n = nt * kBM + i % kBM;
+      const int64_t kbk = (u - t * p.KB) * KS;
+      if (n < p.N) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.pf_s + n * p.K + kbk * kBK));
+        if (p.pf_i) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.pf_i + n * (p.K / 2) + kbk * (kBK / 2)));
+      }
+    }
+  }
   pdl_wait();
 
   if (warp == 0) {
@@ -1120,6 +1139,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.wcol0 = (uint32_t)(2 * mma_warps_for(a.tile_n) * a.tile_n);
   p.acc_bufs = (!wide || 4 * a.tile_n <= 512) ? 2 : 1;  // TMEM: bufs x NM x tile_n columns
   std::memcpy(p.palette, a.palette, 16);
+  p.pf_s = a.S;
+  p.pf_i = a.w1_resident ? a.I : nullptr;
   p.pal_run = 1;
   for (int i = 1; i < 16; ++i)
     if (a.palette[i] != a.palette[0] + i) p.pal_run = 0;

@@ -72,6 +72,7 @@ uw_status uw_gemm_palette_noalloc(uw_handle_t h, const uint16_t* X_dev, void* Y_
   a.X = X_dev;
   a.S = h->d_sm;
   a.I = h->d_pal_idx;
+  a.w1_resident = 1;
   a.esc_bits = h->d_esc_bits;
   a.esc_off = h->d_esc_off;
   a.esc_exp = h->d_esc_exp;

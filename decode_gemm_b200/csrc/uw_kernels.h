@@ -68,6 +68,7 @@ struct GemmArgs {
   const uint8_t* S = nullptr;    // [N, K] sign+mantissa (kGemmExp, kGemmPalette)
   const uint8_t* E = nullptr;    // [N, K] exponents (kGemmExp)
   const uint8_t* I = nullptr;    // [N, K/2] packed palette indices (kGemmPalette)
+  int w1_resident = 0;           // I is the handle's resident array (not a kernel's output)
   const uint32_t* esc_bits = nullptr;
   const uint32_t* esc_off = nullptr;
   const uint8_t* esc_exp = nullptr;
