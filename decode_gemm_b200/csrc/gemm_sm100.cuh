@@ -96,6 +96,12 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
+// Order this thread's generic-proxy view of global memory with its later
+// async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
