@@ -59,9 +59,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum; profiles/*.md), valid only while the kernel source
 # (src_sha, see _kernel_src_sha) is unchanged.
 TRAFFIC = {
-    "gemm_palette": {"bytes_per_launch": 89.788928e6 + 3.738624e6, "src_sha": "8c979cf4aa02d602",
+    "gemm_palette": {"bytes_per_launch": 89.877504e6 + 5.247488e6, "src_sha": "f512bca2bc05b13c",
                      "capture": "profiles/gemm_palette_gate_14336x4096_M1.md (M = 1 launch)"},
-    "decode_full": {"bytes_per_launch": 87.552256e6 + 64.837888e6, "src_sha": "8c979cf4aa02d602",
+    "decode_full": {"bytes_per_launch": 87.519488e6 + 64.510720e6, "src_sha": "f512bca2bc05b13c",
                     "capture": "profiles/decode_full_gate_14336x4096.md (output partly still in L2)"},
 }
 
