@@ -89,6 +89,10 @@ DecodeArgs decode_args(const uw_handle_s* h) {
   a.lut = h->d_lut;
   a.canon = h->d_canon;
   std::memcpy(a.palette, h->palette, 16);
+  bool run = true;
+  for (int i = 1; i < 16; ++i)
+    if (h->palette[i] != h->palette[0] + i) run = false;
+  a.pal_run_b4 = run ? (uint32_t)h->palette[0] * 0x01010101u : 0xFFFFFFFFu;
   a.sm = h->d_sm;
   a.esc_bits = h->d_esc_bits;
   a.status = h->d_status;

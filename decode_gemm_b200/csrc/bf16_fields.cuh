@@ -35,6 +35,15 @@ __device__ __forceinline__ uint2 palette8(uint32_t v, uint32_t p0, uint32_t p1, 
   return make_uint2(__byte_perm(lo0, hi0, pick), __byte_perm(lo1, hi1, pick >> 16));
 }
 
+// Exponent bytes of eight ranks in element order (nibble t of v = element t)
+// for a palette that is the run b..b+15 (b4 = b in every byte): b + rank,
+// element order restored by two byte permutes.
+__device__ __forceinline__ uint2 run8(uint32_t v, uint32_t b4) {
+  const uint32_t ev = (v & 0x0F0F0F0Fu) + b4;         // elements 0 2 4 6
+  const uint32_t od = ((v >> 4) & 0x0F0F0F0Fu) + b4;  // elements 1 3 5 7
+  return make_uint2(__byte_perm(ev, od, 0x5140), __byte_perm(ev, od, 0x7362));
+}
+
 // PTX prmt in its default mode: a selector nibble with bit 3 set fills the
 // byte with the sign bit of the byte it selects (the CUDA intrinsic
 // __byte_perm ignores that bit).

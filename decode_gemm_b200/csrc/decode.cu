@@ -214,6 +214,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   const int64_t cs = a.chunk_syms;
   const int rows_per_chunk = (int)(cs / 64);
   const uint32_t p0 = a.palette[0], p1 = a.palette[1], p2 = a.palette[2], p3 = a.palette[3];
+  const bool pal_run = a.pal_run_b4 != 0xFFFFFFFFu;  // ranks are exponent - b
+  const uint32_t b4 = a.pal_run_b4;
   const int64_t grid_warps = (int64_t)gridDim.x * n_warps;
 
   for (int64_t grp = (int64_t)blockIdx.x * n_warps + warp; grp < groups; grp += grid_warps) {
@@ -348,16 +350,23 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         const int m = lane & 7, jq = lane >> 3;
         const bool in_chunk = rel0 + 16 * m < cs;
         uint8_t* base = static_cast<uint8_t*>(out) + c0 * cs + rel0 + 16 * m;
+        auto write = [&](auto expo) {
 #pragma unroll 4
-        for (int i = 0; i < 8; ++i) {
-          const int j = 4 * i + jq;
-          const int64_t o = (int64_t)j * cs;
-          const uint32_t* sw = stage + j * kStageStride + 2 * m;
-          const uint2 lo = palette8(sw[0], p0, p1, p2, p3);
-          const uint2 hi = palette8(sw[1], p0, p1, p2, p3);
-          st_v4_if(base + o, make_uint4(lo.x, lo.y, hi.x, hi.y),
-                   in_chunk && o + rel0 + 16 * m < grp_syms_left);
-        }
+          for (int i = 0; i < 8; ++i) {
+            const int j = 4 * i + jq;
+            const int64_t o = (int64_t)j * cs;
+            const uint32_t* sw = stage + j * kStageStride + 2 * m;
+            const uint2 lo = expo(sw[0]);
+            const uint2 hi = expo(sw[1]);
+            st_v4_if(base + o, make_uint4(lo.x, lo.y, hi.x, hi.y),
+                     in_chunk && o + rel0 + 16 * m < grp_syms_left);
+          }
+        };
+        // (the palette form is uniform: one loop per form)
+        if (pal_run)
+          write([&](uint32_t v) { return run8(v, b4); });
+        else
+          write([&](uint32_t v) { return palette8(v, p0, p1, p2, p3); });
       } else if (MODE == kDecodeFull) {
         // 16 lanes per chunk, 8 symbols (one rank word) per lane
         const int m = lane & 15, jh = lane >> 4;
@@ -365,25 +374,31 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         const int64_t sym0 = c0 * cs + rel0 + 8 * m;
         const uint8_t* sbase = a.sm + sym0;
         uint16_t* obase = static_cast<uint16_t*>(out) + sym0;
-        // eight loads in flight before their first use
+        auto write = [&](auto expo) {
+          // eight loads in flight before their first use
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint2 sv[8];
+          for (int h = 0; h < 2; ++h) {
+            uint2 sv[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int64_t o = (int64_t)(16 * h + 2 * i + jh) * cs;
-            sv[i] = ld_v2_if(sbase + o, in_chunk && o + rel0 + 8 * m < grp_syms_left);
+            for (int i = 0; i < 8; ++i) {
+              const int64_t o = (int64_t)(16 * h + 2 * i + jh) * cs;
+              sv[i] = ld_v2_if(sbase + o, in_chunk && o + rel0 + 8 * m < grp_syms_left);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int j = 16 * h + 2 * i + jh;
+              const int64_t o = (int64_t)j * cs;
+              const uint2 e = expo(stage[j * kStageStride + m]);
+              const uint2 lo = merge4(sv[i].x, e.x), hi = merge4(sv[i].y, e.y);
+              st_v4_if(obase + o, make_uint4(lo.x, lo.y, hi.x, hi.y),
+                       in_chunk && o + rel0 + 8 * m < grp_syms_left);
+            }
           }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int j = 16 * h + 2 * i + jh;
-            const int64_t o = (int64_t)j * cs;
-            const uint2 e = palette8(stage[j * kStageStride + m], p0, p1, p2, p3);
-            const uint2 lo = merge4(sv[i].x, e.x), hi = merge4(sv[i].y, e.y);
-            st_v4_if(obase + o, make_uint4(lo.x, lo.y, hi.x, hi.y),
-                     in_chunk && o + rel0 + 8 * m < grp_syms_left);
-          }
-        }
+        };
+        if (pal_run)
+          write([&](uint32_t v) { return run8(v, b4); });
+        else
+          write([&](uint32_t v) { return palette8(v, p0, p1, p2, p3); });
       } else {
         // 4 lanes per chunk, 32 symbols (four rank words, half a 64-weight
         // row) per lane; escape rows are written as zeros

@@ -23,6 +23,7 @@ struct DecodeArgs {
   const uint32_t* lut;        // 4096-entry rank table (see DecodeTables)
   const uint32_t* canon;      // canonical-code tables (kCanonWords words)
   uint32_t palette[4];        // the 16 palette exponents, byte i = rank i
+  uint32_t pal_run_b4;        // palette = the run b..b+15: b in every byte, else 0xFFFFFFFF
   const uint8_t* sm;          // sign+mantissa bytes (full decode only)
   const uint32_t* esc_bits;   // escape bitmap (palette transcode only)
   uint32_t* status;           // device status word (bit 0: bad chunk)

@@ -294,3 +294,45 @@ def test_palette_forms_match_fp64(uw, name, exps, planted, tile_n, halves):
     assert np.array_equal(outs["exp"], outs["palette_rt"])
     assert np.array_equal(outs["exp"], outs["palette_direct"])
     h.free()
+
+
+@pytest.mark.parametrize("pipe", PIPES)
+def test_back_to_back_chain_on_one_stream(uw, pipe):
+    """Launches overlap (each kernel starts its set-up before the one ahead of
+    it ends and waits only before touching that kernel's data): a chain of
+    GEMMs where each X is the previous Y, and preprocessing that reuses one
+    workspace, enqueued with no host synchronisation, must equal the same
+    calls run one at a time."""
+    import torch
+    K = 512
+    ws_w = [synthdata.normal(K, K, 0.02, seed=120 + i) for i in range(3)]
+    hs = [_upload(uw, w, chunk=256) for w in ws_w]
+    M = 24
+    need = max(uw.uw_workspace_bytes(h, uw.PIPELINES[pipe], M) for h in hs)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    for h in hs:
+        uw.uw_set_workspace(h, ws)  # one workspace: each decode overwrites the last one's output
+    x = synthdata.activations(M, K, 121)
+    X0 = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+
+    def chain(sync_each):
+        ys = [X0]
+        for h in hs:
+            Y = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+            uw.uw_gemm(h, ys[-1], Y, M, uw.PIPELINES[pipe])
+            if sync_each:
+                torch.cuda.synchronize()
+            ys.append(Y)
+        torch.cuda.synchronize()
+        return [y.float().cpu().numpy() for y in ys[1:]]
+
+    ref = chain(True)
+    for _ in range(3):
+        got = chain(False)
+        for a, b in zip(ref, got):
+            assert np.array_equal(a, b)
+    # and the first link against the FP64 oracle
+    _check(ref[0].astype(np.float64), x, ws_w[0], bf16_out=True)
+    for h in hs:
+        assert uw.uw_last_device_status(h) == uw.UW_OK
+        h.free()
