@@ -185,6 +185,46 @@ def test_down_proj_full_size_sampled(uw, M):
     h.free()
 
 
+@pytest.fixture(scope="module")
+def gate70b(uw):
+    """The 70B-shaped gate projection (Student-t weights, many escape rows),
+    uploaded once for the tests below."""
+    w = synthdata.workload("gate70b_28672x8192")
+    h = _upload(uw, w)
+    yield w, h
+    h.free()
+
+
+@pytest.mark.parametrize("M", [1, 4096])
+def test_gate70b_shape_sampled(uw, gate70b, M):
+    """28672x8192 with heavy tails: every pipeline within tolerance on sampled
+    token rows (all of them at M = 1), the reconstructive ones bitwise equal."""
+    w, h = gate70b
+    assert h.stats()["n_escape_rows"] > 0
+    x = synthdata.activation_for("gate70b_28672x8192", M)
+    _workspace(uw, h, M)
+    rng = np.random.default_rng(70 + M)
+    rows = np.sort(rng.choice(M, size=min(M, 8), replace=False))
+    ref = oracle.gemm_fp64(x[rows], w)
+    bound = oracle.abs_product_sum(x[rows], w)
+    import torch
+    X = torch.from_numpy(x.view(np.int16)).cuda()
+    Y = torch.empty((M, h.N), dtype=torch.float32, device="cuda")
+    sel = torch.from_numpy(rows).cuda()
+    outs = {}
+    for p in PIPES:
+        Y.fill_(float("nan"))
+        uw.uw_gemm_ex(h, X, Y, M, uw.gemm_config(uw.PIPELINES[p]), True)
+        torch.cuda.synchronize()
+        assert uw.uw_last_device_status(h) == uw.UW_OK
+        y = Y.index_select(0, sel).cpu().numpy().astype(np.float64)  # only the sampled rows leave the GPU
+        ok, worst = oracle.within_tolerance(y, ref, bound)
+        assert ok, (p, worst)
+        outs[p] = y
+    assert np.array_equal(outs["exp"], outs["palette_rt"])
+    assert np.array_equal(outs["exp"], outs["palette_direct"])
+
+
 def test_gemm_argument_errors(uw):
     import ctypes as C
     import torch
