@@ -77,6 +77,10 @@ def _args():
     ap.add_argument("--only", choices=("decode_full", "decode_exp", "transcode", "gemm_bf16",
                                        "gemm_exp", "gemm_palette"))
     ap.add_argument("--m", type=int, default=1, help="tokens for --only gemm_*")
+    # the Llama-3.1-8B-shaped MLP stack end to end (prints its own JSON line)
+    ap.add_argument("--mlp-layers", type=int, default=0,
+                    help="time uw_mlp_forward over this many gate/up/down layers")
+    ap.add_argument("--mlp-ms", default="1,64,256,1024")
     return ap.parse_args()
 
 
@@ -609,10 +613,102 @@ def run_only(args):
     return 0
 
 
+def run_mlp(args):
+    """The 32-layer (or --mlp-layers) MLP stack: gate/up 14336x4096 and down
+    4096x14336 per layer, BF16 ~ N(0, 0.02) with independent seeds, SiLU(gate)
+    * up -> down.  Layer 0's projections are autotuned per M and the profile is
+    applied to every layer; uw_mlp_tune_split picks the preprocessing overlap
+    and SM split; uw_mlp_forward is timed with CUDA events (inputs resident)
+    against the same stack in torch on the uncompressed BF16 weights."""
+    import tempfile
+    import numpy as np
+    import torch
+    import decode_gemm_b200 as uw
+    import synthdata
+
+    L = args.mlp_layers
+    Ms = [int(m) for m in args.mlp_ms.split(",")]
+    D, F = 4096, 14336
+    torch.cuda.set_device(0)
+    layers, wbf = [], []
+    comp = bf = 0
+    for i in range(L):
+        trio, bfs = [], []
+        for j, (n, k) in enumerate(((F, D), (F, D), (D, F))):
+            w = synthdata.normal(n, k, 0.02, 2000 + 3 * i + j)
+            h = uw.uw_encode(w)
+            st = h.stats()
+            comp += st["bytes_palette_bundle"] + st["bytes_stream"] + st["bytes_offsets"]
+            bf += 2 * n * k
+            trio.append(h)
+            bfs.append(torch.from_numpy(w.view(np.int16)).cuda().view(torch.bfloat16))
+            del w
+        layers.append(tuple(trio))
+        wbf.append(bfs)
+    flat0 = list(layers[0])
+    need = max(uw.uw_workspace_bytes(h, p, max(Ms)) for h in flat0 for p in (1, 2, 3, 4))
+    ws0 = torch.empty(need, dtype=torch.uint8, device="cuda")
+    for h in flat0:
+        uw.uw_set_workspace(h, ws0)
+    with tempfile.TemporaryDirectory() as d:
+        prof = os.path.join(d, "profile.json")
+        uw.uw_autotune(flat0, Ms, prof)
+        for trio in layers[1:]:
+            uw.uw_load_profile(list(trio), prof)
+    side = torch.cuda.Stream()
+    out = {}
+    for M in Ms:
+        x = synthdata.activations(M, D, 3000 + M)
+        X = torch.from_numpy(x.view(np.int16)).cuda()
+        Y = torch.empty((M, D), dtype=torch.int16, device="cuda")
+        ws = torch.empty(max(uw.uw_mlp_workspace_bytes(layers, M, uw.mlp_opts(o))
+                             for o in (False, True)), dtype=torch.uint8, device="cuda")
+        best = uw.uw_mlp_tune_split(layers, X, Y, M, ws, side_stream=side)
+
+        def timed(fn, it=5):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(it):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / it
+
+        ours = timed(lambda: uw.uw_mlp_forward(layers, X, Y, M, ws, best, side_stream=side))
+        xb = X.view(torch.bfloat16)
+
+        def ref():
+            cur = xb
+            for g, u, dw in wbf:
+                a, b = cur @ g.t(), cur @ u.t()
+                cur = (torch.nn.functional.silu(a.float()) * b.float()).to(torch.bfloat16) @ dw.t()
+            return cur
+
+        base = timed(ref)
+        for h in flat0:
+            if uw.uw_last_device_status(h) != uw.UW_OK:
+                raise RuntimeError("device status")
+        out[f"M{M}"] = {"ms": ours, "torch_bf16_ms": base, "ratio": ours / base,
+                        "pipelines": [uw.uw_get_choice(h, M)["pipeline"] for h in flat0],
+                        "split": best.as_dict()}
+    print(json.dumps({"mode": "mlp_stack", "layers": L, "unit": "ms per forward",
+                      "weights_bf16_bytes": bf, "weights_compressed_bytes": comp,
+                      "data": "synthetic", "results": out}), flush=True)
+    for trio in layers:
+        for h in trio:
+            h.free()
+    return 0
+
+
 def main():
     args = _args()
     if args.only:
         return run_only(args)
+    if args.mlp_layers > 0:
+        return run_mlp(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
