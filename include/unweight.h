@@ -34,6 +34,14 @@
  *     detected on the host before anything is launched.  Kernel-side errors
  *     (corrupt stream, bounded wait expired) set a status word in the handle,
  *     read by uw_last_device_status.  No call aborts, traps or throws.
+ *   - Launch overlap: every kernel of the library is launched with programmatic
+ *     stream serialization (CUDA programmatic dependent launch).  It may begin
+ *     its set-up (barriers, tensor memory, decode tables, reads of the handle's
+ *     own compressed arrays) while the kernel before it on the stream is still
+ *     running, and waits for that kernel to complete (griddepcontrol.wait)
+ *     before it reads or writes anything else: X, Y, workspaces, outputs.  So
+ *     stream order holds for the caller's buffers exactly as with ordinary
+ *     launches, also when the kernel before is the caller's own.
  *   - Thread safety: a handle may be used by one host thread at a time.
  */
 #ifndef UNWEIGHT_H
