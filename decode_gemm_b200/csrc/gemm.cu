@@ -73,9 +73,11 @@ constexpr int kRebuildWarp0 = kEpiWarp0 + kNumEpiWarps;
 constexpr uint32_t kEpiSleepNs = 200;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
 
-__host__ __device__ constexpr int threads_for(int mode) {
-  return (mode == kGemmBf16 ? kRebuildWarp0 : kRebuildWarp0 + kNumRebuildWarps) * 32;
+// The X producer is the last warp.
+__host__ __device__ constexpr int x_warp_for(int mode) {
+  return mode == kGemmBf16 ? kRebuildWarp0 : kRebuildWarp0 + kNumRebuildWarps;
 }
+__host__ __device__ constexpr int threads_for(int mode) { return (x_warp_for(mode) + 1) * 32; }
 
 struct GemmParams {
   CUtensorMap tm_x;   // X [M, K] bf16, box {64, tile_n}, 128B swizzle
@@ -98,6 +100,7 @@ struct GemmParams {
   int32_t halves;    // 128-row halves per unit: 1, or 2 for the wide (large-M) shape
   int32_t acc_bufs;  // TMEM accumulator sets (2: epilogue overlaps the next tile)
   int32_t NG;        // 128-row groups of W (escape groups per K block)
+  int32_t xstages;   // X ring depth (the units' X tiles ride their own ring)
   int32_t tmem_w;    // W slots in TMEM (MMA A from TMEM) rather than shared memory
   uint32_t wcol0;    // first TMEM column of the W slots
   const uint8_t* pf_s;   // the handle's sign+mantissa array, for early L2 prefetch
@@ -114,19 +117,21 @@ struct StageLayout {
   uint32_t x, w0, w1, ebits, erows, bytes;
 };
 
-// A stage holds ks X tiles (one per K block), then the unit's W data: the TMA
-// boxes cover all H*128 rows and ks K blocks at once (row-major inside a box,
-// 64*ks sign+mantissa or exponent bytes, 32*ks index bytes per row).  Palette
-// escape data has one area per (half, K block) part (H * ks <= 2): a 16-byte
-// bitmap, then up to kEscCap rows (kEscArea bytes).
+// A load stage holds the unit's W data: the TMA boxes cover all H*128 rows
+// and ks K blocks at once (row-major inside a box, 64*ks sign+mantissa or
+// exponent bytes, 32*ks index bytes per row).  Palette escape data has one
+// area per (half, K block) part (H * ks <= 2): a 16-byte bitmap, then up to
+// kEscCap rows (kEscArea bytes).  The units' X tiles (ks per unit) ride a
+// separate, shallower ring: they come from L2, while W needs a deep ring to
+// keep HBM busy.
 constexpr uint32_t kEscArea = 16 + kEscCap * 64;
 
 __host__ __device__ inline StageLayout stage_layout(int mode, int tile_n, int halves, int ks) {
   StageLayout L;
-  L.x = 0;
-  const uint32_t xb = (uint32_t)tile_n * kBK * 2;  // multiple of 2048 for tile_n % 16 == 0
-  const uint32_t HK = (uint32_t)(halves * ks);      // 128x64 W blocks per stage
-  L.w0 = (uint32_t)ks * xb;
+  (void)tile_n;
+  L.x = 0;  // (X has its own ring)
+  const uint32_t HK = (uint32_t)(halves * ks);  // 128x64 W blocks per stage
+  L.w0 = 0;
   if (mode == kGemmBf16) {
     L.w1 = L.ebits = L.erows = L.w0 + HK * kWTileBytes;
     L.bytes = L.w0 + HK * kWTileBytes;
@@ -223,14 +228,17 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   const int H = p.halves;
   const bool wide = H == 2;
   const int RU = kBM * H;  // W rows per unit
+  const int SX = p.xstages;
+  const uint32_t xst_bytes = (uint32_t)KS_ * p.x_bytes;  // one unit's X tiles
   uint8_t* ring = smem;
-  uint8_t* wring = ring + (size_t)S * L.bytes;  // rebuilt W tiles (reconstructive modes)
+  uint8_t* xring = ring + (size_t)S * L.bytes;       // X tiles
+  uint8_t* wring = xring + (size_t)SX * xst_bytes;  // rebuilt W tiles (shared-memory path)
   uint8_t* tail = wring + (size_t)(p.tmem_w ? 0 : WS) * kWTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   // barrier indices
-  const int b_full = 0, b_empty = S, b_wfull = 2 * S, b_wfree = 2 * S + WS,
-            b_tfull = 2 * S + 2 * WS, b_tempty = b_tfull + 2, b_drain = b_tempty + 2,
-            b_part = b_drain + 2;
+  const int b_full = 0, b_empty = S, b_xfull = 2 * S, b_xempty = 2 * S + SX,
+            b_wfull = 2 * S + 2 * SX, b_wfree = b_wfull + WS, b_tfull = b_wfree + WS,
+            b_tempty = b_tfull + 2, b_drain = b_tempty + 2, b_part = b_drain + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + b_part + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -241,9 +249,13 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(bar(b_full + s), 1);
-      // released by each half's MMA commit and, reconstructive modes, its
-      // rebuild group's warps
-      mbar_init(bar(b_empty + s), (uint32_t)H * (1 + (MODE == kGemmBf16 ? 0 : kGroupWarps)));
+      // released by each half's reader: its MMA commit (BF16 tiles) or its
+      // rebuild group's warps (compressed tiles)
+      mbar_init(bar(b_empty + s), (uint32_t)H * (MODE == kGemmBf16 ? 1 : kGroupWarps));
+    }
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(bar(b_xfull + s), 1);
+      mbar_init(bar(b_xempty + s), (uint32_t)H);  // each half's MMA commit
     }
     for (int w = 0; w < WS; ++w) {
       mbar_init(bar(b_wfull + w), kGroupWarps);
@@ -309,7 +321,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   // the first stage lands) pull the first ring's immutable weight rows into
   // L2, so the first loads after the wait hit L2.
   if (threadIdx.x == 0) pdl_release();
-  if (MODE != kGemmBf16 && warp >= kRebuildWarp0 && H == 1) {
+  if (MODE != kGemmBf16 && warp >= kRebuildWarp0 && warp < kRebuildWarp0 + kNumRebuildWarps &&
+      H == 1) {
     const int64_t n_pf = imin64(u1 - u0, S);
     const int rt = threadIdx.x - kRebuildWarp0 * 32;
     for (int64_t i = rt; i < n_pf * kBM; i += kNumRebuildWarps * 32) {
@@ -337,8 +350,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int64_t t = u / KB;
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
-      const int64_t nt = t / p.MT, mt = t - nt * p.MT;
-      const int32_t n0 = (int32_t)(nt * RU), m0 = (int32_t)(mt * p.tile_n);
+      const int64_t nt = t / p.MT;
+      const int32_t n0 = (int32_t)(nt * RU);
       for (int kb = kb0; kb < kb1; ++kb, ++qi) {
         uint32_t c0[2] = {0u, 0u}, c1[2] = {0u, 0u};
         if (MODE == kGemmPalette) {
@@ -363,7 +376,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           } else {
             uint8_t* st = ring + (size_t)stage * L.bytes;
             const uint32_t fb = bar(b_full + stage);
-            uint32_t bytes = p.x_bytes * KS;
+            uint32_t bytes = 0;
             if (MODE == kGemmBf16) bytes += NP * kWTileBytes;
             if (MODE == kGemmExp) bytes += NP * 16384;
             // escape rows of each part's 128-row group and K block: one copy of
@@ -390,9 +403,6 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             }
             mbar_expect_tx(fb, bytes);
             const int kbk = kb * KS;  // first K block of the unit
-#pragma unroll
-            for (int j = 0; j < KS; ++j)
-              tma_load_2d(smem_u32(st + L.x + j * p.x_bytes), &p.tm_x, fb, (kbk + j) * kBK, m0);
             tma_load_2d(smem_u32(st + L.w0), &p.tm_w0, fb, kbk * kBK, n0);
             if (MODE == kGemmExp) tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kbk * kBK, n0);
             if (MODE == kGemmPalette) {
@@ -447,8 +457,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const uint32_t idesc = idesc_bf16(kBM, p.tile_n);
       const int WP = wide ? WS / 2 : WS;  // W slot positions this warp cycles through
       // ring positions of the current unit, advanced for every unit of the CTA
-      int stage = 0, wpos = 0;
-      uint32_t phase = 0, wphase = 0;
+      int stage = 0, wpos = 0, xs = 0;
+      uint32_t phase = 0, wphase = 0, xph = 0;
       int q = 0;  // index of the unit among this CTA's units
       int seg = 0;
       bool ok = true;
@@ -472,7 +482,11 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           const bool mine = wide || NM == 1 || (q & 1) == par;
           const int wslot = wide ? 2 * wpos + par : wpos;
           if (mine && lane == 0) {
-            bool got = mbar_wait_bounded(bar(b_full + stage), phase, abort, p.wait_ns);
+            // A: BF16 tiles from the load stage, rebuilt tiles from their slot;
+            // B: the unit's X tiles from the X ring
+            bool got = true;
+            if (MODE == kGemmBf16) got = mbar_wait_bounded(bar(b_full + stage), phase, abort, p.wait_ns);
+            if (got) got = mbar_wait_bounded(bar(b_xfull + xs), xph, abort, p.wait_ns);
             if (got && MODE != kGemmBf16)
               got = mbar_wait_bounded(bar(b_wfull + wslot), wphase, abort, p.wait_ns);
             if (!got) {
@@ -481,14 +495,15 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             } else {
               tc_fence_after();
               uint8_t* st = ring + (size_t)stage * L.bytes;
-              const uint64_t b_desc = smem_desc_sw128(smem_u32(st + L.x));
+              uint8_t* xt = xring + (size_t)xs * xst_bytes;
+              const uint64_t b_desc = smem_desc_sw128(smem_u32(xt));
               if (MODE != kGemmBf16 && p.tmem_w) {
                 // A: 32 columns of the slot per K block, 8 per 16-wide K step;
                 // B: the K block's X tile
                 const uint32_t a_tmem = tmem_base + p.wcol0 + (uint32_t)(wslot * 32 * KS);
 #pragma unroll
                 for (int j = 0; j < KS; ++j) {
-                  const uint64_t bj = smem_desc_sw128(smem_u32(st + L.x + j * p.x_bytes));
+                  const uint64_t bj = smem_desc_sw128(smem_u32(xt + j * p.x_bytes));
 #pragma unroll
                   for (int k = 0; k < kBK / 16; ++k)
                     mma_bf16_tmem_a(d_tmem, a_tmem + 32 * j + 8 * k, bj + 2 * k, idesc,
@@ -504,7 +519,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
                   mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
                            (!first || k > 0) ? 1u : 0u);
               }
-              mma_commit(bar(b_empty + stage));
+              if (MODE == kGemmBf16) mma_commit(bar(b_empty + stage));
+              mma_commit(bar(b_xempty + xs));
               if (MODE != kGemmBf16) mma_commit(bar(b_wfree + wslot));
             }
           }
@@ -514,6 +530,10 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
+          }
+          if (++xs == SX) {
+            xs = 0;
+            xph ^= 1u;
           }
           if (WP && ++wpos == WP) {
             wpos = 0;
@@ -688,6 +708,58 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       if (lane == 0) mbar_arrive(bar(b_tempty + acc));
       u += kb1 - kb0;
       qa += kb1 - kb0;
+    }
+  } else if (warp == x_warp_for(MODE)) {
+    // ---------------------------------------------------------- X producer --
+    // The units' X tiles (K blocks of the token tile), in unit order, into
+    // their own ring: X comes from L2 and needs few stages in flight, so the
+    // load ring's depth goes to W.
+    int xs = 0;
+    uint32_t xph = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t u = u0; u < u1 && ok;) {
+      const int64_t t = u / KB;
+      const int kb0 = (int)(u - t * KB);
+      const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
+      const int32_t m0 = (int32_t)((t - (t / p.MT) * p.MT) * p.tile_n);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (lane == 0) {
+          if (!mbar_wait_bounded(bar(b_xempty + xs), xph ^ 1u, abort, p.wait_ns)) {
+            set_abort(abort, p.status);
+            ok = false;
+          } else {
+            const uint32_t fb = bar(b_xfull + xs);
+            uint8_t* xt = xring + (size_t)xs * xst_bytes;
+            mbar_expect_tx(fb, xst_bytes);
+#pragma unroll
+            for (int j = 0; j < KS; ++j)
+              tma_load_2d(smem_u32(xt + j * p.x_bytes), &p.tm_x, fb, (kb * KS + j) * kBK, m0);
+            ++issued;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (++xs == SX) {
+          xs = 0;
+          xph ^= 1u;
+        }
+      }
+      u += kb1 - kb0;
+    }
+    // in-flight copies must land before the CTA exits
+    if (lane == 0 && *abort) {
+      const int64_t outstanding = issued < SX ? issued : SX;
+      int s = xs;
+      uint32_t ph = xph;
+      for (int64_t i = 0; i < outstanding; ++i) {
+        if (--s < 0) {
+          s = SX - 1;
+          ph ^= 1u;
+        }
+        volatile int no_abort = 0;
+        mbar_wait_bounded(bar(b_xfull + s), ph, &no_abort, p.wait_ns);
+      }
     }
   } else if constexpr (MODE != kGemmBf16) {
     // ------------------------------------------------------------- rebuild --
@@ -1014,13 +1086,14 @@ int tmem_ks_for(const GemmArgs& a) {
   return 0;
 }
 
-size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool tmem_w, int ks) {
+size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool tmem_w, int ks,
+                  int xstages) {
   const StageLayout L = stage_layout(mode, tile_n, halves, ks);
-  if (tmem_w) wslots = 0;  // the W slots live in TMEM
-  const int ws = mode == kGemmBf16 ? 0 : wslots;
+  const int ws = mode == kGemmBf16 ? 0 : wslots;  // W slots (their barriers exist either way)
   size_t b = 1024 /* alignment slack */ + (size_t)stages * L.bytes;
-  b += (size_t)ws * kWTileBytes;
-  b += (size_t)(2 * stages + 2 * ws + 7) * 8 + 16;
+  b += (size_t)xstages * ks * tile_n * kBK * 2;     // X ring
+  if (!tmem_w) b += (size_t)ws * kWTileBytes;       // (TMEM path: the slots live in TMEM)
+  b += (size_t)(2 * stages + 2 * xstages + 2 * ws + 7) * 8 + 16;
   return b;
 }
 
@@ -1068,12 +1141,23 @@ bool gemm_resolve(GemmArgs* a) {
   const int tks = tmem_ks_for(*a);
   a->tmem_w = tks > 0;
   a->ks = tks > 0 ? tks : 1;
+  // X ring: X tiles come from L2; about 48 KB in flight where a rebuild paces
+  // the units, 96 KB (128 KB for 256-token tiles) for the BF16 GEMM whose MMAs
+  // take units as fast as they land (measured: 32 KB starved it at M = 256);
+  // 2..8 units, an even number when two MMA warps alternate units
+  {
+    const int xunit = a->ks * a->tile_n * kBK * 2;
+    int sx = (a->mode == kGemmBf16 ? (a->tile_n > 128 ? 131072 : 98304) : 49152) / xunit;
+    sx = sx < 2 ? 2 : (sx > 8 ? 8 : sx);
+    if (!wide && mma_warps_for(a->tile_n) == 2) sx &= ~1;
+    a->xstages = sx;
+  }
   if (a->stages == 0) {
     for (;;) {
       int s = max_stages;
-      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks) > (size_t)kSmemLimit)
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages) > (size_t)kSmemLimit)
         s -= step;
-      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks) <= (size_t)kSmemLimit ||
+      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages) <= (size_t)kSmemLimit ||
           a->wslots <= 2 || wide) {
         a->stages = s;
         break;
@@ -1082,7 +1166,7 @@ bool gemm_resolve(GemmArgs* a) {
     }
   }
   if (a->stages < 2 || (!wide && (a->stages & 1)) ||
-      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, a->tmem_w, a->ks) > (size_t)kSmemLimit)
+      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages) > (size_t)kSmemLimit)
     return false;
   const int64_t RU = (int64_t)kBM * a->halves;
   const int64_t NT = (a->N + RU - 1) / RU;
@@ -1152,6 +1236,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.K = a.K;
   p.tile_n = a.tile_n;
   p.stages = a.stages;
+  p.xstages = a.xstages;
+  if (p.xstages < 2 || (!wide && mma_warps_for(a.tile_n) == 2 && (p.xstages & 1)))
+    return cudaErrorInvalidValue;  // unresolved
   p.wslots = a.wslots;
   p.NT = (int32_t)((a.N + RU - 1) / RU);
   p.NG = (int32_t)((a.N + kBM - 1) / kBM);
@@ -1178,7 +1265,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.x_bytes = (uint32_t)a.tile_n * kBK * 2;
   p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves, KS).bytes;
   p.wait_ns = wait_limit_ns();
-  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS);
+  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS, a.xstages);
   const int G = a.ctas;
   cudaError_t e = cudaSuccess;
   auto begin = [&](int kind) { return hooks && hooks->begin ? hooks->begin(hooks->ctx, kind) : -1; };

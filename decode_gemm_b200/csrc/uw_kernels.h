@@ -86,6 +86,7 @@ struct GemmArgs {
   int stages = 0;                // load ring depth (0 = auto)
   int wslots = 0;                // rebuilt-W ring depth (0 = auto)
   int ks = 0;                    // resolved: 64-wide K blocks per unit (stage)
+  int xstages = 0;               // resolved: X ring depth
   int tmem_w = 0;                // resolved: W rebuilt into TMEM (else shared memory)
   int ctas = 0;                  // persistent CTAs (0 = SM count)
   int sm_count = 148;
