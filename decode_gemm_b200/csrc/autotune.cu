@@ -53,9 +53,10 @@ std::vector<uw_gemm_config> candidates(const uw_handle_s* h, int64_t M) {
     for (int t : tiles)
       for (int st : {0, 4})
         for (int hv : {0, 1, 2}) {
-          // the wide shape only pays from a few token tiles on
+          // the wide shape (on request only) could pay from a few token
+          // tiles on; one half per unit is the automatic choice
           if (hv == 2 && M < 256) continue;
-          if (hv == 1 && M < 512) continue;  // already the automatic choice
+          if (hv == 1) continue;
           uw_gemm_config c;
           std::memset(&c, 0, sizeof(c));
           c.pipeline = p;

@@ -59,7 +59,7 @@ constexpr int kEscCap = 15;        // escape rows staged per stage (more: read f
                                    // 15 keeps a 16-token palette stage at 15 KB
 constexpr int kMaxWSlots = 8;      // rebuilt-W ring depth (runtime, <= this)
 constexpr int kMaxStages = 16;     // load ring depth (runtime, <= this)
-constexpr int64_t kWideMinM = 512;  // tokens from which units span 256 W rows
+constexpr int64_t kWideMinM = 512;  // tokens from which the BF16 GEMM uses 256-token tiles
 constexpr int kNumEpiWarps = 4;
 constexpr int kNumRebuildWarps = 8;  // two groups of 4, alternating stages
 constexpr int kGroupWarps = kNumRebuildWarps / 2;
@@ -1108,22 +1108,29 @@ cudaError_t set_smem_attr() {
 
 bool gemm_resolve(GemmArgs* a) {
   if (a->M <= 0 || a->N <= 0 || a->K <= 0 || a->K % kBK) return false;
-  // Wide shape (256 W rows per unit, one 128-row half per rebuild group and
-  // MMA warp) from M = 512 on: X is then read once per 256 rows instead of
-  // 128.  Token tiles: all of M up to 128 tokens, 128 above (measured on
-  // 14336x4096: at M = 256 128-token tiles beat one 256-token tile by 13-16%;
-  // 256-token wide tiles fill TMEM, so an epilogue stalls the next tile).
-  // (The plain BF16 GEMM rebuilds nothing, so for it the wide shape only
-  // trades X traffic for TMEM room: it keeps 128-row units, with one 256-token
-  // tile from M = 512.)
-  if (a->halves == 0) a->halves = (a->mode != kGemmBf16 && a->M >= kWideMinM) ? 2 : 1;
+  // Defaults (measured with X on its own ring, 14336x4096, 4096x14336 and
+  // 28672x8192): 128-row units (the wide 256-row shape only on request: it
+  // halves the X reads per W row but, with X off the load stage, one
+  // 256-token tile that rebuilds W once per 256 tokens wins, e.g. palette
+  // M = 1024 on 14336x4096: 171 us against 218).  Token tiles: all of M up
+  // to 128 tokens; the reconstructive modes use one tile up to 256 tokens
+  // when the matrix has enough 128-row tiles to keep the K splits short
+  // (otherwise, 4096x14336 at M = 256: 90 us with 128-token tiles against 102),
+  // and 256-token tiles above; the BF16 GEMM keeps 128-token tiles below
+  // M = 512 and 256 from there.
+  if (a->halves == 0) a->halves = 1;
   if (a->halves != 1 && a->halves != 2) return false;
   const bool wide = a->halves == 2;
   if (a->tile_n == 0) {
+    const int64_t row_tiles = (a->N + kBM - 1) / kBM;
     if (a->M <= 128)
       a->tile_n = (int)((a->M + 15) / 16 * 16);
+    else if (a->mode == kGemmBf16)
+      a->tile_n = a->M >= kWideMinM ? 256 : 128;
+    else if (a->M <= 256)
+      a->tile_n = 3 * row_tiles >= 2 * (int64_t)a->sm_count ? (int)((a->M + 15) / 16 * 16) : 128;
     else
-      a->tile_n = (a->mode == kGemmBf16 && a->M >= kWideMinM) ? 256 : 128;
+      a->tile_n = 256;
   }
   if (a->tile_n < 16 || a->tile_n > 256 || a->tile_n % 16) return false;
   // One half per unit: ring depths are even, consumers alternate units, so an

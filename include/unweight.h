@@ -141,12 +141,12 @@ typedef struct uw_stats_t {
 typedef struct uw_gemm_config {
   int32_t pipeline;      /* uw_pipeline, not AUTO                                  */
   int32_t tile_n;        /* tokens per MMA tile: 16..256, multiple of 16 (0=auto)  */
-  int32_t stages;        /* shared-memory ring depth, 2..16, even unless halves=2
-                            (0 = auto)                                              */
+  int32_t stages;        /* weight load-ring depth, 2..16, even unless halves=2
+                            (0 = auto; X tiles have their own, automatic ring)      */
   int32_t gemm_ctas;     /* persistent GEMM CTAs (0 = one per SM)                   */
   int32_t decode_ctas;   /* SMs (one CTA each) of the preprocessing kernel (0 = all) */
-  int32_t halves;        /* W rows per GEMM unit / 128: 1, or 2 (the wide shape for
-                            large M: X is read once per 256 rows); 0 = by M         */
+  int32_t halves;        /* W rows per GEMM unit / 128: 1, or 2 (the wide shape: X
+                            is read once per 256 rows); 0 = 1                       */
   int32_t reserved[2];
 } uw_gemm_config;
 
