@@ -1149,12 +1149,15 @@ bool gemm_resolve(GemmArgs* a) {
   a->tmem_w = tks > 0;
   a->ks = tks > 0 ? tks : 1;
   // X ring: X tiles come from L2; about 48 KB in flight where a rebuild paces
-  // the units, 96 KB (128 KB for 256-token tiles) for the BF16 GEMM whose MMAs
-  // take units as fast as they land (measured: 32 KB starved it at M = 256);
-  // 2..8 units, an even number when two MMA warps alternate units
+  // the units (96 KB for 256-token tiles: 4096x14336 palette M = 1024 198 ->
+  // 170 us), 96 KB (128 KB for 256-token tiles) for the BF16 GEMM whose MMAs
+  // take units as fast as they land (32 KB starved it at M = 256); 2..8
+  // units, an even number when two MMA warps alternate units
   {
     const int xunit = a->ks * a->tile_n * kBK * 2;
-    int sx = (a->mode == kGemmBf16 ? (a->tile_n > 128 ? 131072 : 98304) : 49152) / xunit;
+    const int x_target = a->mode == kGemmBf16 ? (a->tile_n > 128 ? 131072 : 98304)
+                                              : (a->tile_n > 128 ? 98304 : 49152);
+    int sx = x_target / xunit;
     sx = sx < 2 ? 2 : (sx > 8 ? 8 : sx);
     if (!wide && mma_warps_for(a->tile_n) == 2) sx &= ~1;
     a->xstages = sx;
