@@ -83,6 +83,7 @@ struct GemmParams {
   CUtensorMap tm_x;   // X [M, K] bf16, box {64, tile_n}, 128B swizzle
   CUtensorMap tm_w0;  // bf16 mode: W [N, K] box {64, 128} 128B swizzle; else S [N, K] u8 box {64,128}
   CUtensorMap tm_w1;  // exp mode: E [N, K] u8 box {64, 128}; palette mode: I [N, K/2] u8 box {32, 128}
+  CUtensorMap tm_y;   // Y [M, N] bf16, box {128, 16} (when y_tma)
   const uint32_t* esc_bits;
   const uint32_t* esc_off;
   const uint8_t* esc_exp;
@@ -101,6 +102,7 @@ struct GemmParams {
   int32_t acc_bufs;  // TMEM accumulator sets (2: epilogue overlaps the next tile)
   int32_t NG;        // 128-row groups of W (escape groups per K block)
   int32_t xstages;   // X ring depth (the units' X tiles ride their own ring)
+  int32_t y_tma;     // BF16 Y written by TMA stores of 16-token blocks
   int32_t tmem_w;    // W slots in TMEM (MMA A from TMEM) rather than shared memory
   uint32_t wcol0;    // first TMEM column of the W slots
   const uint8_t* pf_s;   // the handle's sign+mantissa array, for early L2 prefetch
@@ -125,6 +127,8 @@ struct StageLayout {
 // separate, shallower ring: they come from L2, while W needs a deep ring to
 // keep HBM busy.
 constexpr uint32_t kEscArea = 16 + kEscCap * 64;
+// One epilogue block of Y staged for a TMA store: 16 tokens x 128 rows, BF16.
+constexpr uint32_t kYBlockBytes = 16 * kBM * 2;
 
 __host__ __device__ inline StageLayout stage_layout(int mode, int tile_n, int halves, int ks) {
   StageLayout L;
@@ -233,7 +237,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   uint8_t* ring = smem;
   uint8_t* xring = ring + (size_t)S * L.bytes;       // X tiles
   uint8_t* wring = xring + (size_t)SX * xst_bytes;  // rebuilt W tiles (shared-memory path)
-  uint8_t* tail = wring + (size_t)(p.tmem_w ? 0 : WS) * kWTileBytes;
+  uint8_t* ystage = wring + (size_t)(p.tmem_w ? 0 : WS) * kWTileBytes;  // 2 x [16][128] BF16
+  uint8_t* tail = ystage + (p.y_tma ? 2 * kYBlockBytes : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   // barrier indices
   const int b_full = 0, b_empty = S, b_xfull = 2 * S, b_xempty = 2 * S + SX,
@@ -305,6 +310,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&p.tm_x);
     prefetch_tensormap(&p.tm_w0);
+    if (p.y_tma) prefetch_tensormap(&p.tm_y);
     if (MODE != kGemmBf16) prefetch_tensormap(&p.tm_w1);
   }
   if (warp == kMmaWarp0) {
@@ -561,6 +567,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     // last CTA, constant while this launch runs) plus one
     const uint32_t tag = __ldcg(p.sync) + 1u;
     const int64_t part_stride = (int64_t)p.tile_n * RU;  // a CTA's partial-sum tile
+    int yblk = 0;  // Y blocks stored through the staging buffers
     int seg = 0;
     int64_t qa = 0;  // index (among this CTA's units) of the segment's first unit
     for (int64_t u = u0; u < u1; ++seg) {
@@ -684,7 +691,24 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
               for (int j = 0; j < 16; ++j) v[j] += pv[j];
             }
           }
-          if (n < p.N) {
+          if (KS_ == 1 && p.y_tma) {
+            // (128+-token tiles always run with one K block per unit)
+            // the block as [token][row] BF16 in shared memory, then one TMA
+            // store of 16 token rows of 128 outputs each (parts past M or N are
+            // not written); two buffers, so a store overlaps the next block
+            uint16_t* yb = reinterpret_cast<uint16_t*>(ystage + (yblk & 1) * kYBlockBytes);
+            if (leader) bulk_wait_read<1>();  // this buffer's previous store has read it
+            epi_sync();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) yb[j * kBM + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+            fence_proxy_async_smem();
+            epi_sync();
+            if (leader && nt * RU + h * kBM < p.N) {  // (a box wholly past N writes nothing)
+              tma_store_2d(&p.tm_y, smem_u32(yb), (int32_t)(nt * RU + h * kBM), (int32_t)(m0 + c));
+              bulk_commit();
+            }
+            ++yblk;
+          } else if (n < p.N) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               if (c + j < cols) {
@@ -709,6 +733,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       u += kb1 - kb0;
       qa += kb1 - kb0;
     }
+    // the stores must have read the staging buffers (and landed) before exit
+    if (KS_ == 1 && leader && p.y_tma) bulk_wait_all();
   } else if (warp == x_warp_for(MODE)) {
     // ---------------------------------------------------------- X producer --
     // The units' X tiles (K blocks of the token tile), in unit order, into
@@ -1087,12 +1113,13 @@ int tmem_ks_for(const GemmArgs& a) {
 }
 
 size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool tmem_w, int ks,
-                  int xstages) {
+                  int xstages, bool y_tma) {
   const StageLayout L = stage_layout(mode, tile_n, halves, ks);
   const int ws = mode == kGemmBf16 ? 0 : wslots;  // W slots (their barriers exist either way)
   size_t b = 1024 /* alignment slack */ + (size_t)stages * L.bytes;
   b += (size_t)xstages * ks * tile_n * kBK * 2;     // X ring
   if (!tmem_w) b += (size_t)ws * kWTileBytes;       // (TMEM path: the slots live in TMEM)
+  if (y_tma) b += 2 * kYBlockBytes;                 // Y staging
   b += (size_t)(2 * stages + 2 * xstages + 2 * ws + 7) * 8 + 16;
   return b;
 }
@@ -1145,6 +1172,12 @@ bool gemm_resolve(GemmArgs* a) {
   if (a->mode != kGemmBf16 &&
       (a->wslots < 2 || a->wslots > kMaxWSlots || (a->wslots & 1)))
     return false;
+  // BF16 Y by TMA stores of 16-token blocks, for token tiles of 128 and more
+  // (per-thread 2-byte stores of 256-token tiles cost 20 us at M = 1024;
+  // for small tiles the store's completion at the end costs more than it
+  // saves), when a tensor map can describe Y (row pitch a multiple of 16 B)
+  // and the staging leaves the load ring at least 4 stages (checked below)
+  a->y_tma = !a->out_f32 && a->N % 8 == 0 && a->tile_n >= 128;
   const int tks = tmem_ks_for(*a);
   a->tmem_w = tks > 0;
   a->ks = tks > 0 ? tks : 1;
@@ -1163,20 +1196,26 @@ bool gemm_resolve(GemmArgs* a) {
     a->xstages = sx;
   }
   if (a->stages == 0) {
+    const int wslots0 = a->wslots;
     for (;;) {
       int s = max_stages;
-      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages) > (size_t)kSmemLimit)
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma) > (size_t)kSmemLimit)
         s -= step;
-      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages) <= (size_t)kSmemLimit ||
+      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma) <= (size_t)kSmemLimit ||
           a->wslots <= 2 || wide) {
         a->stages = s;
+        if (a->y_tma && s < 4) {  // the staging would cost too much of the load ring
+          a->y_tma = 0;
+          a->wslots = wslots0;
+          continue;
+        }
         break;
       }
       a->wslots -= 2;
     }
   }
   if (a->stages < 2 || (!wide && (a->stages & 1)) ||
-      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages) > (size_t)kSmemLimit)
+      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma) > (size_t)kSmemLimit)
     return false;
   const int64_t RU = (int64_t)kBM * a->halves;
   const int64_t NT = (a->N + RU - 1) / RU;
@@ -1247,6 +1286,13 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.tile_n = a.tile_n;
   p.stages = a.stages;
   p.xstages = a.xstages;
+  p.y_tma = 0;
+  if (a.y_tma && KS == 1) {
+    if (!make_map_2d(&p.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.Y, (uint64_t)a.N,
+                     (uint64_t)a.M, kBM, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    p.y_tma = 1;
+  }
   if (p.xstages < 2 || (!wide && mma_warps_for(a.tile_n) == 2 && (p.xstages & 1)))
     return cudaErrorInvalidValue;  // unresolved
   p.wslots = a.wslots;
@@ -1275,7 +1321,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.x_bytes = (uint32_t)a.tile_n * kBK * 2;
   p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves, KS).bytes;
   p.wait_ns = wait_limit_ns();
-  const size_t smem = smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS, a.xstages);
+  const size_t smem =
+      smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS, a.xstages, a.y_tma != 0);
   const int G = a.ctas;
   cudaError_t e = cudaSuccess;
   auto begin = [&](int kind) { return hooks && hooks->begin ? hooks->begin(hooks->ctx, kind) : -1; };

@@ -87,6 +87,7 @@ struct GemmArgs {
   int wslots = 0;                // rebuilt-W ring depth (0 = auto)
   int ks = 0;                    // resolved: 64-wide K blocks per unit (stage)
   int xstages = 0;               // resolved: X ring depth
+  int y_tma = 0;                 // resolved: BF16 Y through TMA stores
   int tmem_w = 0;                // resolved: W rebuilt into TMEM (else shared memory)
   int ctas = 0;                  // persistent CTAs (0 = SM count)
   int sm_count = 148;
