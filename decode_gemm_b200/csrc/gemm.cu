@@ -923,12 +923,15 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
                 wv[2 * m + 1] = w2.y;
               }
             }
+            // (the store reads its registers at issue: the next K block may
+            // reuse them without waiting for the store to land)
             tmem_st32(tcol + (uint32_t)(32 * j), wv);
-            tmem_st_wait();  // wv is reused by the next K block
           }
-          // the stage's inputs are consumed: release it, then hand the slot over
+          // the stage's inputs are consumed: release it; once the unit's
+          // stores have landed, hand the slot over
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(b_empty + cur_stage));
+          tmem_st_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(b_wfull + cur_wslot));
