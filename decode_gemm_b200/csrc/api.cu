@@ -165,6 +165,7 @@ uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
   a.tile_n = cfg.tile_n;
   a.stages = cfg.stages;
   a.halves = cfg.halves;
+  a.pair = cfg.pair ? 1 : -1;
   a.ctas = cfg.gemm_ctas;
   switch (cfg.pipeline) {
     case UW_PIPE_FULL: a.mode = kGemmBf16; break;
@@ -185,6 +186,8 @@ uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg) {
   if (cfg.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) return UW_ERR_UNSUPPORTED;
   if (cfg.tile_n < 0 || cfg.tile_n > 256 || cfg.tile_n % 16) return UW_ERR_ARG;
   if (cfg.halves < 0 || cfg.halves > 2) return UW_ERR_ARG;
+  if (cfg.pair < 0 || cfg.pair > 1 || (cfg.pair && cfg.halves == 2)) return UW_ERR_ARG;
+  if (cfg.pair && cfg.pipeline != UW_PIPE_FULL) return UW_ERR_UNSUPPORTED;
   if (cfg.stages < 0 || cfg.stages > 16 || (cfg.halves != 2 && (cfg.stages & 1)))
     return UW_ERR_ARG;
   if (cfg.gemm_ctas < 0 || cfg.decode_ctas < 0) return UW_ERR_ARG;

@@ -64,6 +64,12 @@ std::vector<uw_gemm_config> candidates(const uw_handle_s* h, int64_t M) {
           c.stages = st;
           c.halves = hv;
           out.push_back(c);
+          // the BF16 GEMM on CTA pairs (256-token tiles)
+          if (p == UW_PIPE_FULL && M >= 256 && hv != 2 && (t == 0 || t == 256)) {
+            c.pair = 1;
+            c.tile_n = 256;
+            out.push_back(c);
+          }
         }
   }
   return out;
@@ -328,9 +334,10 @@ uw_status uw_autotune(uw_handle_t* hs_in, int32_t n_handles, const int64_t* Ms, 
         const auto& c = chosen[i][j].second;
         std::fprintf(f,
                      "      {\"M\": %lld, \"pipeline\": %d, \"tile_n\": %d, \"stages\": %d, "
-                     "\"gemm_ctas\": %d, \"decode_ctas\": %d, \"halves\": %d, \"us\": %.2f}%s\n",
+                     "\"gemm_ctas\": %d, \"decode_ctas\": %d, \"halves\": %d, \"pair\": %d, "
+                     "\"us\": %.2f}%s\n",
                      (long long)chosen[i][j].first, c.pipeline, c.tile_n, c.stages, c.gemm_ctas,
-                     c.decode_ctas, c.halves, 1e3 * chosen_ms[i][j],
+                     c.decode_ctas, c.halves, c.pair, 1e3 * chosen_ms[i][j],
                      j + 1 < chosen[i].size() ? "," : "");
       }
       std::fprintf(f, "    ]}%s\n", i + 1 < hs.size() ? "," : "");
@@ -367,7 +374,7 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
     const JVal* ch = hv.get("choices");
     if (!ch || ch->kind != JVal::Arr) return UW_ERR_FORMAT;
     for (const JVal& c : ch->arr) {
-      int64_t M = 0, pl = 0, tn = 0, sg = 0, gc = 0, dc = 0, hv2 = 0;
+      int64_t M = 0, pl = 0, tn = 0, sg = 0, gc = 0, dc = 0, hv2 = 0, pr = 0;
       if (c.kind != JVal::Obj || !num_field(c, "M", &M) || !num_field(c, "pipeline", &pl))
         return UW_ERR_FORMAT;
       num_field(c, "tile_n", &tn);
@@ -375,6 +382,7 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
       num_field(c, "gemm_ctas", &gc);
       num_field(c, "decode_ctas", &dc);
       num_field(c, "halves", &hv2);
+      num_field(c, "pair", &pr);
       uw_gemm_config cfg;
       std::memset(&cfg, 0, sizeof(cfg));
       cfg.pipeline = (int32_t)pl;
@@ -383,6 +391,7 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
       cfg.gemm_ctas = (int32_t)gc;
       cfg.decode_ctas = (int32_t)dc;
       cfg.halves = (int32_t)hv2;
+      cfg.pair = (int32_t)pr;
       if (M <= 0 || check_config(hs[i], cfg) != UW_OK) return UW_ERR_FORMAT;
       parsed[i][M] = cfg;
     }

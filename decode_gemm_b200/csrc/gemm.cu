@@ -215,7 +215,7 @@ __device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t tag, vo
 
 // KS_: K blocks per unit (compile time, so the per-block loops unroll); it
 // equals p.ks.
-template <int MODE, int KS_>
+template <int MODE, int KS_, bool PAIR = false>
 __global__ void __launch_bounds__(threads_for(MODE), 1)
     gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -232,11 +232,22 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   const int H = p.halves;
   const bool wide = H == 2;
   const int RU = kBM * H;  // W rows per unit
+  // CTA pairs (two-SM MMA): the CTA's rank in its pair; the rank-0 CTA
+  // issues the MMAs
+  const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
+  const bool lead = crank == 0;
+  // first W row of this CTA in row tile nt (a pair's tile has 256 rows, rank r
+  // holds rows 128 r ..)
+  auto row0_of = [&](int64_t nt) -> int64_t {
+    return PAIR ? nt * (2 * kBM) + (int64_t)crank * kBM : nt * RU;
+  };
   const int SX = p.xstages;
   const uint32_t xst_bytes = (uint32_t)KS_ * p.x_bytes;  // one unit's X tiles
   uint8_t* ring = smem;
   uint8_t* xring = ring + (size_t)S * L.bytes;       // X tiles
-  uint8_t* wring = xring + (size_t)SX * xst_bytes;  // rebuilt W tiles (shared-memory path)
+  // rebuilt W tiles (shared-memory path); a pair keeps a spare X tile's room
+  // after its X ring, so no operand read of the MMA can pass the block's end
+  uint8_t* wring = xring + (size_t)SX * xst_bytes + (PAIR ? xst_bytes : 0);
   uint8_t* ystage = wring + (size_t)(p.tmem_w ? 0 : WS) * kWTileBytes;  // 2 x [16][128] BF16
   uint8_t* tail = ystage + (p.y_tma ? 2 * kYBlockBytes : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
@@ -268,16 +279,21 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(b_tfull + a), (uint32_t)NM);
-      mbar_init(bar(b_tempty + a), kNumEpiWarps);
+      mbar_init(bar(b_tempty + a), PAIR ? 2 * kNumEpiWarps : kNumEpiWarps);
       mbar_init(bar(b_drain + a), 1);
     }
     mbar_init(bar(b_part), 1);
     *abort = 0;
     fence_mbar_init();
   }
-  const int64_t G = gridDim.x;
-  const int64_t u0 = unit_begin(blockIdx.x, p.units, G);
-  const int64_t u1 = unit_begin(blockIdx.x + 1, p.units, G);
+  // CTA pairs: both CTAs of a pair take the pair's units; partitions, their
+  // count and owners are per pair, while partial sums and ready flags stay
+  // per CTA (slot 2 pid + rank)
+  const int64_t G = PAIR ? gridDim.x / 2 : gridDim.x;
+  const int64_t pid = PAIR ? blockIdx.x / 2 : blockIdx.x;
+  auto slot_of = [&](int64_t q) { return PAIR ? 2 * q + crank : q; };
+  const int64_t u0 = unit_begin(pid, p.units, G);
+  const int64_t u1 = unit_begin(pid + 1, p.units, G);
   const int KB = p.KB;    // units along K
   constexpr int KS = KS_;  // K blocks per unit
   const int NP = H * KS;  // escape parts per stage: (half, K block) pairs, at most 2
@@ -314,11 +330,18 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     if (MODE != kGemmBf16) prefetch_tensormap(&p.tm_w1);
   }
   if (warp == kMmaWarp0) {
-    tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // a pair's barriers are all initialised before either CTA signals the other's
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // set-up above touched only the handle's immutable arrays; from here on X,
@@ -357,7 +380,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
       const int64_t nt = t / p.MT;
-      const int32_t n0 = (int32_t)(nt * RU);
+      const int32_t n0 = (int32_t)row0_of(nt);
       for (int kb = kb0; kb < kb1; ++kb, ++qi) {
         uint32_t c0[2] = {0u, 0u}, c1[2] = {0u, 0u};
         if (MODE == kGemmPalette) {
@@ -407,9 +430,15 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
                 }
               }
             }
-            mbar_expect_tx(fb, bytes);
             const int kbk = kb * KS;  // first K block of the unit
-            tma_load_2d(smem_u32(st + L.w0), &p.tm_w0, fb, kbk * kBK, n0);
+            if constexpr (PAIR) {
+              // both CTAs' tiles count on the leader's barrier, which expects both
+              if (lead) mbar_expect_tx(fb, 2 * bytes);
+              tma_load_2d_pair(smem_u32(st + L.w0), &p.tm_w0, mapa_shared(fb, 0), kbk * kBK, n0);
+            } else {
+              mbar_expect_tx(fb, bytes);
+              tma_load_2d(smem_u32(st + L.w0), &p.tm_w0, fb, kbk * kBK, n0);
+            }
             if (MODE == kGemmExp) tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kbk * kBK, n0);
             if (MODE == kGemmPalette) {
               tma_load_2d(smem_u32(st + L.w1), &p.tm_w1, fb, kbk * (kBK / 2), n0);
@@ -433,8 +462,10 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       }
       u += kb1 - kb0;
     }
-    // in-flight copies must land before the CTA exits
-    if (lane == 0 && *abort) {
+    // in-flight copies must land before the CTA exits (a pair's copies count
+    // on the leader's barriers: the leader drains them, and the pair leaves
+    // together)
+    if (lane == 0 && *abort && (!PAIR || lead)) {
       const int64_t outstanding = issued < S ? issued : S;
       int s = stage;
       uint32_t ph = phase;
@@ -459,8 +490,15 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     // par of every unit (W slots go in pairs, slot 2 j + par for pair j) into
     // its own columns.
     const int par = warp - kMmaWarp0;
-    if (par < NM) {
-      const uint32_t idesc = idesc_bf16(kBM, p.tile_n);
+    // (a pair's MMAs are the rank-0 CTA's: they fill both CTAs' TMEM)
+    if (par < NM && (!PAIR || lead)) {
+      const uint32_t idesc = idesc_bf16(PAIR ? 2 * kBM : kBM, p.tile_n);
+      auto commit = [&](uint32_t b) {
+        if constexpr (PAIR)
+          mma_commit_pair(b, 0x3);  // the barrier at this offset in both CTAs
+        else
+          mma_commit(b);
+      };
       const int WP = wide ? WS / 2 : WS;  // W slot positions this warp cycles through
       // ring positions of the current unit, advanced for every unit of the CTA
       int stage = 0, wpos = 0, xs = 0;
@@ -521,13 +559,18 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
                                       : smem_u32(wring + (size_t)wslot * kWTileBytes);
                 const uint64_t a_desc = smem_desc_sw128(a_addr);
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                  mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
-                           (!first || k > 0) ? 1u : 0u);
+                for (int k = 0; k < kBK / 16; ++k) {
+                  if constexpr (PAIR)
+                    mma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
+                                  (!first || k > 0) ? 1u : 0u);
+                  else
+                    mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
+                             (!first || k > 0) ? 1u : 0u);
+                }
               }
-              if (MODE == kGemmBf16) mma_commit(bar(b_empty + stage));
-              mma_commit(bar(b_xempty + xs));
-              if (MODE != kGemmBf16) mma_commit(bar(b_wfree + wslot));
+              if (MODE == kGemmBf16) commit(bar(b_empty + stage));
+              commit(bar(b_xempty + xs));
+              if (MODE != kGemmBf16) commit(bar(b_wfree + wslot));
             }
           }
           if (mine) first = false;
@@ -547,12 +590,12 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           }
         }
         // the segment's accumulator is complete once this warp's MMAs finish
-        if (ok && lane == 0) mma_commit(bar(b_tfull + acc));
+        if (ok && lane == 0) commit(bar(b_tfull + acc));
         u += kb1 - kb0;
       }
       // every issued MMA completes before TMEM is released
       if (lane == 0) {
-        mma_commit(bar(b_drain + par));
+        commit(bar(b_drain + par));
         volatile int no_abort = 0;
         mbar_wait_bounded(bar(b_drain + par), 0, &no_abort, p.wait_ns);
       }
@@ -584,8 +627,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       if (!got) set_abort(abort, p.status);
       if (epi_any(!got)) break;
       tc_fence_after();
-      // a split tile's owner (the CTA with its first K block) collects the
-      // partial sums of CTAs blockIdx.x+1 .. last
+      // a split tile's owner (the CTA, or pair, with its first K block)
+      // collects the partial sums of partitions pid+1 .. last
       const int64_t nt = t / p.MT, mt = t - nt * p.MT;
       const int64_t m0 = mt * p.tile_n;
       const int cols = (int)imin64(p.tile_n, p.M - m0);
@@ -593,7 +636,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       int64_t last = 0;
       if (split) {
         const int64_t ua = t * KB;
-        owner = unit_owner(ua, p.units, G) == (int64_t)blockIdx.x;
+        owner = unit_owner(ua, p.units, G) == pid;
         last = unit_owner(ua + KB - 1, p.units, G);
         if (owner) {
           // The owner's split segment is its CTA's last (the CTA's range ends
@@ -602,18 +645,19 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           // of one L2 round trip per 16 columns.  Measured on 14336x4096 and
           // 4096x14336: a gain for 32..64 columns; for 16 or fewer the copy
           // moves mostly unused columns, for 128..256 its latency does not pay.
-          const int64_t sbytes = (last - (int64_t)blockIdx.x) * part_stride * 4;
-          staged = cols >= 32 && cols <= 64 && sbytes <= (int64_t)S * L.bytes;
+          const int64_t sbytes = (last - pid) * part_stride * 4;
+          // (a pair's contributors' slots are not adjacent)
+          staged = !PAIR && cols >= 32 && cols <= 64 && sbytes <= (int64_t)S * L.bytes;
           bool ok = true;
           if (leader) {
-            for (int64_t q = blockIdx.x + 1; q <= last && ok; ++q)
-              ok = wait_flag(p.sync + 2 + q, tag, abort, p.wait_ns);
+            for (int64_t q = pid + 1; q <= last && ok; ++q)
+              ok = wait_flag(p.sync + 2 + slot_of(q), tag, abort, p.wait_ns);
             if (!ok) {
               set_abort(abort, p.status);
             } else if (staged) {
               fence_proxy_async_global();
               mbar_expect_tx(bar(b_part), (uint32_t)sbytes);
-              bulk_load(smem_u32(ring), p.partials + (int64_t)(blockIdx.x + 1) * part_stride,
+              bulk_load(smem_u32(ring), p.partials + (pid + 1) * part_stride,
                         (uint32_t)sbytes, bar(b_part));
             }
           }
@@ -635,13 +679,13 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
         const uint32_t t0 =
             tmem_base + lanebase + (uint32_t)((acc * NM + (wide ? h : 0)) * p.tile_n);
         const uint32_t t1 = tmem_base + lanebase + (uint32_t)((acc * NM + 1) * p.tile_n);
-        const int64_t n = nt * RU + h * kBM + row;
+        const int64_t n = row0_of(nt) + h * kBM + row;
         const int64_t hoff = (int64_t)h * kBM * p.tile_n;  // the half's place in a partial tile
-        float* part = p.partials + (int64_t)blockIdx.x * part_stride + hoff;
+        float* part = p.partials + slot_of(pid) * part_stride + hoff;
         // an owner reads the first contributor's sums one column block ahead,
         // so their latency overlaps the TMEM reads and the stores
         const bool gather = split && owner;
-        const float* part1 = p.partials + (int64_t)(blockIdx.x + 1) * part_stride + hoff + row;
+        const float* part1 = p.partials + slot_of(pid + 1) * part_stride + hoff + row;
         float pn[16];
         if (gather && !staged) {
 #pragma unroll
@@ -667,7 +711,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           if (gather && staged) {
             // the other CTAs' sums, in K order, from the staged copies
             const float* sp = reinterpret_cast<const float*>(ring) + hoff + (int64_t)c * kBM + row;
-            for (int64_t q = 0; q < last - (int64_t)blockIdx.x; ++q) {
+            for (int64_t q = 0; q < last - pid; ++q) {
 #pragma unroll
               for (int j = 0; j < 16; ++j)
                 if (c + j < cols) v[j] += sp[q * part_stride + j * kBM];
@@ -682,8 +726,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
               for (int j = 0; j < 16; ++j)
                 pn[j] = c + 16 + j < cols ? __ldcg(part1 + (int64_t)(c + 16 + j) * kBM) : 0.f;
             }
-            for (int64_t q = blockIdx.x + 2; q <= last; ++q) {
-              const float* src = p.partials + q * part_stride + hoff + (int64_t)c * kBM + row;
+            for (int64_t q = pid + 2; q <= last; ++q) {
+              const float* src = p.partials + slot_of(q) * part_stride + hoff + (int64_t)c * kBM + row;
               float pv[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j) pv[j] = c + j < cols ? __ldcg(src + j * kBM) : 0.f;
@@ -703,8 +747,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             for (int j = 0; j < 16; ++j) yb[j * kBM + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
             fence_proxy_async_smem();
             epi_sync();
-            if (leader && nt * RU + h * kBM < p.N) {  // (a box wholly past N writes nothing)
-              tma_store_2d(&p.tm_y, smem_u32(yb), (int32_t)(nt * RU + h * kBM), (int32_t)(m0 + c));
+            if (leader && row0_of(nt) + h * kBM < p.N) {  // (a box wholly past N writes nothing)
+              tma_store_2d(&p.tm_y, smem_u32(yb), (int32_t)(row0_of(nt) + h * kBM), (int32_t)(m0 + c));
               bulk_commit();
             }
             ++yblk;
@@ -725,11 +769,16 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       if (split && !owner) {  // hand the partial sum over
         __threadfence();
         epi_sync();
-        if (leader) st_release(p.sync + 2 + blockIdx.x, tag);
+        if (leader) st_release(p.sync + 2 + slot_of(pid), tag);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(b_tempty + acc));
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(mapa_shared(bar(b_tempty + acc), 0));  // the leader's barrier
+        else
+          mbar_arrive(bar(b_tempty + acc));
+      }
       u += kb1 - kb0;
       qa += kb1 - kb0;
     }
@@ -748,7 +797,10 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const int64_t t = u / KB;
       const int kb0 = (int)(u - t * KB);
       const int kb1 = (int)imin64(KB, kb0 + (u1 - u));
-      const int32_t m0 = (int32_t)((t - (t / p.MT) * p.MT) * p.tile_n);
+      // (a pair's CTA loads its half of the token tile: rank r tokens
+      // tile_n / 2 * r ..)
+      const int32_t m0 = (int32_t)((t - (t / p.MT) * p.MT) * p.tile_n +
+                                   (PAIR ? (int64_t)crank * (p.tile_n / 2) : 0));
       for (int kb = kb0; kb < kb1; ++kb) {
         if (lane == 0) {
           if (!mbar_wait_bounded(bar(b_xempty + xs), xph ^ 1u, abort, p.wait_ns)) {
@@ -757,10 +809,18 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
           } else {
             const uint32_t fb = bar(b_xfull + xs);
             uint8_t* xt = xring + (size_t)xs * xst_bytes;
-            mbar_expect_tx(fb, xst_bytes);
+            if constexpr (PAIR) {
+              if (lead) mbar_expect_tx(fb, 2 * xst_bytes);
+              const uint32_t fbl = mapa_shared(fb, 0);
 #pragma unroll
-            for (int j = 0; j < KS; ++j)
-              tma_load_2d(smem_u32(xt + j * p.x_bytes), &p.tm_x, fb, (kb * KS + j) * kBK, m0);
+              for (int j = 0; j < KS; ++j)
+                tma_load_2d_pair(smem_u32(xt + j * p.x_bytes), &p.tm_x, fbl, (kb * KS + j) * kBK, m0);
+            } else {
+              mbar_expect_tx(fb, xst_bytes);
+#pragma unroll
+              for (int j = 0; j < KS; ++j)
+                tma_load_2d(smem_u32(xt + j * p.x_bytes), &p.tm_x, fb, (kb * KS + j) * kBK, m0);
+            }
             ++issued;
           }
         }
@@ -773,8 +833,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       }
       u += kb1 - kb0;
     }
-    // in-flight copies must land before the CTA exits
-    if (lane == 0 && *abort) {
+    // in-flight copies must land before the CTA exits (a pair's: see the
+    // weight producer)
+    if (lane == 0 && *abort && (!PAIR || lead)) {
       const int64_t outstanding = issued < SX ? issued : SX;
       int s = xs;
       uint32_t ph = xph;
@@ -1032,9 +1093,14 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair leaves together: the peer's MMAs read this CTA's shared memory
+  if constexpr (PAIR) cluster_sync();
   if (warp == kMmaWarp0) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, (uint32_t)p.tmem_cols);
+    else
+      tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
   }
   // the last CTA to leave advances the epoch for the next launch
   if (threadIdx.x == 0) {
@@ -1116,21 +1182,22 @@ int tmem_ks_for(const GemmArgs& a) {
 }
 
 size_t smem_bytes(int mode, int tile_n, int stages, int wslots, int halves, bool tmem_w, int ks,
-                  int xstages, bool y_tma) {
+                  int xstages, bool y_tma, bool pair) {
   const StageLayout L = stage_layout(mode, tile_n, halves, ks);
   const int ws = mode == kGemmBf16 ? 0 : wslots;  // W slots (their barriers exist either way)
   size_t b = 1024 /* alignment slack */ + (size_t)stages * L.bytes;
-  b += (size_t)xstages * ks * tile_n * kBK * 2;     // X ring
+  b += (size_t)(xstages + (pair ? 1 : 0)) * ks * (pair ? tile_n / 2 : tile_n) * kBK * 2;  // X ring
+                                                     // (a pair: half tiles and a spare)
   if (!tmem_w) b += (size_t)ws * kWTileBytes;       // (TMEM path: the slots live in TMEM)
   if (y_tma) b += 2 * kYBlockBytes;                 // Y staging
   b += (size_t)(2 * stages + 2 * xstages + 2 * ws + 7) * 8 + 16;
   return b;
 }
 
-template <int MODE, int KS>
+template <int MODE, int KS, bool PAIR = false>
 cudaError_t set_smem_attr() {
   static cudaError_t e = cudaFuncSetAttribute(
-      gemm_kernel<MODE, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+      gemm_kernel<MODE, KS, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
   return e;
 }
 
@@ -1163,6 +1230,14 @@ bool gemm_resolve(GemmArgs* a) {
       a->tile_n = 256;
   }
   if (a->tile_n < 16 || a->tile_n > 256 || a->tile_n % 16) return false;
+  // CTA pairs (BF16, one half per unit): one MMA of 256 W rows x 256 tokens
+  // over an SM pair, each CTA loading its 128 W rows and half of the tokens
+  {
+    const bool want = a->pair > 0;  // (on request only)
+    if (want && (a->mode != kGemmBf16 || wide)) return false;
+    a->pair = want ? 1 : 0;
+    if (a->pair) a->tile_n = 256;
+  }
   // One half per unit: ring depths are even, consumers alternate units, so an
   // even depth keeps every slot with one consumer (see the MMA issuers).  Wide:
   // every consumer takes every stage, any depth works; W slots go in pairs.
@@ -1190,8 +1265,10 @@ bool gemm_resolve(GemmArgs* a) {
   // take units as fast as they land (32 KB starved it at M = 256); 2..8
   // units, an even number when two MMA warps alternate units
   {
-    const int xunit = a->ks * a->tile_n * kBK * 2;
-    const int x_target = a->mode == kGemmBf16 ? (a->tile_n > 128 ? 131072 : 98304)
+    const int xunit = a->ks * (a->pair ? a->tile_n / 2 : a->tile_n) * kBK * 2;
+    // (a pair's CTA: 64 KB, so the W ring keeps 8 stages)
+    const int x_target = a->pair ? 65536
+                         : a->mode == kGemmBf16 ? (a->tile_n > 128 ? 131072 : 98304)
                                               : (a->tile_n > 128 ? 98304 : 49152);
     int sx = x_target / xunit;
     sx = sx < 2 ? 2 : (sx > 8 ? 8 : sx);
@@ -1202,9 +1279,9 @@ bool gemm_resolve(GemmArgs* a) {
     const int wslots0 = a->wslots;
     for (;;) {
       int s = max_stages;
-      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma) > (size_t)kSmemLimit)
+      while (s > 2 && smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma, a->pair != 0) > (size_t)kSmemLimit)
         s -= step;
-      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma) <= (size_t)kSmemLimit ||
+      if (smem_bytes(a->mode, a->tile_n, s, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma, a->pair != 0) <= (size_t)kSmemLimit ||
           a->wslots <= 2 || wide) {
         a->stages = s;
         if (a->y_tma && s < 4) {  // the staging would cost too much of the load ring
@@ -1218,15 +1295,21 @@ bool gemm_resolve(GemmArgs* a) {
     }
   }
   if (a->stages < 2 || (!wide && (a->stages & 1)) ||
-      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma) > (size_t)kSmemLimit)
+      smem_bytes(a->mode, a->tile_n, a->stages, a->wslots, a->halves, a->tmem_w, a->ks, a->xstages, a->y_tma, a->pair != 0) > (size_t)kSmemLimit)
     return false;
-  const int64_t RU = (int64_t)kBM * a->halves;
+  const int64_t RU = (int64_t)kBM * (a->pair ? 2 : a->halves);
   const int64_t NT = (a->N + RU - 1) / RU;
   const int64_t MT = (a->M + a->tile_n - 1) / a->tile_n;
   const int64_t units = NT * MT * (a->K / kBK / a->ks);
   int ctas = a->ctas > 0 ? a->ctas : a->sm_count;
-  if ((int64_t)ctas > units) ctas = (int)units;
   if (ctas > kGemmMaxCtas) ctas = kGemmMaxCtas;
+  if (a->pair) {  // whole pairs, at most one per unit
+    const int64_t pairs = imin64(ctas / 2, units);
+    if (pairs < 1) return false;
+    ctas = (int)(2 * pairs);
+  } else if ((int64_t)ctas > units) {
+    ctas = (int)units;
+  }
   a->ctas = ctas;
   return true;
 }
@@ -1247,8 +1330,12 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   const uint32_t RU = (uint32_t)kBM * (wide ? 2 : 1);
   const bool tw = a.tmem_w != 0;
   if (KS > 1 && (!tw || a.mode == kGemmBf16)) return cudaErrorInvalidValue;
+  const bool pair = a.pair != 0;
+  if (pair && (a.mode != kGemmBf16 || wide || KS != 1 || a.tile_n % 32)) return cudaErrorInvalidValue;
+  // (a pair's CTA loads half of the token tile)
   if (!make_map_2d(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.K,
-                   (uint64_t)a.M, kBK, (uint32_t)a.tile_n, CU_TENSOR_MAP_SWIZZLE_128B))
+                   (uint64_t)a.M, kBK, (uint32_t)(pair ? a.tile_n / 2 : a.tile_n),
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   bool ok = true;
   if (a.mode == kGemmBf16) {
@@ -1299,7 +1386,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   if (p.xstages < 2 || (!wide && mma_warps_for(a.tile_n) == 2 && (p.xstages & 1)))
     return cudaErrorInvalidValue;  // unresolved
   p.wslots = a.wslots;
-  p.NT = (int32_t)((a.N + RU - 1) / RU);
+  p.NT = (int32_t)((a.N + (pair ? 2 * kBM : RU) - 1) / (pair ? 2 * kBM : RU));
   p.NG = (int32_t)((a.N + kBM - 1) / kBM);
   p.halves = wide ? 2 : 1;
   p.MT = (int32_t)((a.M + a.tile_n - 1) / a.tile_n);
@@ -1321,11 +1408,12 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   for (int i = 1; i < 16; ++i)
     if (a.palette[i] != a.palette[0] + i) p.pal_run = 0;
   p.pal_bias = (uint32_t)a.palette[0] * 128u * 65537u;
-  p.x_bytes = (uint32_t)a.tile_n * kBK * 2;
+  p.x_bytes = (uint32_t)(pair ? a.tile_n / 2 : a.tile_n) * kBK * 2;
   p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves, KS).bytes;
   p.wait_ns = wait_limit_ns();
   const size_t smem =
-      smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS, a.xstages, a.y_tma != 0);
+      smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS, a.xstages, a.y_tma != 0,
+                 a.pair != 0);
   const int G = a.ctas;
   cudaError_t e = cudaSuccess;
   auto begin = [&](int kind) { return hooks && hooks->begin ? hooks->begin(hooks->ctx, kind) : -1; };
@@ -1336,8 +1424,35 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   const int slot = begin(3 + a.mode);
   switch (a.mode) {
     case kGemmBf16:
-      if ((e = set_smem_attr<kGemmBf16, 1>()) != cudaSuccess) return e;
-      e = launch_pdl(gemm_kernel<kGemmBf16, 1>, G, threads_for(kGemmBf16), smem, s, p);
+      if (pair) {
+        if ((e = set_smem_attr<kGemmBf16, 1, true>()) != cudaSuccess) return e;
+        // every pair must be resident at once (owners wait for later pairs'
+        // partial sums): at most as many pairs as the GPU holds
+        int G2 = G;
+        {
+          cudaLaunchConfig_t q = {};
+          q.gridDim = dim3(G2);
+          q.blockDim = dim3(threads_for(kGemmBf16));
+          q.dynamicSmemBytes = smem;
+          cudaLaunchAttribute ca[1];
+          ca[0].id = cudaLaunchAttributeClusterDimension;
+          ca[0].val.clusterDim.x = 2;
+          ca[0].val.clusterDim.y = 1;
+          ca[0].val.clusterDim.z = 1;
+          q.attrs = ca;
+          q.numAttrs = 1;
+          int clusters = 0;
+          if ((e = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<kGemmBf16, 1, true>, &q)) !=
+              cudaSuccess)
+            return e;
+          if (clusters < 1) return cudaErrorInvalidConfiguration;
+          if (G2 > 2 * clusters) G2 = 2 * clusters;
+        }
+        e = launch_pdl_pair(gemm_kernel<kGemmBf16, 1, true>, G2, threads_for(kGemmBf16), smem, s, p);
+      } else {
+        if ((e = set_smem_attr<kGemmBf16, 1>()) != cudaSuccess) return e;
+        e = launch_pdl(gemm_kernel<kGemmBf16, 1>, G, threads_for(kGemmBf16), smem, s, p);
+      }
       break;
     case kGemmExp:
       if (KS == 2) {

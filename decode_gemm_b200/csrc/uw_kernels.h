@@ -89,6 +89,8 @@ struct GemmArgs {
   int xstages = 0;               // resolved: X ring depth
   int y_tma = 0;                 // resolved: BF16 Y through TMA stores
   int tmem_w = 0;                // resolved: W rebuilt into TMEM (else shared memory)
+  int pair = 0;                  // CTA pairs with two-SM MMAs: 1 on, -1 off, 0 automatic;
+                                 // resolved to 1 or 0
   int ctas = 0;                  // persistent CTAs (0 = SM count)
   int sm_count = 148;
   uint32_t* status = nullptr;

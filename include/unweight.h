@@ -147,7 +147,12 @@ typedef struct uw_gemm_config {
   int32_t decode_ctas;   /* SMs (one CTA each) of the preprocessing kernel (0 = all) */
   int32_t halves;        /* W rows per GEMM unit / 128: 1, or 2 (the wide shape: X
                             is read once per 256 rows); 0 = 1                       */
-  int32_t reserved[2];
+  int32_t pair;          /* 1: the BF16 GEMM (pipeline 1) on CTA pairs: one two-SM
+                            MMA of 256 W rows x 256 tokens per step over an SM pair,
+                            each CTA loading its 128 rows and half of the tokens
+                            (256-token tiles; one half per unit); 0: one CTA per
+                            tile.  Other pipelines: UW_ERR_UNSUPPORTED              */
+  int32_t reserved;
 } uw_gemm_config;
 
 typedef struct uw_host_s* uw_host_t;       /* host-side encoded matrix         */

@@ -306,6 +306,47 @@ def test_wide_units_match_fp64(uw, M, N, K, kind, pipe, tile_n):
     h.free()
 
 
+PAIR_SHAPES = [
+    # (M, N, K, weight maker): the BF16 GEMM on CTA pairs (256 W rows x 256
+    # tokens per two-SM MMA step; each CTA holds 128 rows and half the tokens)
+    (256, 512, 512, "normal"),
+    (300, 640, 384, "student_t"),   # ragged M: the second tile's tokens mostly past M
+    (40, 200, 192, "special_finite"),  # M < 128: rank 1's token half entirely past M; N < 256
+    (513, 384, 1024, "normal"),     # three token tiles, N not a multiple of 256
+]
+
+
+@pytest.mark.parametrize("M,N,K,kind", PAIR_SHAPES)
+@pytest.mark.parametrize("out_f32", [True, False])
+def test_pair_bf16_matches_fp64(uw, M, N, K, kind, out_f32):
+    """Pipeline 1 with the two-SM MMA on CTA pairs, against the FP64 oracle; with
+    few pairs the tiles' K ranges split between pairs (partial sums per CTA)."""
+    w = _weights(kind, N, K, seed=90 + M)
+    x = synthdata.activations(M, K, seed=91 + N)
+    h = _upload(uw, w, chunk=128)
+    ws = _workspace(uw, h, M)
+    for ctas in (0, 6):  # one CTA per SM, or three pairs
+        y = _gemm(uw, h, x, "full", out_f32=out_f32, pair=1, gemm_ctas=ctas)
+        _check(y, x, w, bf16_out=not out_f32)
+    h.free()
+
+
+def test_pair_config_checked(uw):
+    """CTA pairs are a BF16-GEMM variant: other pipelines and values are refused."""
+    import ctypes as C
+    import torch
+    w = synthdata.normal(256, 256, 0.02, seed=103)
+    h = uw.uw_encode(w)
+    X = torch.zeros((256, 256), dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros((256, 256), dtype=torch.bfloat16, device="cuda")
+    for pipe, pair, halves, want in ((4, 1, 0, uw.UW_ERR_UNSUPPORTED), (2, 1, 0, uw.UW_ERR_UNSUPPORTED),
+                                     (1, 2, 0, uw.UW_ERR_ARG), (1, 1, 2, uw.UW_ERR_ARG)):
+        cfg = uw.gemm_config(pipe, pair=pair, halves=halves)
+        assert uw.lib.uw_gemm_ex(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 256,
+                                 C.byref(cfg), 0) == want
+    h.free()
+
+
 PALETTE_CASES = [
     ("lookup", list(range(100, 132, 2)), 0),   # 16 exponents, not a run: palette lookup
     ("run_base0", list(range(0, 16)), 0),      # the run 0..15 (zero and subnormal weights)
