@@ -313,9 +313,19 @@ def _load_build():
     return mod
 
 
-def _kernel_src_sha():
+# The sources each kernel is built from (a capture's counters stay valid while
+# they are unchanged).
+KERNEL_SOURCES = {
+    "decode": ("decode.cu", "bf16_fields.cuh", "pdl.cuh"),
+    "gemm": ("gemm.cu", "gemm_sm100.cuh", "bf16_fields.cuh", "pdl.cuh"),
+}
+
+
+def _kernel_src_sha(kind=None):
+    """Digest of the sources of one kernel family ("decode" or "gemm"), or of both."""
+    files = KERNEL_SOURCES[kind] if kind else sorted(set(sum(KERNEL_SOURCES.values(), ())))
     h = hashlib.sha256()
-    for f in ("decode.cu", "gemm.cu", "gemm_sm100.cuh", "bf16_fields.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "decode_gemm_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -462,7 +472,8 @@ def run_ours(args):
                   f"{N_SETS} weight sets rotated)")
     achieved = blk_bytes / (blk_ms * 1e-3) / 1e9
     traffic = TRAFFIC.get(dominant)
-    if traffic and traffic.get("src_sha") != _kernel_src_sha():
+    if traffic and traffic.get("src_sha") != _kernel_src_sha(
+            "decode" if dominant.startswith("decode") or dominant == "transcode" else "gemm"):
         traffic = None
     roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
