@@ -59,9 +59,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum; profiles/*.md), valid only while the kernel source
 # (src_sha, see _kernel_src_sha) is unchanged.
 TRAFFIC = {
-    "gemm_palette": {"bytes_per_launch": 89.727744e6 + 4.889088e6, "src_sha": "130db6751de935ad",
+    "gemm_palette": {"bytes_per_launch": 89.686016e6 + 3.780352e6, "src_sha": "c8fceb82ccca36fe",
                      "capture": "profiles/gemm_palette_gate_14336x4096_M1.md (M = 1 launch)"},
-    "decode_full": {"bytes_per_launch": 87.153920e6 + 66.200064e6, "src_sha": "130db6751de935ad",
+    "decode_full": {"bytes_per_launch": 87.243776e6 + 66.097408e6, "src_sha": "3ad9520e689dbfbd",
                     "capture": "profiles/decode_full_gate_14336x4096.md (output partly still in L2)"},
 }
 
