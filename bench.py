@@ -275,6 +275,24 @@ def cpu_oracle_sample(rows=4, ms=MS, target_s=None):
     return alg / dt / 1e9, dt, desc
 
 
+def max_over_ranks(x, world, device="cuda"):
+    """The largest of every rank's x (each rank's device time of the same timed
+    steps): the job's time is its slowest replica's."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(bytes_per_rank, max_ms, world):
+    """Whole-job throughput in GB/s: every replica processes bytes_per_rank in
+    the timed region, which lasts max_ms (the slowest rank's time)."""
+    return bytes_per_rank * world / (max_ms * 1e-3) / 1e9
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -414,12 +432,9 @@ def run_ours(args):
         st = uw.uw_last_device_status(h)
         if st != uw.UW_OK:
             raise RuntimeError(f"device status {uw.uw_status_str(st)}")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
     ms_per_step = elapsed_ms / args.steps
-    value = total_bytes / (elapsed_ms * 1e-3) / 1e9 * world
+    value = job_rate(total_bytes, elapsed_ms, world)
 
     # ---- traced pass: per-kernel attribution (runs rotate over handles)
     for h in handles:
@@ -541,12 +556,8 @@ def run_ours(args):
             Yh[k].copy_(Y[k], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = e2e_bytes / (e2e_ms * 1e-3) / 1e9 * world
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = job_rate(e2e_bytes, e2e_ms, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
