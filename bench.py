@@ -38,6 +38,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -59,9 +60,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum; profiles/*.md), valid only while the kernel source
 # (src_sha, see _kernel_src_sha) is unchanged.
 TRAFFIC = {
-    "gemm_palette": {"bytes_per_launch": 89.686016e6 + 3.780352e6, "src_sha": "c8fceb82ccca36fe",
+    "gemm_palette": {"bytes_per_launch": 89.686016e6 + 3.780352e6, "src_sha": "86199055be906a41",
                      "capture": "profiles/gemm_palette_gate_14336x4096_M1.md (M = 1 launch)"},
-    "decode_full": {"bytes_per_launch": 87.243776e6 + 66.097408e6, "src_sha": "3ad9520e689dbfbd",
+    "decode_full": {"bytes_per_launch": 87.243776e6 + 66.097408e6, "src_sha": "ee0a4d48dea442f1",
                     "capture": "profiles/decode_full_gate_14336x4096.md (output partly still in L2)"},
 }
 
@@ -339,13 +340,21 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """C++ source without comments and blank space: what the compiler sees."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def _kernel_src_sha(kind=None):
-    """Digest of the sources of one kernel family ("decode" or "gemm"), or of both."""
+    """Digest of the code (comments and layout aside) of one kernel family's
+    sources ("decode" or "gemm"), or of both."""
     files = KERNEL_SOURCES[kind] if kind else sorted(set(sum(KERNEL_SOURCES.values(), ())))
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "decode_gemm_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "decode_gemm_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,13 +14,19 @@
 //   * tcgen05.mma (kind::f16, BF16 x BF16 -> FP32) issued by one thread,
 //     accumulating in TMEM; two accumulators so the epilogue of one output
 //     tile overlaps the main loop of the next.
-//   * Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner),
-//     warps 2-5 epilogue (TMEM -> registers -> global), warps 6-13 rebuild
-//     (reconstructive modes only).
-//   * Rebuild: 8 weights per 16-byte store into the 128-byte-swizzled K-major
-//     layout the MMA descriptor expects; palette lookup is three byte permutes
-//     per 4 weights; the escape decision is taken once per 64-weight row from a
-//     16-byte bitmap staged with the tile.
+//   * Warp roles: warp 0 weight producer (TMA), warps 1-2 MMA issuers (units
+//     alternate between them by parity, each with its own accumulators; warp
+//     1 owns TMEM), warps 3-6 epilogue (TMEM -> registers -> global), warps
+//     7-14 rebuild in two groups of 4 taking alternate units (reconstructive
+//     modes only), and the last warp the X producer (X tiles on a ring of
+//     their own, so the weight ring's depth goes to HBM traffic).
+//   * Rebuild: for token tiles up to 96, each thread rebuilds one W row of
+//     the unit's K blocks and writes it to TMEM (tcgen05.st); the MMA reads A
+//     from TMEM.  Larger tiles rebuild into the 128-byte-swizzled K-major
+//     shared layout the MMA descriptor expects.  A palette that is one run
+//     of exponents rebuilds with a multiply-add per BF16 pair, any other with
+//     byte-permute lookups; the escape decision is taken once per 64-weight
+//     row from a 16-byte bitmap staged with the tile.
 //   * Persistent CTAs split the flattened (output tile, K block) space evenly
 //     (stream-K).  A tile shared by several CTAs is finished inside the kernel
 //     by the CTA holding its first K block: that tile is the last it works on,
@@ -29,10 +35,13 @@
 //     epoch); it adds them in K order, so results are deterministic.  The
 //     epoch lives on the device (the last CTA to exit advances it), so stale
 //     flags from earlier launches, aborted ones or graph replays never match.
+//   * CTA pairs (BF16 mode, on request): two-SM MMAs of 256 W rows over a
+//     cluster of two CTAs, the same stream-K split per pair.
 //   * Every mbarrier wait is bounded in wall time; on expiry the kernel records
 //     a timeout in the status word, drains its MMAs and copies, frees TMEM and
 //     returns.
-//   * No cluster multicast anywhere.
+//   * No TMA load with cluster multicast anywhere (CTA pairs load their own
+//     halves; only MMA commits arrive on both CTAs' barriers).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
