@@ -180,6 +180,8 @@ class HostEncoded:
 
     def __init__(self, ptr):
         self._ptr = _vp(ptr)
+        # (module globals may be gone when __del__ runs at interpreter exit)
+        self._free, self._null = lib.uw_host_free, _vp(0)
 
     @property
     def ptr(self):
@@ -199,9 +201,10 @@ class HostEncoded:
         return s.as_dict()
 
     def __del__(self):
-        if getattr(self, "_ptr", None) and self._ptr.value:
-            lib.uw_host_free(self._ptr)
-            self._ptr = _vp(0)
+        ptr, free = getattr(self, "_ptr", None), getattr(self, "_free", None)
+        if ptr is not None and ptr.value and free is not None:
+            free(ptr)
+            self._ptr = self._null
 
 
 def uw_encode_host(w: np.ndarray, opts: uw_encode_opts | None = None) -> HostEncoded:
@@ -278,6 +281,8 @@ class Handle:
         self._ptr = _vp(ptr)
         self.N, self.K = int(N), int(K)
         self._ws = None  # torch tensor kept alive while registered
+        # (module globals may be gone when __del__ runs at interpreter exit)
+        self._free, self._null = lib.uw_free, _vp(0)
 
     @property
     def ptr(self):
@@ -289,9 +294,10 @@ class Handle:
         return s.as_dict()
 
     def free(self):
-        if getattr(self, "_ptr", None) is not None and self._ptr.value:
-            lib.uw_free(self._ptr)
-            self._ptr = _vp(0)
+        ptr = getattr(self, "_ptr", None)
+        if ptr is not None and ptr.value:
+            self._free(ptr)
+            self._ptr = self._null
 
     def __del__(self):
         try:
