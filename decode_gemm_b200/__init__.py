@@ -30,6 +30,7 @@ lib = C.CDLL(LIB_PATH)
 # ----------------------------------------------------------------- constants --
 UW_OK, UW_ERR_ARG, UW_ERR_SHAPE, UW_ERR_FORMAT, UW_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
 UW_ERR_OOM, UW_ERR_CUDA, UW_ERR_DEVICE, UW_ERR_TIMEOUT, UW_ERR_WORKSPACE = 5, 6, 7, 8, 9
+UW_ERR_IO = 10
 UW_PIPE_AUTO, UW_PIPE_FULL, UW_PIPE_EXP, UW_PIPE_PALETTE_RT, UW_PIPE_PALETTE_DIRECT = 0, 1, 2, 3, 4
 PIPELINES = {"full": UW_PIPE_FULL, "exp": UW_PIPE_EXP, "palette_rt": UW_PIPE_PALETTE_RT,
              "palette_direct": UW_PIPE_PALETTE_DIRECT}
@@ -102,6 +103,9 @@ _SIGS = {
     "uw_host_free": ([_vp], None),
     "uw_validate_format": ([C.POINTER(uw_format)], C.c_int),
     "uw_host_stats": ([_vp, C.POINTER(uw_stats_t)], C.c_int),
+    "uw_host_save": ([_vp, C.c_char_p], C.c_int),
+    "uw_host_load": ([C.c_char_p, C.POINTER(_vp)], C.c_int),
+    "uw_load": ([C.c_char_p, C.POINTER(uw_encode_opts), _vp, C.POINTER(_vp)], C.c_int),
     "uw_upload": ([C.POINTER(uw_format), C.POINTER(uw_encode_opts), _vp, C.POINTER(_vp)], C.c_int),
     "uw_encode": ([_vp, _i64, _i64, C.POINTER(uw_encode_opts), _vp, C.POINTER(_vp)], C.c_int),
     "uw_free": ([_vp], C.c_int),
@@ -304,6 +308,29 @@ class Handle:
             self.free()
         except Exception:
             pass
+
+
+def uw_host_save(h: HostEncoded, path: str) -> None:
+    """Write a host encoding to a bundle file (see include/unweight.h)."""
+    _check(lib.uw_host_save(h.ptr, os.fsencode(path)), "uw_host_save")
+
+
+def uw_host_load(path: str) -> HostEncoded:
+    """Read a bundle file into a host encoding (checksummed and validated)."""
+    out = _vp()
+    _check(lib.uw_host_load(os.fsencode(path), C.byref(out)), "uw_host_load")
+    return HostEncoded(out.value)
+
+
+def uw_load(path: str, opts: uw_encode_opts | None = None, stream=None) -> Handle:
+    """A bundle file straight to the device (uw_host_load + uw_upload)."""
+    out = _vp()
+    _check(lib.uw_load(os.fsencode(path), C.byref(opts) if opts else None,
+                       _vp(_stream_ptr(stream)), C.byref(out)), "uw_load")
+    h = Handle(out.value, 0, 0)
+    st = h.stats()
+    h.N, h.K = int(st["N"]), int(st["K"])
+    return h
 
 
 def uw_upload(fmt: uw_format, opts: uw_encode_opts | None = None, stream=None) -> Handle:

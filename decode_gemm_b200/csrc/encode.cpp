@@ -423,6 +423,7 @@ const char* uw_status_str(uw_status s) {
     case UW_ERR_DEVICE: return "device reported corrupt input";
     case UW_ERR_TIMEOUT: return "device wait timed out";
     case UW_ERR_WORKSPACE: return "workspace missing or too small";
+    case UW_ERR_IO: return "file input/output failed";
   }
   return "unknown status";
 }

@@ -72,7 +72,8 @@ typedef enum uw_status {
   UW_ERR_CUDA = 6,         /* a CUDA runtime call failed                        */
   UW_ERR_DEVICE = 7,       /* a kernel reported corrupt input                   */
   UW_ERR_TIMEOUT = 8,      /* a kernel's bounded wait expired                   */
-  UW_ERR_WORKSPACE = 9     /* the pipeline needs a (larger) workspace           */
+  UW_ERR_WORKSPACE = 9,    /* the pipeline needs a (larger) workspace           */
+  UW_ERR_IO = 10           /* a file could not be opened, read or written       */
 } uw_status;
 
 /* Execution pipelines (*Unweight*, "Four ways to use compressed weights"). */
@@ -184,6 +185,19 @@ UW_API uw_status uw_validate_format(const uw_format* f);
 /* Statistics of a host-side encoding (no GPU). */
 UW_API uw_status uw_host_stats(uw_host_t h, uw_stats_t* out);
 
+/* Distribution bundle (*Unweight*, the untitled passage on format and execution:
+ * the Huffman package is what is shipped, and at load it is transcoded to the
+ * form inference runs on).  uw_host_save writes h to `path`: a 16-byte-aligned
+ * little-endian file holding the header (shape, code lengths, palette, exponent
+ * histogram, array sizes), the arrays of uw_format in their order, then a 64-bit
+ * FNV-1a checksum of all preceding bytes and an end tag.  uw_host_load reads such
+ * a file into a new host encoding (owned by the caller: uw_host_free) after
+ * checking the tag, the checksum, the header and uw_validate_format.  Errors:
+ * UW_ERR_ARG (null), UW_ERR_IO (open, read or write failed), UW_ERR_FORMAT
+ * (truncated, corrupted or not a bundle), UW_ERR_SHAPE, UW_ERR_OOM. */
+UW_API uw_status uw_host_save(uw_host_t h, const char* path);
+UW_API uw_status uw_host_load(const char* path, uw_host_t* out);
+
 /* ---- device side ---------------------------------------------------------- */
 
 /* Validate f, copy it to the current CUDA device on `stream` (a cudaStream_t,
@@ -193,6 +207,11 @@ UW_API uw_status uw_host_stats(uw_host_t h, uw_stats_t* out);
  * UW_ERR_CUDA. */
 UW_API uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream,
                     uw_handle_t* out);
+/* uw_host_load + uw_upload: a bundle straight to the device (with the load-time
+ * palette transcode when opts->prepare_direct; opts may be NULL for the
+ * defaults).  Errors: as uw_host_load and uw_upload. */
+UW_API uw_status uw_load(const char* path, const uw_encode_opts* opts, void* stream,
+                         uw_handle_t* out);
 /* uw_encode_host + uw_upload (the load-time entry point). */
 UW_API uw_status uw_encode(const uint16_t* w_host, int64_t N, int64_t K,
                     const uw_encode_opts* opts, void* stream, uw_handle_t* out);

@@ -163,3 +163,31 @@ def test_device_argument_errors(uw):
     assert uw.lib.uw_decode_exp(h.ptr, C.c_void_p(t.data_ptr() + 1)) == uw.UW_ERR_ARG
     assert uw.lib.uw_decode_full(None, C.c_void_p(t.data_ptr())) == uw.UW_ERR_ARG
     h.free()
+
+
+def test_bundle_load_to_device(uw, tmp_path):
+    """A distribution bundle loaded straight to the device (uw_load: read,
+    check, upload, load-time palette transcode) decodes bit-exactly and serves
+    the direct-palette matmul within tolerance."""
+    import torch
+    w = synthdata.student_t(256, 512, 3.0, 0.015, seed=67)  # with escape rows
+    he = uw.uw_encode_host(w, uw.default_opts(chunk_syms=128))
+    path = str(tmp_path / "m.uwb")
+    uw.uw_host_save(he, path)
+    h = uw.uw_load(path)
+    assert (h.N, h.K) == (256, 512)
+    assert h.stats()["n_escape_rows"] == he.stats()["n_escape_rows"] > 0
+    n, k = w.shape
+    wd, ed, idx = _run_all(uw, h, n, k)
+    assert np.array_equal(wd, w)
+    assert np.array_equal(ed, oracle.exponent_bytes(w))
+    x = synthdata.activations(8, k, seed=68)
+    X = torch.from_numpy(x.view(np.int16)).cuda()
+    Y = torch.empty((8, n), dtype=torch.float32, device="cuda")
+    uw.uw_gemm_f32(h, X, Y, 8, uw.UW_PIPE_PALETTE_DIRECT)
+    torch.cuda.synchronize()
+    assert uw.uw_last_device_status(h) == uw.UW_OK
+    ok, worst = oracle.within_tolerance(Y.cpu().numpy().astype(np.float64),
+                                        oracle.gemm_fp64(x, w), oracle.abs_product_sum(x, w))
+    assert ok, worst
+    h.free()
