@@ -184,6 +184,9 @@ def test_bundle_load_to_device(uw, tmp_path):
     x = synthdata.activations(8, k, seed=68)
     X = torch.from_numpy(x.view(np.int16)).cuda()
     Y = torch.empty((8, n), dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(uw.uw_workspace_bytes(h, uw.UW_PIPE_PALETTE_DIRECT, 8), 256),
+                     dtype=torch.uint8, device="cuda")  # split-K partial sums
+    uw.uw_set_workspace(h, ws)
     uw.uw_gemm_f32(h, X, Y, 8, uw.UW_PIPE_PALETTE_DIRECT)
     torch.cuda.synchronize()
     assert uw.uw_last_device_status(h) == uw.UW_OK
