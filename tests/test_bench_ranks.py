@@ -77,3 +77,15 @@ def test_reference_arm_rank0_line():
     assert d["higher_is_better"] is True and d["steps"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_source_digest_ignores_comments_only():
+    """The traffic figures stay valid across comment and layout edits, not code edits."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f(int x) {  // doubles x\n  return 2 * x; /* twice */\n}\n"
+    b = "// header\nint f(int x) {\n\n    return 2 * x;\n}\n"
+    c = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert len(bench._kernel_src_sha("gemm")) == 16 and bench._kernel_src_sha("decode") != bench._kernel_src_sha("gemm")
