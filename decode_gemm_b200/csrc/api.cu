@@ -392,6 +392,9 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
     free_handle(h);
     return map_cuda(e);
   }
+  // the allocation-free matmul serves handles with resident indices: its
+  // scratch array is brought into being now, while allocating is allowed
+  if (h->d_pal_idx) noalloc_prepare_device(h->device);
   *out = h;
   return UW_OK;
 }

@@ -78,4 +78,8 @@ struct DeviceGuard {
 // slot to pass to trace_end, or -1.
 int trace_begin(uw_handle_s* h, int kind);
 void trace_end(uw_handle_s* h, int slot);
+// Allocation-free matmul (noalloc.cu): make the scratch array of device `dev`
+// (current) exist and remember its address; called when a handle is uploaded
+// with the load-time palette transcode.
+void noalloc_prepare_device(int dev);
 }

@@ -10,6 +10,13 @@
 // Cost of the convenience: every GPU on which the library's device code is
 // loaded holds the array (kScratchFloats floats, 5 MiB) until the process
 // exits, and all calls share it.
+//
+// When the array comes into being: the CUDA driver allocates it when it loads
+// this file's device module, and with lazy module loading that happens at the
+// first lookup of its address.  uw_upload with prepare_direct (the only kind
+// of handle this entry point serves) does that lookup, so the allocation
+// happens at load time, when the caller can still allocate, not at the first
+// matmul.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -30,21 +37,42 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 float* g_scratch_ptr[kMaxDevices] = {nullptr};
 
-// Device address of the scratch array for the current device (looked up once
-// per device; the host-side symbol itself is not a device address).
+// Look up the scratch array's device address on the current device `dev` and
+// remember it (the host-side symbol itself is not a device address).
+uw_status lookup_scratch(int dev) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_gemm_scratch) != cudaSuccess || !p) return UW_ERR_CUDA;
+  g_scratch_ptr[dev] = static_cast<float*>(p);
+  return UW_OK;
+}
+
+// The remembered address for the current device `dev`; looked up here only if
+// no handle was uploaded with prepare_direct on this device before.
 uw_status scratch_for_device(int dev, float** out) {
   if (dev < 0 || dev >= kMaxDevices) return UW_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_gemm_scratch) != cudaSuccess || !p) return UW_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<float*>(p);
+    const uw_status st = lookup_scratch(dev);
+    if (st != UW_OK) return st;
   }
   *out = g_scratch_ptr[dev];
   return UW_OK;
 }
 
 }  // namespace
+
+namespace uw {
+// Called by uw_upload (prepare_direct) with the handle's device current: loads
+// the module that holds the array, so the driver allocates it now, and looks
+// its address up again.  Looking it up at every such upload also replaces an
+// address left over from a context that was destroyed (cudaDeviceReset) and
+// recreated since: every handle of the new context passes through here.
+void noalloc_prepare_device(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return;
+  std::lock_guard<std::mutex> lock(g_mu);
+  lookup_scratch(dev);  // a failure here resurfaces as UW_ERR_CUDA at the call
+}
+}  // namespace uw
 
 extern "C" {
 

@@ -277,9 +277,14 @@ UW_API uw_status uw_gemm_ex(uw_handle_t h, const uint16_t* X_dev, void* Y_dev, i
  *   - Limit: M <= 64 (UW_ERR_SHAPE above that).  The array is 5 MiB and is
  *     held on every GPU where the library's device code is loaded, until the
  *     process exits.
- *   - The handle's device must be current (UW_ERR_ARG otherwise).  The first
- *     call on a device looks up the array's device address once; make that
- *     first call before any stream capture.
+ *   - When the array is allocated: the CUDA driver allocates it when it loads
+ *     the library module that holds it.  uw_upload / uw_encode / uw_load with
+ *     prepare_direct load that module and look up the array's device address
+ *     on the handle's device, so the 5 MiB are taken at load time, not by this
+ *     call.  (Only if no such upload happened on the device does the first
+ *     call do the lookup itself; make that first call before any stream
+ *     capture.)
+ *   - The handle's device must be current (UW_ERR_ARG otherwise).
  *   - All calls on one GPU share the one array: calls whose kernels overlap
  *     on that GPU (for example on two streams) race and give wrong results.
  *     Nothing in it needs to start at zero, and its contents after a call

@@ -49,13 +49,21 @@ def test_noalloc_matches_uw_gemm_twice(uw, N, K, M, kind):
     y_exact = oracle.gemm_fp64(x, w)
     bound = oracle.abs_product_sum(x, w)
     assert oracle.within_tolerance(ref_np, y_exact, bound)[0]
-    # the allocation-free call, twice in a row, through the C ABI
-    for _ in range(2):
-        Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    # the allocation-free call, twice in a row, through the C ABI; the output
+    # buffers are made before the calls, so device memory use around each call
+    # shows what the call itself allocated
+    outs = [torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+            for _ in range(2)]
+    torch.cuda.synchronize()
+    for Y in outs:
+        free_before, _ = torch.cuda.mem_get_info()
+        torch_before = torch.cuda.memory_allocated()
         st = uw.lib.uw_gemm_palette_noalloc(h.ptr, C.c_void_p(X.data_ptr()),
                                             C.c_void_p(Y.data_ptr()), M, 1)
         assert st == uw.UW_OK, uw.uw_status_str(st)
         torch.cuda.synchronize()
+        assert torch.cuda.mem_get_info()[0] == free_before
+        assert torch.cuda.memory_allocated() == torch_before
         y = Y.cpu().numpy().astype(np.float64)
         ok, worst = oracle.within_tolerance(y, ref_np, bound)
         assert ok, worst
