@@ -131,6 +131,8 @@ _SIGS = {
                                 C.POINTER(_sz)], C.c_int),
     "uw_mlp_forward": ([C.POINTER(uw_mlp_layer), _i32, _vp, _vp, _i64, _vp, _sz, _vp, _vp,
                         C.POINTER(uw_mlp_opts)], C.c_int),
+    "uw_mlp_forward_record": ([C.POINTER(uw_mlp_layer), _i32, _vp, _vp, _i64, _vp, _sz, _vp,
+                               _vp, C.POINTER(uw_mlp_opts), _vp], C.c_int),
     "uw_mlp_tune_split": ([C.POINTER(uw_mlp_layer), _i32, _vp, _vp, _i64, _vp, _sz, _vp, _vp,
                            C.POINTER(uw_mlp_opts)], C.c_int),
     "uw_trace_read": ([_vp, C.POINTER(_i32), C.POINTER(C.c_float), _i32, C.POINTER(_i32)], C.c_int),
@@ -461,6 +463,19 @@ def uw_mlp_forward(layers, X, Y, M: int, ws, opts: uw_mlp_opts | None = None, st
     _check(lib.uw_mlp_forward(arr, len(layers), _vp(_dptr(X)), _vp(_dptr(Y)), int(M),
                               _vp(_dptr(ws)), nbytes, _vp(_stream_ptr(stream)), side,
                               C.byref(opts) if opts else None), "uw_mlp_forward")
+
+
+def uw_mlp_forward_record(layers, X, Y, M: int, ws, act, opts: uw_mlp_opts | None = None,
+                          stream=None, side_stream=None) -> None:
+    """uw_mlp_forward, also writing each layer's g, u, h and output into act
+    (device, per layer M*(3F + D) BF16 values in that order)."""
+    arr = mlp_layers(layers)
+    nbytes = ws.numel() * ws.element_size()
+    side = _vp(_stream_ptr(side_stream)) if side_stream is not None else None
+    _check(lib.uw_mlp_forward_record(arr, len(layers), _vp(_dptr(X)), _vp(_dptr(Y)), int(M),
+                                     _vp(_dptr(ws)), nbytes, _vp(_stream_ptr(stream)), side,
+                                     C.byref(opts) if opts else None, _vp(_dptr(act))),
+           "uw_mlp_forward_record")
 
 
 def uw_mlp_tune_split(layers, X, Y, M: int, ws, stream=None, side_stream=None) -> uw_mlp_opts:

@@ -172,9 +172,15 @@ uw_status uw_mlp_workspace_bytes(const uw_mlp_layer* layers, int32_t n_layers, i
   return UW_OK;
 }
 
-uw_status uw_mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uint16_t* X_dev,
-                         uint16_t* Y_dev, int64_t M, void* ws_dev, size_t ws_bytes,
-                         void* stream, void* side_stream, const uw_mlp_opts* opts) {
+}  // extern "C"
+
+namespace {
+
+// The stacked forward; when act is not null, each layer's g, u, h and output
+// are also copied there (main stream, right after they are produced).
+uw_status mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uint16_t* X_dev,
+                      uint16_t* Y_dev, int64_t M, void* ws_dev, size_t ws_bytes, void* stream,
+                      void* side_stream, const uw_mlp_opts* opts, uint16_t* act) {
   const uw_mlp_opts o = opts_or_default(opts);
   if (o.decode_ctas < 0 || o.gemm_ctas < 0) return UW_ERR_ARG;
   Plan pl;
@@ -243,6 +249,16 @@ uw_status uw_mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uin
     st = enqueue_pre(0);
   }
   const size_t xbytes = (size_t)M * pl.D * 2;
+  const size_t fbytes = (size_t)M * pl.F * 2;
+  // act layout per layer: g [M, F], u [M, F], h [M, F], output [M, D]
+  const size_t act_layer = (size_t)M * (3 * pl.F + pl.D);
+  auto record = [&](int layer, int part, const uint16_t* src, size_t bytes) -> uw_status {
+    if (!act) return UW_OK;
+    uint16_t* dst = act + (size_t)layer * act_layer + (size_t)part * M * pl.F;
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, ms) == cudaSuccess
+               ? UW_OK
+               : UW_ERR_CUDA;
+  };
   if (st == UW_OK && cudaMemcpyAsync(xb[0], X_dev, xbytes, cudaMemcpyDeviceToDevice, ms) != cudaSuccess)
     st = UW_ERR_CUDA;
   size_t hk = 0;  // index into `hard` of the next hard projection
@@ -271,9 +287,14 @@ uw_status uw_mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uin
       }
       ++hk;
     }
+    const int layer = (int)(i / 3);
+    if (st == UW_OK && pr.which == 0) st = record(layer, 0, gbuf, fbytes);
+    if (st == UW_OK && pr.which == 1) st = record(layer, 1, ubuf, fbytes);
     if (st == UW_OK && pr.which == 1) {  // h = SiLU(g) * u, in place over g
       if (launch_swiglu(gbuf, ubuf, gbuf, M * pl.F, ms) != cudaSuccess) st = UW_ERR_CUDA;
+      if (st == UW_OK) st = record(layer, 2, gbuf, fbytes);
     }
+    if (st == UW_OK && pr.which == 2) st = record(layer, 3, xb[cur ^ 1], xbytes);
     if (pr.which == 2) cur ^= 1;
   }
   if (st == UW_OK &&
@@ -281,6 +302,26 @@ uw_status uw_mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uin
     st = UW_ERR_CUDA;
   cleanup();
   return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+uw_status uw_mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uint16_t* X_dev,
+                         uint16_t* Y_dev, int64_t M, void* ws_dev, size_t ws_bytes,
+                         void* stream, void* side_stream, const uw_mlp_opts* opts) {
+  return mlp_forward(layers, n_layers, X_dev, Y_dev, M, ws_dev, ws_bytes, stream, side_stream,
+                     opts, nullptr);
+}
+
+uw_status uw_mlp_forward_record(const uw_mlp_layer* layers, int32_t n_layers,
+                                const uint16_t* X_dev, uint16_t* Y_dev, int64_t M, void* ws_dev,
+                                size_t ws_bytes, void* stream, void* side_stream,
+                                const uw_mlp_opts* opts, uint16_t* act_dev) {
+  if (!act_dev || (reinterpret_cast<uintptr_t>(act_dev) & 15)) return UW_ERR_ARG;
+  return mlp_forward(layers, n_layers, X_dev, Y_dev, M, ws_dev, ws_bytes, stream, side_stream,
+                     opts, act_dev);
 }
 
 uw_status uw_mlp_tune_split(const uw_mlp_layer* layers, int32_t n_layers, const uint16_t* X_dev,

@@ -363,6 +363,20 @@ UW_API uw_status uw_mlp_workspace_bytes(const uw_mlp_layer* layers, int32_t n_la
 UW_API uw_status uw_mlp_forward(const uw_mlp_layer* layers, int32_t n_layers, const uint16_t* X_dev,
                                 uint16_t* Y_dev, int64_t M, void* ws_dev, size_t ws_bytes,
                                 void* stream, void* side_stream, const uw_mlp_opts* opts);
+/* uw_mlp_forward that also records every layer's intermediate activations,
+ * for checking a compressed stack layer by layer against a reference.  act_dev
+ * (caller-owned, 16-byte aligned) receives, per layer l, at element offset
+ * l * M * (3F + D): g = x_l Wg^T [M, F], u = x_l Wu^T [M, F],
+ * h = SiLU(g) * u [M, F], x_{l+1} = h Wd^T [M, D] (BF16, row-major; F and D
+ * from the first layer's gate: [F, D]).  The copies are device-to-device on
+ * `stream`, right after each value is produced; the arithmetic, the variants
+ * and the overlap are those of uw_mlp_forward.  Errors as uw_mlp_forward, and
+ * UW_ERR_ARG for a null or misaligned act_dev. */
+UW_API uw_status uw_mlp_forward_record(const uw_mlp_layer* layers, int32_t n_layers,
+                                       const uint16_t* X_dev, uint16_t* Y_dev, int64_t M,
+                                       void* ws_dev, size_t ws_bytes, void* stream,
+                                       void* side_stream, const uw_mlp_opts* opts,
+                                       uint16_t* act_dev);
 /* Decoder/GEMM SM split for the overlapped stack: time uw_mlp_forward (overlap
  * on) for a few (decode_ctas, gemm_ctas) pairs and no split, return the
  * fastest in *best.  Synchronises `stream`. */

@@ -1,10 +1,11 @@
 """MLP stack driver, SwiGLU, autotuner and profile I/O on the GPU, through the C ABI.
 
-The stacked forward must equal, bit for bit, the same projections run one by
-one through uw_gemm_ex with the same variants plus uw_swiglu - with and
-without the side-stream overlap and the decoder/GEMM SM split (the split only
-changes which SMs run what, not the arithmetic, when the GEMM CTA count is
-the same).
+Every projection of the stacked forward is checked against the FP64 oracle
+given the GPU's own BF16 input to it (uw_mlp_forward_record), with and without
+the side-stream overlap and the decoder/GEMM SM split.  The stacked forward
+must also equal, bit for bit, the same projections run one by one through
+uw_gemm_ex with the same variants plus uw_swiglu (the split only changes which
+SMs run what, not the arithmetic, when the GEMM CTA count is the same).
 """
 import json
 import os
@@ -133,6 +134,62 @@ def test_mlp_forward_equals_call_sequence(uw, M):
                                    oracle.abs_product_sum(x, weights[0][0]))[0]
     for h in flat:
         h.free()
+
+
+SPLITS = {
+    "serial": dict(overlap=False),
+    "overlap": dict(overlap=True),
+    "overlap_decode4": dict(overlap=True, decode_ctas=4),
+    "overlap_decode4_gemm100": dict(overlap=True, decode_ctas=4, gemm_ctas=100),
+    "serial_gemm60": dict(overlap=False, gemm_ctas=60),
+}
+
+
+@pytest.mark.parametrize("M", [1, 24])
+@pytest.mark.parametrize("split", list(SPLITS))
+def test_mlp_stack_projections_against_fp64(uw, M, split):
+    """Every projection of a 3-layer stack run by uw_mlp_forward (hard and easy
+    pipelines mixed; preprocessing overlap and SM split on and off) against the
+    FP64 oracle, each given the GPU's own BF16 input to it; SwiGLU against the
+    oracle given the GPU's own g and u (*Unweight*, "Sharing the GPU between
+    decode and compute")."""
+    import torch
+    layers, weights = _layers(uw, 3, PIPES)
+    _load_pipelines(uw, layers, PIPES, M)
+    x = synthdata.activations(M, D, seed=160 + M)
+    X = torch.from_numpy(x.view(np.int16)).cuda()
+    side = torch.cuda.Stream()
+    opts = uw.mlp_opts(**SPLITS[split])
+    ws = torch.empty(uw.uw_mlp_workspace_bytes(layers, M, opts), dtype=torch.uint8, device="cuda")
+    per = M * (3 * F + D)
+    act = torch.full((len(layers) * per,), -1, dtype=torch.int16, device="cuda")
+    Y = torch.full((M, D), -1, dtype=torch.int16, device="cuda")
+    uw.uw_mlp_forward_record(layers, X, Y, M, ws, act, opts, side_stream=side)
+    torch.cuda.synchronize()
+    a = act.cpu().numpy().view(np.uint16).reshape(len(layers), per)
+    cur = x
+    for l, (wg, wu, wd) in enumerate(weights):
+        g = a[l, :M * F].reshape(M, F)
+        u = a[l, M * F:2 * M * F].reshape(M, F)
+        hh = a[l, 2 * M * F:3 * M * F].reshape(M, F)
+        nxt = a[l, 3 * M * F:].reshape(M, D)
+        for name, out, inp, w in (("gate", g, cur, wg), ("up", u, cur, wu), ("down", nxt, hh, wd)):
+            ok, worst = oracle.within_tolerance(oracle.to_float64(out), oracle.gemm_fp64(inp, w),
+                                                oracle.abs_product_sum(inp, w), bf16_output=True)
+            assert ok, (split, l, name, PIPES[l], worst)
+        ref = oracle.swiglu(g, u)
+        assert np.all(np.abs(oracle.to_float64(hh) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
+        cur = nxt
+    assert np.array_equal(Y.cpu().numpy().view(np.uint16), cur)
+    # recording changes nothing: the plain forward gives the same Y bit for bit
+    Y2 = torch.full((M, D), -1, dtype=torch.int16, device="cuda")
+    uw.uw_mlp_forward(layers, X, Y2, M, ws, opts, side_stream=side)
+    torch.cuda.synchronize()
+    assert np.array_equal(Y2.cpu().numpy().view(np.uint16), cur)
+    for trio in layers:
+        for h in trio:
+            assert uw.uw_last_device_status(h) == uw.UW_OK
+            h.free()
 
 
 def test_mlp_split_tuner_and_gemm_cta_cap(uw):
