@@ -92,6 +92,14 @@ def _palette_frequency_order(hist):
     return np.array(ranked, np.uint8)
 
 
+def _tolerance_full_step(bound, y_ref, bf16_output):
+    # a whole BF16 step allowed for the final rounding instead of half of one
+    tol = 1e-3 * bound + 1e-6
+    if bf16_output:
+        tol = tol + 2.0 ** -7 * np.abs(y_ref)
+    return tol
+
+
 CASES = [
     ("canonical order", oracle, "canonical_codes", _canonical_desc_within_length,
      pins.test_canonical_codes_rfc1951_example),
@@ -111,6 +119,8 @@ CASES = [
      pins.test_palette_order_and_padding),
     ("index halves swapped", oracle, "pack_nibbles", _pack_halves_swapped,
      pins.test_transcode_and_nibble_order),
+    ("BF16 allowance a full step", G, "tolerance", _tolerance_full_step,
+     pins.test_bf16_output_tolerance_branch),
 ]
 
 

@@ -348,6 +348,37 @@ def test_tolerance_rejects_transposed_operand():
     assert not oracle.within_tolerance(wrong, y, b)[0]
 
 
+def test_bf16_output_tolerance_branch():
+    """The BF16-output allowance covers the one final rounding to BF16 and no
+    more.  Exact sums are built from BF16 values with every product of one
+    sign (so sum |x w| = |y|, and the accumulation term is 1e-3 |y|):
+    round-to-nearest-even passes, rounding the wrong way or landing one BF16
+    step off fails.  (A BF16 step at y in [2^e, 2^(e+1)) is 2^(e-7).)"""
+    def bits(vals):
+        return synthdata.to_bf16_bits(np.array(vals, np.float32)).reshape(1, -1)
+
+    # y = 1 + 3 * 2^-9: between the BF16 values 1 and 1 + 2^-7, nearer the latter
+    x = bits([1.0, 1.0, 1.0] + [0.0] * 61)
+    w = bits([1.0, 2.0 ** -8, 2.0 ** -9] + [0.0] * 61)
+    y_ref = oracle.gemm_fp64(x, w)
+    b = oracle.abs_product_sum(x, w)
+    assert y_ref[0, 0] == 1.0 + 3 * 2.0 ** -9 and b[0, 0] == y_ref[0, 0]
+    ok = lambda y: oracle.within_tolerance(np.array([[y]]), y_ref, b, bf16_output=True)[0]
+    assert ok(1.0 + 2.0 ** -7)            # nearest BF16
+    assert not ok(1.0)                    # rounded the wrong way (3 * 2^-9 off)
+    assert not ok(1.0 + 2.0 ** -6)        # one BF16 step above the right answer
+    # y = 1.5 exactly representable: itself passes, one step (2^-7) either side fails
+    x1 = bits([1.0, 1.0] + [0.0] * 62)
+    w1 = bits([1.0, 0.5] + [0.0] * 62)
+    y1, b1 = oracle.gemm_fp64(x1, w1), oracle.abs_product_sum(x1, w1)
+    assert y1[0, 0] == 1.5
+    ok1 = lambda y: oracle.within_tolerance(np.array([[y]]), y1, b1, bf16_output=True)[0]
+    assert ok1(1.5)
+    assert not ok1(1.5 + 2.0 ** -7) and not ok1(1.5 - 2.0 ** -7)
+    # the FP32-output rule has no rounding allowance: 1 + 2^-7 fails there too
+    assert not oracle.within_tolerance(np.array([[1.0 + 2.0 ** -7]]), y_ref, b)[0]
+
+
 def test_synthetic_row_prefix_is_stable():
     a = synthdata.workload("gate_14336x4096", rows=8)
     b = synthdata.normal(32, 4096, 0.02, seed=10)[:8]
