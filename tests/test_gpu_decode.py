@@ -57,6 +57,13 @@ CASES = {
     "ragged_tail": lambda: (synthdata.normal(37, 192, 0.02, seed=46), 1024),
     "many_chunks_ragged_warp": lambda: (synthdata.normal(1000, 320, 0.02, seed=47), 64),
     "big_chunks": lambda: (synthdata.normal(128, 4096, 0.02, seed=48), 4096),
+    # small and mid-size chunks over special values, heavy tails, every
+    # exponent, a ragged last warp and many chunk groups per warp
+    "special_c64": lambda: (synthdata.special_values(96, 640, seed=52), 64),
+    "student_t_c256": lambda: (synthdata.student_t(300, 1280, 3.0, 0.015, seed=53), 256),
+    "all_exponents_c64": lambda: (synthdata.exponent_pattern(64, 1024, range(256), seed=54), 64),
+    "ragged_c256": lambda: (synthdata.normal(1000, 320, 0.02, seed=55), 256),
+    "many_groups_c256": lambda: (synthdata.normal(2048, 2048, 0.02, seed=56), 256),
 }
 
 
@@ -68,7 +75,7 @@ def test_decode_paths_match_oracle(uw, name):
     ref = oracle.encode(w, chunk_syms=chunk) if w.size <= 1 << 20 else None
     gw, ge, gi = _run_all(uw, h, n, k)
     assert np.array_equal(gw, w)
-    palette = np.array(h_palette(uw, h, w, chunk), np.uint8)
+    palette = oracle.build_palette(oracle.exponent_histogram(oracle.exponent_bytes(w)))
     esc = oracle.escape_rows(oracle.exponent_bytes(w), palette)
     e, i = _expect(w, palette, esc)
     assert np.array_equal(ge, e)
@@ -77,11 +84,6 @@ def test_decode_paths_match_oracle(uw, name):
         assert np.array_equal(palette, ref.palette)
         assert np.array_equal(oracle.transcode_from_stream(ref), gi)
     h.free()
-
-
-def h_palette(uw, h, w, chunk):
-    # the palette of the library's encoding (host encoder is byte-identical to the oracle's)
-    return uw.uw_encode_host(w, uw.default_opts(chunk_syms=chunk)).arrays()["palette"]
 
 
 def test_gpu_decodes_oracle_encoded_stream(uw):
@@ -107,7 +109,7 @@ def test_decode_full_size_bit_exact(uw, name):
     assert np.array_equal(gw, w)
     s, e = oracle.split_fields(w)
     assert np.array_equal(ge, e)
-    pal = np.asarray(h_palette(uw, h, w, 256))
+    pal = oracle.build_palette(oracle.exponent_histogram(e))
     esc = oracle.escape_rows(e, pal)
     assert np.array_equal(gi, oracle.pack_nibbles(oracle.transcode(e, pal, esc)))
     # sampled chunks through the oracle's bit-by-bit decoder on the library stream

@@ -168,21 +168,72 @@ def test_gate_proj_full_size(uw, M):
     h.free()
 
 
-@pytest.mark.parametrize("M", [256, 1024])
-def test_down_proj_full_size_sampled(uw, M):
-    w = synthdata.workload("down_4096x14336")
-    x = synthdata.activation_for("down_4096x14336", M)
-    h = _upload(uw, w)
-    ws = _workspace(uw, h, M)
-    rng = np.random.default_rng(M)
-    rows = rng.choice(M, size=min(M, 24), replace=False)
+def _sampled_rows_check(uw, h, w, x, M, seed, n_rows):
+    """Every pipeline at M tokens against FP64 on n_rows sampled token rows
+    (all of them when M <= n_rows); only those rows leave the GPU.  Returns the
+    sampled outputs per pipeline."""
+    import torch
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(M, size=min(M, n_rows), replace=False))
     ref = oracle.gemm_fp64(x[rows], w)
     bound = oracle.abs_product_sum(x[rows], w)
+    X = torch.from_numpy(x.view(np.int16)).cuda()
+    Y = torch.empty((M, h.N), dtype=torch.float32, device="cuda")
+    sel = torch.from_numpy(rows).cuda()
+    outs = {}
     for p in PIPES:
-        y = _gemm(uw, h, x, p)[rows]
+        Y.fill_(float("nan"))
+        uw.uw_gemm_ex(h, X, Y, M, uw.gemm_config(uw.PIPELINES[p]), True)
+        torch.cuda.synchronize()
+        assert uw.uw_last_device_status(h) == uw.UW_OK
+        y = Y.index_select(0, sel).cpu().numpy().astype(np.float64)
         ok, worst = oracle.within_tolerance(y, ref, bound)
         assert ok, (p, worst)
+        assert not torch.isnan(Y).any().item(), p  # every output element written
+        outs[p] = y
+    return outs
+
+
+@pytest.fixture(scope="module")
+def down8b(uw):
+    """The Llama-3.1-8B down_proj shape 4096x14336, uploaded once."""
+    w = synthdata.workload("down_4096x14336")
+    h = _upload(uw, w)
+    yield w, h
     h.free()
+
+
+@pytest.mark.parametrize("M", [256, 1024, 4096])
+def test_down_proj_full_size_sampled(uw, down8b, M):
+    w, h = down8b
+    x = synthdata.activation_for("down_4096x14336", M)
+    _workspace(uw, h, M)
+    outs = _sampled_rows_check(uw, h, w, x, M, seed=M, n_rows=24 if M < 4096 else 32)
+    assert np.array_equal(outs["exp"], outs["palette_rt"])
+    assert np.array_equal(outs["exp"], outs["palette_direct"])
+
+
+@pytest.fixture(scope="module")
+def down70b(uw):
+    """The 70B-shaped down projection 8192x28672 (Student-t weights)."""
+    w = synthdata.workload("down70b_8192x28672")
+    h = _upload(uw, w)
+    yield w, h
+    h.free()
+
+
+@pytest.mark.parametrize("M", [1, 4096])
+def test_down70b_shape_sampled(uw, down70b, M):
+    """8192x28672 (K = 28672, the longest reduction here) with heavy tails:
+    every pipeline within tolerance on sampled token rows, the reconstructive
+    ones bitwise equal."""
+    w, h = down70b
+    assert h.stats()["n_escape_rows"] > 0
+    x = synthdata.activation_for("down70b_8192x28672", M)
+    _workspace(uw, h, M)
+    outs = _sampled_rows_check(uw, h, w, x, M, seed=71 + M, n_rows=8)
+    assert np.array_equal(outs["exp"], outs["palette_rt"])
+    assert np.array_equal(outs["exp"], outs["palette_direct"])
 
 
 @pytest.fixture(scope="module")
