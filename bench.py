@@ -57,13 +57,13 @@ CPU_BASELINE_ROWS = 300   # oracle rows for the cpu_baseline leg (~12 s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum; profiles/*.md), valid only while the kernel source
+# dram__bytes_write.sum of one launch), valid only while the kernel source
 # (src_sha, see _kernel_src_sha) is unchanged.
 TRAFFIC = {
     "gemm_palette": {"bytes_per_launch": 89.686016e6 + 3.780352e6, "src_sha": "86199055be906a41",
-                     "capture": "profiles/gemm_palette_gate_14336x4096_M1.md (M = 1 launch)"},
+                     "capture": "palette GEMM, 14336x4096, M = 1 launch"},
     "decode_full": {"bytes_per_launch": 87.243776e6 + 66.097408e6, "src_sha": "ee0a4d48dea442f1",
-                    "capture": "profiles/decode_full_gate_14336x4096.md (output partly still in L2)"},
+                    "capture": "full decode, 14336x4096 (output partly still in L2)"},
 }
 
 def _args():

@@ -27,16 +27,17 @@ CPP_FLAGS = COMMON + ["-Wno-deprecated-gpu-targets"]
 
 SOURCES = ["encode.cpp", "bundle.cpp", "api.cu", "decode.cu", "gemm.cu", "autotune.cu", "noalloc.cu",
            "mlp.cu"]
-HEADERS = ["uw_internal.h", "uw_kernels.h", "handle.h", "gemm_sm100.cuh"]
+
+
+def _headers() -> list:
+    """Every header a source may include: the public one and all of csrc's."""
+    hs = [os.path.join(INCLUDE, "unweight.h")]
+    hs += [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".h", ".cuh"))]
+    return hs
 
 
 def _newest_header() -> float:
-    t = os.path.getmtime(os.path.join(INCLUDE, "unweight.h"))
-    for h in HEADERS:
-        p = os.path.join(CSRC, h)
-        if os.path.exists(p):
-            t = max(t, os.path.getmtime(p))
-    return t
+    return max(os.path.getmtime(p) for p in _headers())
 
 
 def _compile(src: str, verbose: bool) -> str:
