@@ -74,6 +74,8 @@ def _args():
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-large-m", action="store_true",
+                    help="skip the large-M matmul block (gate M = 1024, down M = 256, 1024)")
     # single-kernel runs for profilers: three launches of one kernel, nothing timed
     ap.add_argument("--only", choices=("decode_full", "decode_exp", "transcode", "gemm_bf16",
                                        "gemm_exp", "gemm_palette"))
@@ -82,6 +84,10 @@ def _args():
     ap.add_argument("--mlp-layers", type=int, default=0,
                     help="time uw_mlp_forward over this many gate/up/down layers")
     ap.add_argument("--mlp-ms", default="1,64,256,1024")
+    ap.add_argument("--mlp-force-down", default="",
+                    help="comma list of pipelines (2, 3) to force on every down_proj, gate/up "
+                         "on pipeline 4: times the stack with the preprocessing overlap off, "
+                         "on, and with the tuned decoder/GEMM SM split")
     return ap.parse_args()
 
 
@@ -158,6 +164,105 @@ def _block_time(uw, torch, kind, handles, stats, X, Y, Ms, N, K, stream, rounds)
     torch.cuda.synchronize()
     n = rounds * (len(Ms) if kind.startswith("gemm") else 1) * len(handles)
     return e0.elapsed_time(e1), n, total
+
+
+# Large-M matmul block of the bench line: (workload, M) pairs, and the
+# weight sets rotated per call so a pipeline's weights are not in L2.
+LARGE_M = (("gate_14336x4096", 1024), ("down_4096x14336", 256), ("down_4096x14336", 1024))
+LARGE_M_SETS = 2
+
+
+def _large_m_block(uw, torch, stream, peaks, reps=8):
+    """Every pipeline at the metric's large M on the gate and down shapes:
+    whole-pipeline time (calls back to back between two events, weight sets
+    rotated), its split into preprocessing and GEMM (the library's traced
+    events), the GEMM's TFLOP/s and its roofline time max(2MNK / BF16 peak,
+    algorithmic bytes / HBM peak), and torch.matmul on the decoded BF16
+    weights for context."""
+    import numpy as np
+    import synthdata
+    out = {}
+    by_wl = {}
+    for wl, M in LARGE_M:
+        by_wl.setdefault(wl, []).append(M)
+    for wl, Ms in by_wl.items():
+        spec = synthdata.WORKLOADS[wl]
+        N, K = spec["N"], spec["K"]
+        hs, sts = [], []
+        for i in range(LARGE_M_SETS):
+            w = synthdata.normal(N, K, spec["std"], spec["seed_w"] + 2 * i)
+            h = uw.uw_encode(w, stream=stream)
+            hs.append(h)
+            sts.append(h.stats())
+            del w
+        need = max(uw.uw_workspace_bytes(hs[0], uw.PIPELINES[p], m) for p in PIPES for m in Ms)
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        for h in hs:
+            uw.uw_set_workspace(h, ws)
+        wbf = []
+        for h in hs:
+            t = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+            uw.uw_decode_full(h, t)
+            wbf.append(t)
+        for M in Ms:
+            X = torch.from_numpy(synthdata.activations(M, K, spec["seed_x"] + M).view(np.int16)) \
+                .cuda().view(torch.bfloat16)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            flops = 2.0 * M * N * K
+            rec = {}
+            for p in PIPES:
+                pre, gemm = _run_kernels(p)
+                call = lambda i: uw.uw_gemm(hs[i % LARGE_M_SETS], X, Y, M, uw.PIPELINES[p])
+                for i in range(3):
+                    call(i)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for i in range(reps):
+                    call(i)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                total_us = 1e3 * e0.elapsed_time(e1) / reps
+                # traced split (events around each kernel)
+                for h in hs:
+                    uw.uw_trace_read(h)
+                    uw.uw_trace_enable(h, True)
+                for i in range(reps):
+                    call(i)
+                torch.cuda.synchronize()
+                tr = [x for h in hs for x in uw.uw_trace_read(h)]
+                for h in hs:
+                    uw.uw_trace_enable(h, False)
+                g_ms = [ms for kind, ms in tr if kind == gemm]
+                p_ms = [ms for kind, ms in tr if kind == pre] if pre else []
+                gemm_us = 1e3 * statistics.median(g_ms)
+                pre_us = 1e3 * statistics.median(p_ms) if p_ms else 0.0
+                gbytes = _alg_bytes(gemm, sts[0], M, N, K)
+                t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), gbytes / (peaks["hbm_gbs"] * 1e9))
+                rec[p] = {"total_us": total_us, "preprocess_us_traced": pre_us,
+                          "gemm_us_traced": gemm_us, "gemm_tflops": flops / (gemm_us * 1e-6) / 1e12,
+                          "gemm_roofline_us": 1e6 * t_roof,
+                          "gemm_frac": 1e6 * t_roof / gemm_us,
+                          "gemm_bound": "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >=
+                          gbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+            ts = []
+            for i in range(3 + reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                torch.matmul(X, wbf[i % LARGE_M_SETS].t())
+                b.record(stream)
+                b.synchronize()
+                if i >= 3:
+                    ts.append(1e3 * a.elapsed_time(b))
+            rec["torch_matmul_bf16_us"] = statistics.median(ts)
+            rec["torch_matmul_bf16_tflops"] = flops / (rec["torch_matmul_bf16_us"] * 1e-6) / 1e12
+            out[f"{wl}/M{M}"] = rec
+        for h in hs:
+            if uw.uw_last_device_status(h) != uw.UW_OK:
+                raise RuntimeError("device status")
+            h.free()
+        del wbf, ws
+    return out
 
 
 def _run_kernels(pipe):
@@ -274,6 +379,86 @@ def cpu_oracle_sample(rows=4, ms=MS, target_s=None):
     desc = (f"first {rows} rows of {WORKLOAD} ({rows * k} weights) encoded on their own; "
             f"4 pipelines x M in {list(ms)}; oracle bit-by-bit decode + FP64 matmul, 1 thread")
     return alg / dt / 1e9, dt, desc
+
+
+def _oracle_decode_range(args):
+    """Worker of the all-cores CPU leg: the oracle's bit-by-bit decode of the
+    chunks [c0, c1) of one encoded sample (module-level so a spawned process
+    can run it)."""
+    import numpy as np
+    import oracle
+    words, offsets, lengths, total, cs, c0, c1 = args
+    words = [int(x) for x in words]  # one conversion per job, as decode_bitstream does
+    out = []
+    for c in range(c0, c1):
+        n = min(cs, total - c * cs)
+        syms, _ = oracle.decode_chunk(words, int(offsets[c]), n, lengths)
+        out.append(np.asarray(syms, dtype=np.uint8))
+    return c0, out
+
+
+def cpu_oracle_sample_all_cores(rows=CPU_BASELINE_ROWS, ms=MS):
+    """The same sample and work as cpu_oracle_sample on every host core: each
+    pipeline's bit-by-bit decode split into chunk ranges over a spawned
+    process pool (chunks decode independently by construction), the FP64
+    matmul with BLAS on all threads.  Returns (GB/s, seconds, cores)."""
+    import multiprocessing as mp
+    import numpy as np
+    import oracle
+    import synthdata
+    from oracle.container import rebuild_from_palette
+    cores = os.cpu_count() or 1
+    w = synthdata.workload(WORKLOAD, rows=rows)
+    n, k = w.shape
+    enc = oracle.encode(w, chunk_syms=256)
+    st = {"bytes_stream": (enc.total_bits + 7) // 8, "bytes_offsets": enc.offsets.size * 4,
+          "bytes_escape": enc.esc_exp.size + enc.esc_bits.size * 4 + enc.esc_off.size * 4}
+    xs = {m: synthdata.activation_for(WORKLOAD, m) for m in ms}
+    n_chunks = enc.offsets.size - 1
+    step = -(-n_chunks // cores)
+    jobs = []
+    for c0 in range(0, n_chunks, step):
+        c1 = min(c0 + step, n_chunks)
+        # each job gets only its stretch of the stream, offsets rebased to it
+        w0 = int(enc.offsets[c0]) // 32
+        w1 = min(int(enc.offsets[c1]) // 32 + 2, enc.words.size)
+        offs = enc.offsets.astype(np.int64) - 32 * w0
+        jobs.append((enc.words[w0:w1].copy(), offs[:c1 + 1], enc.lengths, n * k,
+                     enc.chunk_syms, c0, c1))
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(min(cores, len(jobs))) as pool:
+        pool.map(_oracle_decode_range, jobs[:1])  # workers up and importing before timing
+
+        def decode_exp():
+            parts = sorted(pool.map(_oracle_decode_range, jobs), key=lambda t: t[0])
+            return np.concatenate([np.concatenate(p[1]) for p in parts]).reshape(n, k)
+
+        alg = 0
+        t0 = time.perf_counter()
+        for m in ms:
+            x = xs[m]
+            for pipe in PIPES:
+                if pipe == "full":
+                    wd = oracle.join_fields(enc.sm, decode_exp())
+                elif pipe == "exp":
+                    wd = oracle.join_fields(enc.sm, decode_exp())
+                elif pipe == "palette_rt":
+                    e = decode_exp()
+                    wd = rebuild_from_palette(enc, oracle.pack_nibbles(
+                        oracle.transcode(e, enc.palette, enc.esc)))
+                else:
+                    packed = oracle.pack_nibbles(oracle.transcode(oracle.exponent_bytes(w),
+                                                                  enc.palette, enc.esc))
+                    wd = rebuild_from_palette(enc, packed)
+                y = oracle.gemm_fp64(x, wd)
+                assert y.shape == (m, n)
+                pre, gemm = _run_kernels(pipe)
+                frac = n / synthdata.WORKLOADS[WORKLOAD]["N"]
+                if pre:
+                    alg += _alg_bytes(pre, st, m, n, k, frac)
+                alg += _alg_bytes(gemm, st, m, n, k, frac)
+        dt = time.perf_counter() - t0
+    return alg / dt / 1e9, dt, cores
 
 
 def max_over_ranks(x, world, device="cuda"):
@@ -523,6 +708,16 @@ def run_ours(args):
                                   "gemm_tflops": 2 * m * N * K / (g * 1e-6) / 1e12
                                   if g > 0 else None}
 
+    # ---- each preprocessing kernel alone, back to back (the traced figures
+    # above carry each launch's own event and start-up cost)
+    for kind in ("decode_full", "decode_exp", "transcode"):
+        if kind in kernels:
+            bt = _block_time(uw, torch, kind, handles, stats, X, Y, Ms, N, K, stream,
+                             rounds=max(args.steps // 2, 3))
+            gbs = bt[2] / (bt[0] * 1e-3) / 1e9
+            kernels[kind].update({"b2b_launches": bt[1], "b2b_us": 1e3 * bt[0] / bt[1],
+                                  "b2b_GBps": gbs, "b2b_frac_hbm": gbs / peaks["hbm_gbs"]})
+
     # ---- BF16 torch.matmul on the same box (context only)
     wbf = []
     for h in handles:
@@ -543,6 +738,9 @@ def run_ours(args):
                 ts.append(a.elapsed_time(b) * 1e3)
         tm[f"M{m}"] = statistics.median(ts)
     del wbf
+
+    # ---- the metric's large-M matmuls (gate and down shapes)
+    gemm_large = None if args.no_large_m else _large_m_block(uw, torch, stream, peaks)
 
     # ---- end to end through the public call with host buffers
     Xh = {m: X[m].cpu().pin_memory() for m in Ms}
@@ -570,9 +768,13 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, dt, desc = cpu_oracle_sample(rows=CPU_BASELINE_ROWS)
-        cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
-               "seconds": dt}
+        v1, dt1, desc = cpu_oracle_sample(rows=CPU_BASELINE_ROWS)
+        va, dta, cores = cpu_oracle_sample_all_cores(rows=CPU_BASELINE_ROWS)
+        cpu = {"value": va, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": desc.replace(", 1 thread", "") + f"; on all {cores} host cores "
+                         "(decode chunks over a spawned process pool, BLAS on all threads)",
+               "seconds": dta, "host_cpu_count": os.cpu_count(),
+               "single_core": {"value": v1, "cores": 1, "seconds": dt1}}
 
     st0 = stats[0]
     line = {
@@ -590,6 +792,7 @@ def run_ours(args):
         "kernels": kernels,
         "pipelines": pipelines,
         "torch_matmul_bf16_us": tm,
+        "gemm_large_m": gemm_large,
         "gpu_launches": launches,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -676,6 +879,10 @@ def run_mlp(args):
             del w
         layers.append(tuple(trio))
         wbf.append(bfs)
+    side = torch.cuda.Stream()
+    if args.mlp_force_down:
+        return _mlp_overlap_modes(args, uw, torch, np, synthdata, layers, wbf, Ms, D, side, bf,
+                                  comp)
     flat0 = list(layers[0])
     need = max(uw.uw_workspace_bytes(h, p, max(Ms)) for h in flat0 for p in (1, 2, 3, 4))
     ws0 = torch.empty(need, dtype=torch.uint8, device="cuda")
@@ -686,7 +893,6 @@ def run_mlp(args):
         uw.uw_autotune(flat0, Ms, prof)
         for trio in layers[1:]:
             uw.uw_load_profile(list(trio), prof)
-    side = torch.cuda.Stream()
     out = {}
     for M in Ms:
         x = synthdata.activations(M, D, 3000 + M)
@@ -728,6 +934,84 @@ def run_mlp(args):
     print(json.dumps({"mode": "mlp_stack", "layers": L, "unit": "ms per forward",
                       "weights_bf16_bytes": bf, "weights_compressed_bytes": comp,
                       "data": "synthetic", "results": out}), flush=True)
+    for trio in layers:
+        for h in trio:
+            h.free()
+    return 0
+
+
+def _mlp_overlap_modes(args, uw, torch, np, synthdata, layers, wbf, Ms, D, side, bf, comp):
+    """The stack with every down_proj forced onto a hard pipeline (one that
+    needs Huffman preprocessing) and gate/up on pipeline 4 (*Unweight*,
+    "Sharing the GPU between decode and compute": down_proj gains most from
+    overlapping its preprocessing).  For each M: the forward with the
+    preprocessing serial on the main stream, overlapped on a side stream (all
+    SMs for each kernel), and with the SM split uw_mlp_tune_split picks;
+    torch BF16 on the uncompressed weights for context."""
+    import json as _json
+    import tempfile
+    results = {}
+    for pd in [int(x) for x in args.mlp_force_down.split(",") if x]:
+        per_m = {}
+        for M in Ms:
+            prof = {"version": 1, "handles": []}
+            for trio in layers:
+                for h, p in zip(trio, (4, 4, pd)):
+                    prof["handles"].append({"N": h.N, "K": h.K, "choices": [
+                        {"M": M, "pipeline": p, "tile_n": 0, "stages": 0, "gemm_ctas": 0,
+                         "decode_ctas": 0}]})
+            with tempfile.NamedTemporaryFile("w", suffix=".json", delete=False) as f:
+                _json.dump(prof, f)
+                path = f.name
+            uw.uw_load_profile([h for trio in layers for h in trio], path)
+            os.unlink(path)
+            x = synthdata.activations(M, D, 3000 + M)
+            X = torch.from_numpy(x.view(np.int16)).cuda()
+            Y = torch.empty((M, D), dtype=torch.int16, device="cuda")
+            ws = torch.empty(max(uw.uw_mlp_workspace_bytes(layers, M, uw.mlp_opts(o))
+                                 for o in (False, True)), dtype=torch.uint8, device="cuda")
+
+            def timed(fn, it=5):
+                for _ in range(2):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(it):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                return e0.elapsed_time(e1) / it
+
+            serial = timed(lambda: uw.uw_mlp_forward(layers, X, Y, M, ws, uw.mlp_opts(False),
+                                                     side_stream=side))
+            overlap = timed(lambda: uw.uw_mlp_forward(layers, X, Y, M, ws, uw.mlp_opts(True),
+                                                      side_stream=side))
+            best = uw.uw_mlp_tune_split(layers, X, Y, M, ws, side_stream=side)
+            tuned = timed(lambda: uw.uw_mlp_forward(layers, X, Y, M, ws, best, side_stream=side))
+            xb = X.view(torch.bfloat16)
+
+            def ref():
+                cur = xb
+                for g, u, dw in wbf:
+                    a, b = cur @ g.t(), cur @ u.t()
+                    cur = (torch.nn.functional.silu(a.float()) * b.float()).to(torch.bfloat16) \
+                        @ dw.t()
+                return cur
+
+            base = timed(ref)
+            for trio in layers:
+                for h in trio:
+                    if uw.uw_last_device_status(h) != uw.UW_OK:
+                        raise RuntimeError("device status")
+            per_m[f"M{M}"] = {"serial_ms": serial, "overlap_ms": overlap, "tuned_split_ms": tuned,
+                              "tuned_split": best.as_dict(), "torch_bf16_ms": base,
+                              "overlap_gain": serial / overlap, "tuned_gain": serial / tuned}
+        results[f"down_pipeline_{pd}"] = per_m
+    print(json.dumps({"mode": "mlp_overlap", "layers": len(layers), "unit": "ms per forward",
+                      "gate_up_pipeline": 4, "weights_bf16_bytes": bf,
+                      "weights_compressed_bytes": comp, "data": "synthetic",
+                      "results": results}), flush=True)
     for trio in layers:
         for h in trio:
             h.free()
