@@ -78,7 +78,8 @@ def _args():
                     help="skip the large-M matmul block (gate M = 1024, down M = 256, 1024)")
     # single-kernel runs for profilers: three launches of one kernel, nothing timed
     ap.add_argument("--only", choices=("decode_full", "decode_exp", "transcode", "gemm_bf16",
-                                       "gemm_exp", "gemm_palette"))
+                                       "gemm_exp", "gemm_palette", "gemv_bf16", "gemv_exp",
+                                       "gemv_palette"))
     ap.add_argument("--m", type=int, default=1, help="tokens for --only gemm_*")
     # the Llama-3.1-8B-shaped MLP stack end to end (prints its own JSON line)
     ap.add_argument("--mlp-layers", type=int, default=0,
@@ -110,14 +111,15 @@ def _alg_bytes(kind, st, M, N, K, x_frac=1.0):
     stream = st["bytes_stream"] + st["bytes_offsets"]
     esc = st["bytes_escape"]
     xy = x_frac * 2 * M * K + 2 * M * N
-    return {
+    b = {
         "decode_full": stream + T + 2 * T,
         "decode_exp": stream + T,
         "transcode": stream + T // 2,
         "gemm_bf16": 2 * T + xy,
         "gemm_exp": 2 * T + xy,
         "gemm_palette": T + T // 2 + esc + xy,
-    }[kind]
+    }
+    return b[kind.replace("gemv_", "gemm_")]
 
 
 def _block_time(uw, torch, kind, handles, stats, X, Y, Ms, N, K, stream, rounds):
@@ -127,6 +129,7 @@ def _block_time(uw, torch, kind, handles, stats, X, Y, Ms, N, K, stream, rounds)
     alone (the BF16 and exponent GEMMs always follow their decode)."""
     if kind not in ("decode_full", "decode_exp", "transcode", "gemm_palette"):
         return None
+
     out = None
     if kind == "decode_full":
         out = torch.empty(N * K, dtype=torch.int16, device="cuda")
@@ -147,7 +150,7 @@ def _block_time(uw, torch, kind, handles, stats, X, Y, Ms, N, K, stream, rounds)
 
     def one_round():
         b = 0
-        for m in (Ms if kind.startswith("gemm") else Ms[:1]):
+        for m in (Ms if kind.startswith(("gemm", "gemv")) else Ms[:1]):
             for i, h in enumerate(handles):
                 launch(h, m)
                 b += _alg_bytes(kind, stats[i], m, N, K)
@@ -162,7 +165,7 @@ def _block_time(uw, torch, kind, handles, stats, X, Y, Ms, N, K, stream, rounds)
         total += one_round()
     e1.record(stream)
     torch.cuda.synchronize()
-    n = rounds * (len(Ms) if kind.startswith("gemm") else 1) * len(handles)
+    n = rounds * (len(Ms) if kind.startswith(("gemm", "gemv")) else 1) * len(handles)
     return e0.elapsed_time(e1), n, total
 
 
@@ -211,7 +214,7 @@ def _large_m_block(uw, torch, stream, peaks, reps=8):
             flops = 2.0 * M * N * K
             rec = {}
             for p in PIPES:
-                pre, gemm = _run_kernels(p)
+                pre, gemm = _run_kernels(p, M)
                 call = lambda i: uw.uw_gemm(hs[i % LARGE_M_SETS], X, Y, M, uw.PIPELINES[p])
                 for i in range(3):
                     call(i)
@@ -265,11 +268,13 @@ def _large_m_block(uw, torch, stream, peaks, reps=8):
     return out
 
 
-def _run_kernels(pipe):
+def _run_kernels(pipe, M):
+    """(preprocessing kernel or None, matmul kernel) of a pipeline at M tokens
+    with the library's default variant (the tensor-core GEMM at every M)."""
     pre = {"full": "decode_full", "exp": "decode_exp", "palette_rt": "transcode",
            "palette_direct": None}[pipe]
-    gemm = {"full": "gemm_bf16", "exp": "gemm_exp"}.get(pipe, "gemm_palette")
-    return pre, gemm
+    gemm = {"full": "bf16", "exp": "exp"}.get(pipe, "palette")
+    return pre, "gemm_" + gemm
 
 
 # ------------------------------------------------------------------- clocks --
@@ -368,7 +373,7 @@ def cpu_oracle_sample(rows=4, ms=MS, target_s=None):
                 wd = rebuild_from_palette(enc, packed)
             y = oracle.gemm_fp64(x, wd)
             assert y.shape == (m, n)
-            pre, gemm = _run_kernels(pipe)
+            pre, gemm = _run_kernels(pipe, m)
             frac = n / synthdata.WORKLOADS[WORKLOAD]["N"]  # this slice's share of X traffic
             if pre:
                 alg += _alg_bytes(pre, st, m, n, k, frac)
@@ -452,7 +457,7 @@ def cpu_oracle_sample_all_cores(rows=CPU_BASELINE_ROWS, ms=MS):
                     wd = rebuild_from_palette(enc, packed)
                 y = oracle.gemm_fp64(x, wd)
                 assert y.shape == (m, n)
-                pre, gemm = _run_kernels(pipe)
+                pre, gemm = _run_kernels(pipe, m)
                 frac = n / synthdata.WORKLOADS[WORKLOAD]["N"]
                 if pre:
                     alg += _alg_bytes(pre, st, m, n, k, frac)
@@ -522,6 +527,7 @@ def _load_build():
 KERNEL_SOURCES = {
     "decode": ("decode.cu", "bf16_fields.cuh", "pdl.cuh"),
     "gemm": ("gemm.cu", "gemm_sm100.cuh", "bf16_fields.cuh", "pdl.cuh"),
+    "gemv": ("gemv.cu", "bf16_fields.cuh", "pdl.cuh"),
 }
 
 
@@ -595,7 +601,7 @@ def run_ours(args):
         tot = 0
         for j, (m, p) in enumerate(runs):
             st = stats[(run0 + j) % N_SETS]
-            pre, gemm = _run_kernels(p)
+            pre, gemm = _run_kernels(p, m)
             if pre:
                 tot += _alg_bytes(pre, st, m, N, K)
             tot += _alg_bytes(gemm, st, m, N, K)
@@ -608,7 +614,7 @@ def run_ours(args):
 
     # ---- device-resident timed region (untraced)
     total_bytes = sum(step_bytes(run0 + s * len(runs)) for s in range(args.steps))
-    launches = args.steps * sum(1 + (_run_kernels(p)[0] is not None) for (_, p) in runs)
+    launches = args.steps * sum(1 + (_run_kernels(p, m)[0] is not None) for (m, p) in runs)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         if world > 1:
@@ -649,7 +655,7 @@ def run_ours(args):
         for j, (m, p) in enumerate(runs):
             idx = (run_start + s * len(runs) + j) % N_SETS
             tr = traces[idx]
-            pre, gemm = _run_kernels(p)
+            pre, gemm = _run_kernels(p, m)
             st = stats[idx]
             rec = {}
             for kind in ([pre] if pre else []) + [gemm]:
@@ -662,7 +668,7 @@ def run_ours(args):
                     agg["ms"] += tr[c][1]
                     agg["n"] += 1
                     agg["bytes"] += b
-                    if kind.startswith("gemm"):
+                    if kind.startswith(("gemm", "gemv")):
                         agg["flops"] += 2 * m * N * K
             per_run.setdefault((m, p), []).append(rec)
     dominant = max(per_kind, key=lambda k: per_kind[k]["ms"])
@@ -681,8 +687,9 @@ def run_ours(args):
                   f"{N_SETS} weight sets rotated)")
     achieved = blk_bytes / (blk_ms * 1e-3) / 1e9
     traffic = TRAFFIC.get(dominant)
-    if traffic and traffic.get("src_sha") != _kernel_src_sha(
-            "decode" if dominant.startswith("decode") or dominant == "transcode" else "gemm"):
+    fam = ("decode" if dominant.startswith("decode") or dominant == "transcode"
+           else "gemv" if dominant.startswith("gemv") else "gemm")
+    if traffic and traffic.get("src_sha") != _kernel_src_sha(fam):
         traffic = None
     roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
@@ -701,7 +708,7 @@ def run_ours(args):
         def med(kind):
             xs = [r[kind] for r in recs if kind in r]
             return 1e3 * statistics.median(xs) if xs else None
-        pre, gemm = _run_kernels(p)
+        pre, gemm = _run_kernels(p, m)
         g = med(gemm) or 0.0
         pr = med(pre) if pre else 0.0
         pipelines[f"{p}/M{m}"] = {"preprocess_us": pr, "gemm_us": g, "total_us": pr + g,
@@ -812,7 +819,8 @@ def run_ours(args):
 def run_only(args):
     """Three launches of one kernel on the bench workload (first set of weights),
     for a profiler to capture (select by kernel name: decode_kernel<0|1|2> is
-    exponent / full / transcode, gemm_kernel<0|1|2> bf16 / exponent / palette).
+    exponent / full / transcode, gemm_kernel<0|1|2> bf16 / exponent / palette,
+    gemv_kernel<0|1|2, tokens> the matrix-vector kernels).
     The handle is uploaded without the load-time transcode unless the palette
     GEMM needs it (that launch comes first)."""
     import numpy as np
@@ -822,9 +830,12 @@ def run_only(args):
 
     w = synthdata.workload(args.workload)
     N, K = w.shape
-    h = uw.uw_encode(w, uw.default_opts(prepare_direct=1 if args.only == "gemm_palette" else 0))
+    direct = args.only in ("gemm_palette", "gemv_palette")
+    h = uw.uw_encode(w, uw.default_opts(prepare_direct=1 if direct else 0))
     out = torch.empty(2 * N * K, dtype=torch.uint8, device="cuda")
-    pipe = {"gemm_bf16": 1, "gemm_exp": 2, "gemm_palette": 4}.get(args.only)
+    pipe = {"gemm_bf16": 1, "gemm_exp": 2, "gemm_palette": 4,
+            "gemv_bf16": 1, "gemv_exp": 2, "gemv_palette": 4}.get(args.only)
+    gemv = args.only.startswith("gemv")
     if pipe:
         M = args.m
         X = torch.from_numpy(synthdata.activations(M, K, seed=11 + M).view(np.int16)).cuda()
@@ -838,6 +849,8 @@ def run_only(args):
             uw.uw_decode_exp(h, out)
         elif args.only == "transcode":
             uw.uw_transcode_palette(h, out)
+        elif gemv:  # the CUDA-core matrix-vector kernel (M <= 2)
+            uw.uw_gemm_ex(h, X, Y, M, uw.gemm_config(pipe, gemv=1), False)
         else:  # pipelines 1 and 2 run their decode first (select the GEMM by name)
             uw.uw_gemm(h, X, Y, M, pipe)
     torch.cuda.synchronize()

@@ -74,11 +74,11 @@ class uw_stats_t(C.Structure):
 class uw_gemm_config(C.Structure):
     _fields_ = [("pipeline", C.c_int32), ("tile_n", C.c_int32), ("stages", C.c_int32),
                 ("gemm_ctas", C.c_int32), ("decode_ctas", C.c_int32), ("halves", C.c_int32),
-                ("pair", C.c_int32), ("reserved", C.c_int32)]
+                ("pair", C.c_int32), ("gemv", C.c_int32)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k in ("pipeline", "tile_n", "stages", "gemm_ctas",
-                                               "decode_ctas", "halves", "pair")}
+                                               "decode_ctas", "halves", "pair", "gemv")}
 
 
 class uw_mlp_layer(C.Structure):
@@ -407,11 +407,14 @@ def uw_gemm_f32(h: Handle, X, Y, M: int, pipeline: int = UW_PIPE_AUTO) -> None:
 
 
 def gemm_config(pipeline: int, tile_n: int = 0, stages: int = 0, gemm_ctas: int = 0,
-                decode_ctas: int = 0, halves: int = 0, pair: int = 0) -> uw_gemm_config:
+                decode_ctas: int = 0, halves: int = 0, pair: int = 0,
+                gemv: int = 0) -> uw_gemm_config:
+    """A variant: gemv = 1 selects the CUDA-core matrix-vector kernel (M <= 2),
+    0 the tensor-core GEMM."""
     c = uw_gemm_config()
     c.pipeline, c.tile_n, c.stages = int(pipeline), int(tile_n), int(stages)
     c.gemm_ctas, c.decode_ctas, c.halves = int(gemm_ctas), int(decode_ctas), int(halves)
-    c.pair = int(pair)
+    c.pair, c.gemv = int(pair), int(gemv)
     return c
 
 
@@ -508,7 +511,7 @@ def uw_get_choice(h: Handle, M: int) -> dict:
 
 
 KERNEL_KINDS = ("decode_full", "decode_exp", "transcode", "gemm_bf16", "gemm_exp",
-                "gemm_palette", "splitk_fixup")
+                "gemm_palette", "splitk_fixup", "gemv_bf16", "gemv_exp", "gemv_palette")
 
 
 def uw_trace_enable(h: Handle, enable: bool = True) -> None:

@@ -25,8 +25,8 @@ COMMON = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibilit
 CU_FLAGS = ARCH + ["-lineinfo", "--expt-relaxed-constexpr", "-Xptxas", "-v", "-Wno-deprecated-gpu-targets"] + COMMON
 CPP_FLAGS = COMMON + ["-Wno-deprecated-gpu-targets"]
 
-SOURCES = ["encode.cpp", "bundle.cpp", "api.cu", "decode.cu", "gemm.cu", "autotune.cu", "noalloc.cu",
-           "mlp.cu"]
+SOURCES = ["encode.cpp", "bundle.cpp", "api.cu", "decode.cu", "gemm.cu", "gemv.cu", "autotune.cu",
+           "noalloc.cu", "mlp.cu"]
 
 
 def _headers() -> list:

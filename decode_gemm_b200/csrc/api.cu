@@ -181,8 +181,13 @@ uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
   return UW_OK;
 }
 
+// Whether a request runs on the matrix-vector kernel (uw_gemm_config.gemv = 1;
+// the autotuner tries it at M <= 2 and keeps it where it measures faster).
+bool use_gemv(const uw_gemm_config& c, int64_t M) { return c.gemv > 0 && M <= kGemvMaxM; }
+
 uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg) {
   if (!valid_pipeline(cfg.pipeline)) return UW_ERR_ARG;
+  if (cfg.gemv < 0 || cfg.gemv > 1) return UW_ERR_ARG;
   if (cfg.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) return UW_ERR_UNSUPPORTED;
   if (cfg.tile_n < 0 || cfg.tile_n > 256 || cfg.tile_n % 16) return UW_ERR_ARG;
   if (cfg.halves < 0 || cfg.halves > 2) return UW_ERR_ARG;
@@ -209,9 +214,53 @@ uw_status run_preprocess(uw_handle_s* h, int pipeline, void* out, int ctas, cuda
 
 // The GEMM of a pipeline on weights already preprocessed into `pre` (ignored
 // for pipeline 4), partial sums in `partials` (gemm_partials_bytes of the plan).
+// The matrix-vector kernel for (handle, pipeline) on weights already
+// preprocessed into `pre` (ignored for pipeline 4).
+uw_status run_gemv_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M, int pipeline,
+                      int out_f32, const void* pre, cudaStream_t s) {
+  if (M > kGemvMaxM) return UW_ERR_UNSUPPORTED;
+  GemmArgs a = base_gemm_args(h);
+  a.M = M;
+  a.X = X;
+  a.Y = Y;
+  a.out_f32 = out_f32;
+  switch (pipeline) {
+    case UW_PIPE_FULL:
+      a.mode = kGemmBf16;
+      a.W = static_cast<const uint16_t*>(pre);
+      break;
+    case UW_PIPE_EXP:
+      a.mode = kGemmExp;
+      a.E = static_cast<const uint8_t*>(pre);
+      break;
+    case UW_PIPE_PALETTE_RT:
+      a.mode = kGemmPalette;
+      a.I = static_cast<const uint8_t*>(pre);
+      break;
+    default:
+      a.mode = kGemmPalette;
+      a.I = h->d_pal_idx;
+      a.w1_resident = 1;
+      break;
+  }
+  if (!gemv_supported(a)) return UW_ERR_UNSUPPORTED;
+  LaunchHooks hooks;
+  hooks.ctx = h;
+  hooks.begin = hook_begin;
+  hooks.end = hook_end;
+  return map_cuda(launch_gemv(a, s, &hooks));
+}
+
+// The matrix-vector kernel serves (handle, M, variant).
+bool gemv_for(const uw_handle_s* h, const uw_gemm_config& cfg, int64_t M) {
+  (void)h;
+  return use_gemv(cfg, M);
+}
+
 uw_status run_gemm_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
                       const uw_gemm_config& cfg, int out_f32, const void* pre, float* partials,
                       size_t partials_bytes, cudaStream_t s) {
+  if (gemv_for(h, cfg, M)) return run_gemv_on(h, X, Y, M, cfg.pipeline, out_f32, pre, s);
   GemmArgs a;
   size_t need = 0, pre_b = 0;
   uw_status st = plan_gemm(h, X, Y, M, cfg, out_f32, &a, &need, &pre_b);
@@ -243,6 +292,20 @@ uw_status run_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
   }
   uw_status st = check_config(h, cfg);
   if (st != UW_OK) return st;
+  if (cfg.gemv > 0 && M > kGemvMaxM) return UW_ERR_UNSUPPORTED;
+  if (gemv_for(h, cfg, M)) {
+    // preprocessed weights (pipelines 1-3) in the workspace; no partial sums
+    const size_t pre_b = align_up(preprocess_bytes(h, cfg.pipeline), 256);
+    if (pre_b > 0 && (!h->ws || h->ws_bytes < pre_b)) return UW_ERR_WORKSPACE;
+    if (cfg.pipeline != UW_PIPE_PALETTE_DIRECT) {
+      const int mode = cfg.pipeline == UW_PIPE_FULL
+                           ? kDecodeFull
+                           : (cfg.pipeline == UW_PIPE_EXP ? kDecodeExp : kDecodePalette);
+      st = run_decode(h, mode, h->ws, cfg.decode_ctas, h->stream);
+      if (st != UW_OK) return st;
+    }
+    return run_gemv_on(h, X, Y, M, cfg.pipeline, out_f32, h->ws, h->stream);
+  }
   GemmArgs a;
   size_t need = 0, pre = 0;
   st = plan_gemm(h, X, Y, M, cfg, out_f32, &a, &need, &pre);

@@ -50,6 +50,18 @@ std::vector<uw_gemm_config> candidates(const uw_handle_s* h, int64_t M) {
   std::vector<uw_gemm_config> out;
   for (int p = UW_PIPE_FULL; p <= UW_PIPE_PALETTE_DIRECT; ++p) {
     if (p == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) continue;
+    if (M <= kGemvMaxM) {  // the matrix-vector kernel on the CUDA cores, if it fits
+      uw_gemm_config c;
+      std::memset(&c, 0, sizeof(c));
+      c.pipeline = p;
+      c.gemv = 1;
+      GemmArgs a;
+      a.M = M;
+      a.N = h->N;
+      a.K = h->K;
+      a.mode = p == UW_PIPE_FULL ? kGemmBf16 : (p == UW_PIPE_EXP ? kGemmExp : kGemmPalette);
+      if (gemv_supported(a)) out.push_back(c);
+    }
     for (int t : tiles)
       for (int st : {0, 4})
         for (int hv : {0, 1, 2}) {
@@ -77,6 +89,10 @@ std::vector<uw_gemm_config> candidates(const uw_handle_s* h, int64_t M) {
 
 bool fits(uw_handle_s* h, int64_t M, const uw_gemm_config& c) {
   if (check_config(h, c) != UW_OK) return false;
+  if (gemv_for(h, c, M)) {  // preprocessed weights only
+    const size_t need = preprocessed_bytes(h, c.pipeline);
+    return need == 0 || (h->ws && h->ws_bytes >= need);
+  }
   GemmArgs a;
   size_t need = 0, pre = 0;
   if (plan_gemm(h, nullptr, nullptr, M, c, 0, &a, &need, &pre) != UW_OK) return false;
@@ -335,9 +351,9 @@ uw_status uw_autotune(uw_handle_t* hs_in, int32_t n_handles, const int64_t* Ms, 
         std::fprintf(f,
                      "      {\"M\": %lld, \"pipeline\": %d, \"tile_n\": %d, \"stages\": %d, "
                      "\"gemm_ctas\": %d, \"decode_ctas\": %d, \"halves\": %d, \"pair\": %d, "
-                     "\"us\": %.2f}%s\n",
+                     "\"gemv\": %d, \"us\": %.2f}%s\n",
                      (long long)chosen[i][j].first, c.pipeline, c.tile_n, c.stages, c.gemm_ctas,
-                     c.decode_ctas, c.halves, c.pair, 1e3 * chosen_ms[i][j],
+                     c.decode_ctas, c.halves, c.pair, c.gemv, 1e3 * chosen_ms[i][j],
                      j + 1 < chosen[i].size() ? "," : "");
       }
       std::fprintf(f, "    ]}%s\n", i + 1 < hs.size() ? "," : "");
@@ -374,7 +390,7 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
     const JVal* ch = hv.get("choices");
     if (!ch || ch->kind != JVal::Arr) return UW_ERR_FORMAT;
     for (const JVal& c : ch->arr) {
-      int64_t M = 0, pl = 0, tn = 0, sg = 0, gc = 0, dc = 0, hv2 = 0, pr = 0;
+      int64_t M = 0, pl = 0, tn = 0, sg = 0, gc = 0, dc = 0, hv2 = 0, pr = 0, gv = 0;
       if (c.kind != JVal::Obj || !num_field(c, "M", &M) || !num_field(c, "pipeline", &pl))
         return UW_ERR_FORMAT;
       num_field(c, "tile_n", &tn);
@@ -383,6 +399,7 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
       num_field(c, "decode_ctas", &dc);
       num_field(c, "halves", &hv2);
       num_field(c, "pair", &pr);
+      num_field(c, "gemv", &gv);
       uw_gemm_config cfg;
       std::memset(&cfg, 0, sizeof(cfg));
       cfg.pipeline = (int32_t)pl;
@@ -392,6 +409,7 @@ uw_status uw_load_profile(uw_handle_t* hs, int32_t n_handles, const char* profil
       cfg.decode_ctas = (int32_t)dc;
       cfg.halves = (int32_t)hv2;
       cfg.pair = (int32_t)pr;
+      cfg.gemv = (int32_t)gv;
       if (M <= 0 || check_config(hs[i], cfg) != UW_OK) return UW_ERR_FORMAT;
       parsed[i][M] = cfg;
     }

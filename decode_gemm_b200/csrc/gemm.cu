@@ -1157,15 +1157,6 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const v
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-uint64_t wait_limit_ns() {
-  static uint64_t ns = [] {
-    const char* s = std::getenv("UW_WAIT_LIMIT_MS");
-    const long long ms = s ? std::atoll(s) : 2000;
-    return (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
-  }();
-  return ns;
-}
-
 int mma_warps_for(int tile_n) { return tile_n <= 128 ? 2 : 1; }
 
 // TMEM columns: two accumulator sets, then (TMEM path) the W slots.

@@ -58,6 +58,8 @@ DecodeArgs decode_args(const uw_handle_s* h);
 // Shared by the C ABI, the autotuner and the MLP driver (api.cu).
 uw_gemm_config choose_variant(const uw_handle_s* h, int64_t M);
 uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg);
+bool use_gemv(const uw_gemm_config& c, int64_t M);
+bool gemv_for(const uw_handle_s* h, const uw_gemm_config& cfg, int64_t M);
 size_t preprocessed_bytes(const uw_handle_s* h, int pipeline);
 uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
                     const uw_gemm_config& cfg, int out_f32, GemmArgs* ga, size_t* ws_need,

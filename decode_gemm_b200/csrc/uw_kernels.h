@@ -4,8 +4,20 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 
 namespace uw {
+
+// Limit of every bounded wait inside a kernel (UW_WAIT_LIMIT_MS, default 2 s);
+// a wait that runs out sets the timeout status and the kernel returns.
+inline uint64_t wait_limit_ns() {
+  static const uint64_t ns = [] {
+    const char* s = std::getenv("UW_WAIT_LIMIT_MS");
+    const long long ms = s ? std::atoll(s) : 2000;
+    return (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
+  }();
+  return ns;
+}
 
 enum DecodeMode { kDecodeExp = 0, kDecodeFull = 1, kDecodePalette = 2 };
 
@@ -103,6 +115,14 @@ struct LaunchHooks {
   int (*begin)(void* ctx, int kind) = nullptr;
   void (*end)(void* ctx, int slot) = nullptr;
 };
+
+// Matrix-vector kernel on the CUDA cores for M <= kGemvMaxM tokens (gemv.cu):
+// the same arguments as the GEMM (mode, M, N, K, X, the weight arrays of the
+// mode, escape data, palette, Y, out_f32, w1_resident); no partial sums, no
+// workspace of its own.  Traced as kinds 7 (BF16), 8 (exponent), 9 (palette).
+constexpr int kGemvMaxM = 2;
+bool gemv_supported(const GemmArgs& a);
+cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const LaunchHooks* hooks = nullptr);
 
 // Fill in automatic tile_n / stages / ctas; returns false for unsupported shapes.
 bool gemm_resolve(GemmArgs* a);

@@ -153,7 +153,10 @@ typedef struct uw_gemm_config {
                             each CTA loading its 128 rows and half of the tokens
                             (256-token tiles; one half per unit); 0: one CTA per
                             tile.  Other pipelines: UW_ERR_UNSUPPORTED              */
-  int32_t reserved;
+  int32_t gemv;          /* 1: the matrix-vector kernel on the CUDA cores, M <= 2 only
+                            (each weight rebuilt in registers and multiplied in FP32,
+                            no tensor cores; UW_ERR_UNSUPPORTED above M = 2); 0: the
+                            tensor-core GEMM.  The autotuner tries 1 at M <= 2      */
 } uw_gemm_config;
 
 typedef struct uw_host_s* uw_host_t;       /* host-side encoded matrix         */
@@ -320,7 +323,8 @@ UW_API uw_status uw_get_choice(uw_handle_t h, int64_t M, uw_gemm_config* cfg);
 typedef enum uw_kernel_kind {
   UW_KERNEL_DECODE_FULL = 0, UW_KERNEL_DECODE_EXP = 1, UW_KERNEL_TRANSCODE = 2,
   UW_KERNEL_GEMM_BF16 = 3, UW_KERNEL_GEMM_EXP = 4, UW_KERNEL_GEMM_PALETTE = 5,
-  UW_KERNEL_SPLITK_FIXUP = 6  /* reserved: split tiles are summed inside the GEMM */
+  UW_KERNEL_SPLITK_FIXUP = 6,  /* reserved: split tiles are summed inside the GEMM */
+  UW_KERNEL_GEMV_BF16 = 7, UW_KERNEL_GEMV_EXP = 8, UW_KERNEL_GEMV_PALETTE = 9
 } uw_kernel_kind;
 UW_API uw_status uw_trace_enable(uw_handle_t h, int32_t enable);
 UW_API uw_status uw_trace_read(uw_handle_t h, int32_t* kinds, float* ms, int32_t capacity,

@@ -468,3 +468,93 @@ def test_back_to_back_chain_on_one_stream(uw, pipe):
     for h in hs:
         assert uw.uw_last_device_status(h) == uw.UW_OK
         h.free()
+
+
+# ---------------------------------------------------------------- M <= 2 ----
+def _finite_specials(rows, cols, seed):
+    """The BF16 corner cases that keep a matmul finite: +-0, subnormals, the
+    smallest normal (Inf, NaN and the largest normals replaced by 1.0)."""
+    w = synthdata.special_values(rows, cols, seed).copy()
+    w[(w & 0x7F80) >= 0x7F00] = 0x3F80
+    return w
+
+
+GEMV_CASES = {
+    "mat1024": lambda: synthdata.workload("mat1024"),
+    "ragged_k1536": lambda: synthdata.normal(1000, 1536, 0.02, seed=170),   # a half segment
+    "heavy_tail": lambda: synthdata.student_t(600, 3584, 3.0, 0.015, seed=171),
+    "zeros_subnormals": lambda: _finite_specials(96, 640, seed=172),
+    "not_a_run": lambda: synthdata.exponent_pattern(130, 2048, [100, 104, 108, 112, 113, 114, 115,
+                                                                116, 117, 118, 119, 120, 121, 122,
+                                                                126, 130, 7], seed=173),
+}
+
+
+@pytest.mark.parametrize("name", list(GEMV_CASES))
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_matches_fp64(uw, name, M):
+    """The CUDA-core matrix-vector kernel (M <= 2, uw_gemm_config.gemv = 1) of
+    every pipeline against the FP64 oracle, FP32 and BF16 outputs; the
+    reconstructive pipelines give bitwise the same result (same rebuilt
+    weights, same summation order); escape rows, a palette that is not one run
+    of exponents, a K that ends inside a 1024-weight segment."""
+    w = GEMV_CASES[name]()
+    x = synthdata.activations(M, w.shape[1], seed=174 + M)
+    h = _upload(uw, w, chunk=256)
+    _workspace(uw, h, M)
+    ref = oracle.gemm_fp64(x, w)
+    bound = oracle.abs_product_sum(x, w)
+    outs = {}
+    for p in PIPES:
+        y = _gemm(uw, h, x, p, gemv=1)
+        ok, worst = oracle.within_tolerance(y, ref, bound)
+        assert ok, (p, worst)
+        outs[p] = y
+        yb = _gemm(uw, h, x, p, out_f32=False, gemv=1)
+        assert oracle.within_tolerance(yb, ref, bound, bf16_output=True)[0], p
+    assert np.array_equal(outs["exp"], outs["palette_rt"])
+    assert np.array_equal(outs["exp"], outs["palette_direct"])
+    # the tensor-core GEMM (the default) agrees within tolerance
+    yt = _gemm(uw, h, x, "palette_direct")
+    assert oracle.within_tolerance(yt, ref, bound)[0]
+    h.free()
+
+
+def test_gemv_limits_and_trace(uw):
+    import ctypes as C
+    import torch
+    w = synthdata.normal(256, 512, 0.02, seed=176)
+    h = uw.uw_encode(w)
+    X = torch.zeros((3, 512), dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros((3, 256), dtype=torch.float32, device="cuda")
+    c = uw.gemm_config(4, gemv=1)
+    assert uw.lib.uw_gemm_ex(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 3,
+                             C.byref(c), 1) == uw.UW_ERR_UNSUPPORTED
+    for bad in (2, -1):
+        c = uw.gemm_config(4, gemv=bad)
+        assert uw.lib.uw_gemm_ex(h.ptr, C.c_void_p(X.data_ptr()), C.c_void_p(Y.data_ptr()), 1,
+                                 C.byref(c), 1) == uw.UW_ERR_ARG
+    # pipeline 4 at M = 1 needs no workspace on this path; traced as the matrix-vector kernel
+    uw.uw_trace_enable(h, True)
+    uw.uw_gemm_ex(h, X, Y, 1, uw.gemm_config(4, gemv=1), True)
+    kinds = [k for k, _ in uw.uw_trace_read(h)]
+    assert kinds == ["gemv_palette"]
+    assert uw.uw_last_device_status(h) == uw.UW_OK
+    h.free()
+
+
+@pytest.mark.parametrize("name,M", [("gate_14336x4096", 1), ("down70b_8192x28672", 2)])
+def test_gemv_full_size(uw, name, M):
+    """Full-size shapes on the matrix-vector kernel: every output row against
+    FP64 (gate, M = 1) and the 70B down shape (K = 28672, 28 segments)."""
+    w = synthdata.workload(name)
+    x = synthdata.activation_for(name, M)
+    h = _upload(uw, w, chunk=256)
+    _workspace(uw, h, M)
+    ref = oracle.gemm_fp64(x, w)
+    bound = oracle.abs_product_sum(x, w)
+    for p in PIPES:
+        y = _gemm(uw, h, x, p, gemv=1)
+        ok, worst = oracle.within_tolerance(y, ref, bound)
+        assert ok, (p, worst)
+    h.free()
