@@ -116,6 +116,7 @@ _SIGS = {
     "uw_alloc_workspace": ([_vp, _sz], C.c_int),
     "uw_decode_full": ([_vp, _vp], C.c_int),
     "uw_decode_exp": ([_vp, _vp], C.c_int),
+    "uw_decode_rows": ([_vp, _vp, _i64, _vp], C.c_int),
     "uw_transcode_palette": ([_vp, _vp], C.c_int),
     "uw_gemm": ([_vp, _vp, _vp, _i64, C.c_int], C.c_int),
     "uw_gemm_f32": ([_vp, _vp, _vp, _i64, C.c_int], C.c_int),
@@ -395,6 +396,13 @@ def uw_decode_exp(h: Handle, e_out) -> None:
 
 def uw_transcode_palette(h: Handle, idx_out) -> None:
     _check(lib.uw_transcode_palette(h.ptr, _vp(_dptr(idx_out))), "uw_transcode_palette")
+
+
+def uw_decode_rows(h: Handle, rows, out) -> None:
+    """BF16 rows `rows` (device int64 tensor) of the encoded matrix into `out`
+    ([len(rows), K] on the device): an embedding lookup on compressed weights."""
+    _check(lib.uw_decode_rows(h.ptr, _vp(_dptr(rows)), int(rows.numel()), _vp(_dptr(out))),
+           "uw_decode_rows")
 
 
 def uw_gemm(h: Handle, X, Y, M: int, pipeline: int = UW_PIPE_AUTO) -> None:

@@ -598,6 +598,29 @@ uw_status uw_transcode_palette(uw_handle_t h, uint8_t* idx_dev) {
   return run_decode(h, kDecodePalette, idx_dev, 0, h->stream);
 }
 
+uw_status uw_decode_rows(uw_handle_t h, const int64_t* rows_dev, int64_t n_rows,
+                         uint16_t* w_dev) {
+  if (!h) return UW_ERR_ARG;
+  if (n_rows < 0) return UW_ERR_SHAPE;
+  if (n_rows == 0) return UW_OK;
+  if (!rows_dev || (reinterpret_cast<uintptr_t>(rows_dev) & 7)) return UW_ERR_ARG;
+  uw_status st = check_out_ptr(w_dev);
+  if (st != UW_OK) return st;
+  if (h->K % h->chunk_syms) return UW_ERR_UNSUPPORTED;  // rows must be whole chunks
+  DeviceGuard g(h->device);
+  DecodeArgs a = decode_args(h);
+  a.cpr = (int32_t)(h->K / h->chunk_syms);
+  a.rows = rows_dev;
+  a.gather_rows = n_rows;
+  a.matrix_rows = h->N;
+  a.n_chunks = n_rows * a.cpr;
+  a.total_syms = n_rows * h->K;
+  const int slot = trace_begin(h, UW_KERNEL_DECODE_FULL);
+  const cudaError_t e = launch_decode(kDecodeFull, a, w_dev, 0, h->stream);
+  trace_end(h, slot);
+  return map_cuda(e);
+}
+
 uw_status uw_gemm_ex(uw_handle_t h, const uint16_t* X_dev, void* Y_dev, int64_t M,
                      const uw_gemm_config* cfg, int32_t out_f32) {
   if (!h || !cfg) return UW_ERR_ARG;

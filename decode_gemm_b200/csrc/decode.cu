@@ -184,7 +184,10 @@ __device__ __forceinline__ void pack(Packer& pk, uint32_t e, uint32_t c4) {
       : "memory");
 }
 
-template <int MODE>
+// GATHER (full decode only): the launch's chunks are the chunks of the rows
+// a.rows[] (see DecodeArgs); a lane reads its chunk's stream and S at the real
+// chunk and writes its output at the launch's (virtual) chunk.
+template <int MODE, bool GATHER>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     decode_kernel(const DecodeArgs a, void* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -225,10 +228,25 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     uint32_t start = 0, end = 0;
     int nsyms = 0;
     bool bad = false;
-    if (live) {
-      start = __ldg(a.chunk_off + c);
-      end = __ldg(a.chunk_off + c + 1);
-      const int64_t left = a.total_syms - c * cs;
+    int64_t cr = c;  // the chunk of the matrix this lane decodes
+    if (GATHER && !waited) {  // the row ids are the caller's: after the kernel before
+      pdl_wait();
+      waited = true;
+    }
+    if (GATHER && live) {
+      const int64_t v = c / a.cpr;
+      const int64_t row = a.rows[v];
+      if (row < 0 || row >= a.matrix_rows) {  // not a row of the matrix: nothing is read
+        bad = true;
+        cr = -1;
+      } else {
+        cr = row * a.cpr + (c - v * a.cpr);
+      }
+    }
+    if (live && cr >= 0) {
+      start = __ldg(a.chunk_off + cr);
+      end = __ldg(a.chunk_off + cr + 1);
+      const int64_t left = GATHER ? cs : a.total_syms - c * cs;
       nsyms = (int)(left < cs ? left : cs);
       if (start > stream_bits) {  // corrupt offset: nothing is read
         bad = true;
@@ -236,8 +254,9 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         nsyms = 0;
       }
     }
+    if (cr < 0) cr = 0;  // (a rejected row reads nothing; S accesses stay in bounds)
     // the stream of this warp's next group: into L2 while this one decodes
-    {
+    if (!GATHER) {
       const int64_t cn = c + grid_warps * 32;
       if (cn < a.n_chunks) {
         const uint32_t nb = __ldg(a.chunk_off + cn) >> 3;
@@ -322,7 +341,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
       pk.sp = st_addr;
       if (MODE == kDecodeFull && r < my_rounds) {
         // this round's sign+mantissa bytes into L2 while the round decodes
-        const uint8_t* sp8 = a.sm + c * cs + (int64_t)r * kRoundSyms;
+        const uint8_t* sp8 = a.sm + cr * cs + (int64_t)r * kRoundSyms;
         asm volatile("prefetch.global.L2 [%0];" :: "l"(sp8));
       }
       if (r < my_rounds - 1) {
@@ -381,8 +400,14 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             uint2 sv[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const int64_t o = (int64_t)(16 * h + 2 * i + jh) * cs;
-              sv[i] = ld_v2_if(sbase + o, in_chunk && o + rel0 + 8 * m < grp_syms_left);
+              const int j = 16 * h + 2 * i + jh;
+              const int64_t o = (int64_t)j * cs;
+              // S of chunk j: consecutive in the matrix, or (gather) at its real chunk
+              const uint8_t* sp =
+                  GATHER ? a.sm + (int64_t)(uint32_t)__shfl_sync(0xffffffffu, (uint32_t)cr, j) * cs +
+                               rel0 + 8 * m
+                         : sbase + o;
+              sv[i] = ld_v2_if(sp, in_chunk && o + rel0 + 8 * m < grp_syms_left);
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -450,7 +475,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             if (MODE == kDecodeExp) {
               static_cast<uint8_t*>(out)[o] = (uint8_t)(x & 0xFFu);
             } else {
-              const uint32_t s = a.sm[o];
+              const uint32_t s = a.sm[cr * cs + pos];
               static_cast<uint16_t*>(out)[o] =
                   (uint16_t)(((s & 0x80u) << 8) | ((x & 0xFFu) << 7) | (s & 0x7Fu));
             }
@@ -476,7 +501,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         if (MODE == kDecodeExp) {
           static_cast<uint8_t*>(out)[base + i] = (uint8_t)ex;
         } else {
-          const uint32_t s = a.sm[base + i];
+          const uint32_t s = a.sm[cr * cs + i];
           static_cast<uint16_t*>(out)[base + i] =
               (uint16_t)(((s & 0x80u) << 8) | (ex << 7) | (s & 0x7Fu));
         }
@@ -549,16 +574,25 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cu
   const dim3 block(32 * warps);
   switch (mode) {
     case kDecodeExp:
-      e = set_attrs(decode_kernel<kDecodeExp>, smem);
-      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodeExp>, grid, block, smem, s, a, out);
+      if (a.rows) return cudaErrorInvalidValue;
+      e = set_attrs(decode_kernel<kDecodeExp, false>, smem);
+      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodeExp, false>, grid, block, smem, s, a, out);
       break;
     case kDecodeFull:
-      e = set_attrs(decode_kernel<kDecodeFull>, smem);
-      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodeFull>, grid, block, smem, s, a, out);
+      if (a.rows) {
+        e = set_attrs(decode_kernel<kDecodeFull, true>, smem);
+        if (e == cudaSuccess)
+          e = launch_pdl(decode_kernel<kDecodeFull, true>, grid, block, smem, s, a, out);
+      } else {
+        e = set_attrs(decode_kernel<kDecodeFull, false>, smem);
+        if (e == cudaSuccess)
+          e = launch_pdl(decode_kernel<kDecodeFull, false>, grid, block, smem, s, a, out);
+      }
       break;
     case kDecodePalette:
-      e = set_attrs(decode_kernel<kDecodePalette>, smem);
-      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodePalette>, grid, block, smem, s, a, out);
+      if (a.rows) return cudaErrorInvalidValue;
+      e = set_attrs(decode_kernel<kDecodePalette, false>, smem);
+      if (e == cudaSuccess) e = launch_pdl(decode_kernel<kDecodePalette, false>, grid, block, smem, s, a, out);
       break;
     default:
       return cudaErrorInvalidValue;

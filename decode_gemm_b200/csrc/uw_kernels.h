@@ -45,6 +45,14 @@ struct DecodeArgs {
   int32_t chunk_syms;
   int32_t kb_per_row;         // K / 64
   int32_t esc_nw;             // escape-bitmap words per K block: 4*ceil(N/128)
+  // Row gather (full decode only): decode the rows rows[0 .. gather_rows-1] of
+  // the matrix into consecutive output rows.  Chunk v of the launch (n_chunks =
+  // gather_rows * cpr, total_syms = gather_rows * K) is chunk v % cpr of row
+  // rows[v / cpr]; needs K % chunk_syms == 0 (cpr = K / chunk_syms).
+  const int64_t* rows = nullptr;
+  int64_t gather_rows = 0;
+  int64_t matrix_rows = 0;    // N
+  int32_t cpr = 0;
 };
 
 // Decode/transcode every chunk into `out` (layout per mode: BF16 [N*K],

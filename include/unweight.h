@@ -241,6 +241,19 @@ UW_API uw_status uw_alloc_workspace(uw_handle_t h, size_t bytes);
 /* Full Huffman decode ("Four ways...", pipeline 1 preprocessing): writes the
  * N*K BF16 weights to w_dev (caller-owned, 16-byte aligned).  Bit-exact. */
 UW_API uw_status uw_decode_full(uw_handle_t h, uint16_t* w_dev);
+/* Row gather on compressed weights: the BF16 rows rows_dev[0 .. n_rows-1] of
+ * W (an embedding lookup: token ids into a [vocab, dim] table) decoded into
+ * w_dev, [n_rows, K] row-major, row i of the output = row rows_dev[i] of W.
+ * Only the requested rows' chunks are decoded (the same table-driven decoder
+ * as uw_decode_full).  "Exponents are surprisingly predictable" and the
+ * closing remarks of *Unweight*: the format is not specific to MLP weights.
+ * rows_dev: device int64 array, 8-byte aligned; ids may repeat; an id outside
+ * [0, N) leaves its output row unspecified and makes uw_last_device_status
+ * report UW_ERR_DEVICE.  w_dev 16-byte aligned.  Needs K to be a multiple of
+ * the encoding's chunk_syms (UW_ERR_UNSUPPORTED otherwise).  n_rows == 0
+ * returns UW_OK and launches nothing. */
+UW_API uw_status uw_decode_rows(uw_handle_t h, const int64_t* rows_dev, int64_t n_rows,
+                                uint16_t* w_dev);
 /* Exponent-only decode (pipeline 2 preprocessing): N*K exponent bytes to e_dev
  * (16-byte aligned), row-major. */
 UW_API uw_status uw_decode_exp(uw_handle_t h, uint8_t* e_dev);

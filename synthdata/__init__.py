@@ -110,6 +110,15 @@ WORKLOADS = {
                                seed_x=52, Ms=(1, 4096)),
     "down70b_8192x28672": dict(N=8192, K=28672, kind="student_t", std=0.015, nu=3.0, seed_w=51,
                                seed_x=53, Ms=(1, 4096)),
+    # Llama-3.1-8B attention projections (q/o 4096x4096, k/v 1024x4096 with
+    # grouped-query attention) and a vocabulary-sized embedding table
+    # (128256 x 4096 in the model; a 32768-row slice here), N(0, 0.02)
+    "attn_q_4096x4096": dict(N=4096, K=4096, kind="normal", std=0.02, seed_w=60, seed_x=61,
+                             Ms=(1, 64, 1024)),
+    "attn_kv_1024x4096": dict(N=1024, K=4096, kind="normal", std=0.02, seed_w=62, seed_x=63,
+                              Ms=(1, 64, 1024)),
+    "embed_32768x4096": dict(N=32768, K=4096, kind="normal", std=0.02, seed_w=64, seed_x=65,
+                             Ms=(1, 64)),
 }
 
 

@@ -196,3 +196,78 @@ def test_bundle_load_to_device(uw, tmp_path):
                                         oracle.gemm_fp64(x, w), oracle.abs_product_sum(x, w))
     assert ok, worst
     h.free()
+
+
+# ------------------------------------------------- rows of an embedding table ----
+@pytest.mark.parametrize("name,chunk", [("normal", 256), ("student_t", 128), ("special", 64),
+                                        ("wide_rows", 1024)])
+def test_decode_rows_bit_exact(uw, name, chunk):
+    """uw_decode_rows (an embedding lookup on compressed weights): the requested
+    rows, repeats and the first and last row included, bit-exact."""
+    import torch
+    w = {"normal": lambda: synthdata.normal(2000, 1024, 0.02, seed=180),
+         "student_t": lambda: synthdata.student_t(777, 512, 3.0, 0.015, seed=181),
+         "special": lambda: synthdata.special_values(300, 640, seed=182),
+         "wide_rows": lambda: synthdata.normal(96, 4096, 0.02, seed=183)}[name]()
+    n, k = w.shape
+    h = uw.uw_encode(w, uw.default_opts(chunk_syms=chunk, prepare_direct=0))
+    rng = np.random.default_rng(184)
+    for count in (1, 5, 33, 300):
+        ids = rng.integers(0, n, size=count)
+        ids[0] = n - 1
+        if count > 1:
+            ids[1] = 0
+            ids[-1] = ids[0]  # a repeat
+        rows = torch.from_numpy(ids.astype(np.int64)).cuda()
+        out = _dev_empty(2 * count * k)
+        uw.uw_decode_rows(h, rows, out)
+        torch.cuda.synchronize()
+        assert uw.uw_last_device_status(h) == uw.UW_OK
+        got = out[: 2 * count * k].cpu().numpy().view(np.uint16).reshape(count, k)
+        assert np.array_equal(got, w[ids])
+    h.free()
+
+
+def test_decode_rows_embedding_table_slice(uw):
+    """A 32768 x 4096 slice of a vocabulary-sized embedding table: 64 token ids."""
+    import torch
+    w = synthdata.workload("embed_32768x4096")
+    h = uw.uw_encode(w, uw.default_opts(prepare_direct=0))
+    ids = np.random.default_rng(185).integers(0, w.shape[0], size=64)
+    rows = torch.from_numpy(ids.astype(np.int64)).cuda()
+    out = _dev_empty(2 * 64 * w.shape[1])
+    uw.uw_decode_rows(h, rows, out)
+    torch.cuda.synchronize()
+    assert uw.uw_last_device_status(h) == uw.UW_OK
+    got = out[: 2 * 64 * w.shape[1]].cpu().numpy().view(np.uint16).reshape(64, -1)
+    assert np.array_equal(got, w[ids])
+    h.free()
+
+
+def test_decode_rows_errors(uw):
+    import ctypes as C
+    import torch
+    w = synthdata.normal(64, 320, 0.02, seed=186)  # K = 320: not a multiple of 256
+    h = uw.uw_encode(w, uw.default_opts(chunk_syms=256, prepare_direct=0))
+    rows = torch.zeros(4, dtype=torch.int64, device="cuda")
+    out = _dev_empty(2 * 4 * 320)
+    rp, op = C.c_void_p(rows.data_ptr()), C.c_void_p(out.data_ptr())
+    assert uw.lib.uw_decode_rows(h.ptr, rp, 4, op) == uw.UW_ERR_UNSUPPORTED
+    h.free()
+    h = uw.uw_encode(w, uw.default_opts(chunk_syms=64, prepare_direct=0))
+    assert uw.lib.uw_decode_rows(h.ptr, rp, 0, op) == uw.UW_OK
+    assert uw.lib.uw_decode_rows(h.ptr, rp, -1, op) == uw.UW_ERR_SHAPE
+    assert uw.lib.uw_decode_rows(h.ptr, None, 4, op) == uw.UW_ERR_ARG
+    assert uw.lib.uw_decode_rows(h.ptr, C.c_void_p(rows.data_ptr() + 4), 3, op) == uw.UW_ERR_ARG
+    assert uw.lib.uw_decode_rows(h.ptr, rp, 4, C.c_void_p(out.data_ptr() + 2)) == uw.UW_ERR_ARG
+    # ids outside [0, N): the call returns, the device status reports it
+    bad = torch.tensor([3, 64, -1, 5], dtype=torch.int64, device="cuda")
+    assert uw.lib.uw_decode_rows(h.ptr, C.c_void_p(bad.data_ptr()), 4, op) == uw.UW_OK
+    assert uw.uw_last_device_status(h) == uw.UW_ERR_DEVICE
+    good = torch.tensor([3, 63], dtype=torch.int64, device="cuda")
+    uw.uw_decode_rows(h, good, out)
+    torch.cuda.synchronize()
+    assert uw.uw_last_device_status(h) == uw.UW_OK
+    got = out[: 2 * 2 * 320].cpu().numpy().view(np.uint16).reshape(2, 320)
+    assert np.array_equal(got, w[[3, 63]])
+    h.free()

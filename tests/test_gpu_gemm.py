@@ -558,3 +558,20 @@ def test_gemv_full_size(uw, name, M):
         ok, worst = oracle.within_tolerance(y, ref, bound)
         assert ok, (p, worst)
     h.free()
+
+
+# ------------------------------------------------- attention-shaped weights ----
+@pytest.mark.parametrize("name", ["attn_q_4096x4096", "attn_kv_1024x4096"])
+@pytest.mark.parametrize("M", [1, 64, 1024])
+def test_attention_projections(uw, name, M):
+    """The format on Llama-3.1-8B attention projections (q/o 4096x4096, k/v
+    1024x4096): every pipeline against FP64 (sampled token rows at M = 1024),
+    the reconstructive ones bitwise equal."""
+    w = synthdata.workload(name)
+    x = synthdata.activation_for(name, M)
+    h = _upload(uw, w, chunk=256)
+    _workspace(uw, h, M)
+    outs = _sampled_rows_check(uw, h, w, x, M, seed=190 + M, n_rows=M if M <= 64 else 24)
+    assert np.array_equal(outs["exp"], outs["palette_rt"])
+    assert np.array_equal(outs["exp"], outs["palette_direct"])
+    h.free()
