@@ -749,25 +749,60 @@ def run_ours(args):
     # ---- the metric's large-M matmuls (gate and down shapes)
     gemm_large = None if args.no_large_m else _large_m_block(uw, torch, stream, peaks)
 
-    # ---- end to end through the public call with host buffers
+    # ---- end to end through the public call with host buffers: every step
+    # copies its X in from pinned host memory and its Y out to pinned host
+    # memory.  The copies run on a copy stream, double-buffered, so step s's
+    # Y copy and step s+1's X copy overlap step s+1's and step s's compute; the
+    # timed region ends when the last step's Y has reached the host.
     Xh = {m: X[m].cpu().pin_memory() for m in Ms}
-    Yh = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in Y.items()}
+    Yh = [{k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in Y.items()}
+          for _ in range(2)]
     h2d = sum(x.numel() * 2 for x in Xh.values())
-    d2h = sum(y.numel() * 2 for y in Yh.values())
+    d2h = sum(y.numel() * 2 for y in Yh[0].values())
+    Xb = [X, {m: torch.empty_like(v) for m, v in X.items()}]
+    Yb = [Y, {k: torch.empty_like(v) for k, v in Y.items()}]
+    copy = torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    x_ready, x_free, y_done, y_free = ([ev(), ev()] for _ in range(4))
+    start = ev()
+
+    def step_io(run0, Xd, Yd):
+        for j, (m, p) in enumerate(runs):
+            h = handles[(run0 + j) % N_SETS]
+            uw.uw_gemm(h, Xd[m], Yd[(m, p)], m, uw.PIPELINES[p])
+        return run0 + len(runs)
+
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
+    start.record(stream)
+    copy.wait_event(start)
     run_e = run0
     e2e_bytes = 0
-    for _ in range(args.steps):
-        for m in Ms:
-            X[m].copy_(Xh[m], non_blocking=True)
+    for s_i in range(args.steps):
+        b = s_i % 2
+        with torch.cuda.stream(copy):
+            if s_i >= 2:
+                copy.wait_event(x_free[b])  # compute two steps ago is done with Xb[b]
+            for m in Ms:
+                Xb[b][m].copy_(Xh[m], non_blocking=True)
+            x_ready[b].record(copy)
+        stream.wait_event(x_ready[b])
+        if s_i >= 2:
+            stream.wait_event(y_free[b])  # Yb[b] from two steps ago is on the host
         e2e_bytes += step_bytes(run_e)
-        run_e = step(run_e)
-        for k in Y:
-            Yh[k].copy_(Y[k], non_blocking=True)
+        run_e = step_io(run_e, Xb[b], Yb[b])
+        x_free[b].record(stream)
+        y_done[b].record(stream)
+        with torch.cuda.stream(copy):
+            copy.wait_event(y_done[b])
+            for k in Y:
+                Yh[b][k].copy_(Yb[b][k], non_blocking=True)
+            y_free[b].record(copy)
+    for b in range(min(2, args.steps)):
+        stream.wait_event(y_free[b])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
