@@ -60,15 +60,15 @@ def _layers(uw, n_layers, pipes):
     return layers, weights
 
 
-def _load_pipelines(uw, layers, pipes, M, gemm_ctas=0):
-    """Pin each projection's pipeline for M through a profile file."""
+def _load_pipelines(uw, layers, pipes, M, gemm_ctas=0, gemv=0):
+    """Pin each projection's pipeline (and matmul kernel) for M through a profile file."""
     flat = [h for trio in layers for h in trio]
     prof = {"version": 1, "handles": []}
     for (trio, ps) in zip(layers, pipes):
         for h, p in zip(trio, ps):
             prof["handles"].append({"N": h.N, "K": h.K, "choices": [
                 {"M": M, "pipeline": p, "tile_n": 0, "stages": 0, "gemm_ctas": gemm_ctas,
-                 "decode_ctas": 0}]})
+                 "decode_ctas": 0, "gemv": gemv}]})
     with tempfile.NamedTemporaryFile("w", suffix=".json", delete=False) as f:
         json.dump(prof, f)
         path = f.name
@@ -142,10 +142,11 @@ SPLITS = {
     "overlap_decode4": dict(overlap=True, decode_ctas=4),
     "overlap_decode4_gemm100": dict(overlap=True, decode_ctas=4, gemm_ctas=100),
     "serial_gemm60": dict(overlap=False, gemm_ctas=60),
+    "overlap_matvec": dict(overlap=True),  # every projection on the matrix-vector kernel
 }
 
 
-@pytest.mark.parametrize("M", [1, 24])
+@pytest.mark.parametrize("M", [1, 2, 24])
 @pytest.mark.parametrize("split", list(SPLITS))
 def test_mlp_stack_projections_against_fp64(uw, M, split):
     """Every projection of a 3-layer stack run by uw_mlp_forward (hard and easy
@@ -154,8 +155,11 @@ def test_mlp_stack_projections_against_fp64(uw, M, split):
     oracle given the GPU's own g and u (*Unweight*, "Sharing the GPU between
     decode and compute")."""
     import torch
+    gemv = 1 if split == "overlap_matvec" else 0
+    if gemv and M > 2:
+        pytest.skip("the matrix-vector kernel serves M <= 2")
     layers, weights = _layers(uw, 3, PIPES)
-    _load_pipelines(uw, layers, PIPES, M)
+    _load_pipelines(uw, layers, PIPES, M, gemv=gemv)
     x = synthdata.activations(M, D, seed=160 + M)
     X = torch.from_numpy(x.view(np.int16)).cuda()
     side = torch.cuda.Stream()
