@@ -231,7 +231,7 @@ def test_down70b_shape_sampled(uw, down70b, M):
     assert h.stats()["n_escape_rows"] > 0
     x = synthdata.activation_for("down70b_8192x28672", M)
     _workspace(uw, h, M)
-    outs = _sampled_rows_check(uw, h, w, x, M, seed=71 + M, n_rows=8)
+    outs = _sampled_rows_check(uw, h, w, x, M, seed=71 + M, n_rows=24)
     assert np.array_equal(outs["exp"], outs["palette_rt"])
     assert np.array_equal(outs["exp"], outs["palette_direct"])
 
@@ -255,7 +255,7 @@ def test_gate70b_shape_sampled(uw, gate70b, M):
     x = synthdata.activation_for("gate70b_28672x8192", M)
     _workspace(uw, h, M)
     rng = np.random.default_rng(70 + M)
-    rows = np.sort(rng.choice(M, size=min(M, 8), replace=False))
+    rows = np.sort(rng.choice(M, size=min(M, 24), replace=False))
     ref = oracle.gemm_fp64(x[rows], w)
     bound = oracle.abs_product_sum(x[rows], w)
     import torch
