@@ -749,6 +749,26 @@ def run_ours(args):
             if it >= 3:
                 ts.append(a.elapsed_time(b) * 1e3)
         tm[f"M{m}"] = statistics.median(ts)
+    # like for like, launched back to back over the rotated weight sets: torch
+    # BF16 against the pipeline-4 matmul on the compressed weights
+    b2b = {}
+    for m in Ms:
+        def chain(fn, reps=40):
+            for i in range(N_SETS):
+                fn(i)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(reps):
+                fn(i)
+            b.record(stream)
+            torch.cuda.synchronize()
+            return 1e3 * a.elapsed_time(b) / reps
+        b2b[f"M{m}"] = {
+            "torch_matmul_bf16_us": chain(lambda i: torch.matmul(X[m], wbf[i % N_SETS].t())),
+            "palette_direct_us": chain(lambda i: uw.uw_gemm(handles[i % N_SETS], X[m],
+                                                            Y[(m, "palette_direct")], m,
+                                                            uw.PIPELINES["palette_direct"]))}
     del wbf
 
     # ---- the metric's large-M matmuls (gate and down shapes)
@@ -854,6 +874,7 @@ def run_ours(args):
         "kernels": kernels,
         "pipelines": pipelines,
         "torch_matmul_bf16_us": tm,
+        "back_to_back_us": b2b,
         "gemm_large_m": gemm_large,
         "gpu_launches": launches,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
