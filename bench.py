@@ -180,8 +180,9 @@ def _large_m_block(uw, torch, stream, peaks, reps=8):
     whole-pipeline time (calls back to back between two events, weight sets
     rotated), its split into preprocessing and GEMM (the library's traced
     events), the GEMM's TFLOP/s and its roofline time max(2MNK / BF16 peak,
-    algorithmic bytes / HBM peak), and torch.matmul on the decoded BF16
-    weights for context."""
+    algorithmic bytes / HBM peak); then the autotuner's choice for that M
+    (uw_autotune over pipelines, token tiles, ring depths, CTA pairs) timed
+    the same way; torch.matmul on the decoded BF16 weights for context."""
     import numpy as np
     import synthdata
     out = {}
@@ -248,6 +249,23 @@ def _large_m_block(uw, torch, stream, peaks, reps=8):
                           "gemm_frac": 1e6 * t_roof / gemm_us,
                           "gemm_bound": "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >=
                           gbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+            # the autotuner's choice for this M (pipeline, token tile, ring
+            # depth, CTA pairs), timed the same way
+            uw.uw_autotune(hs, [M])
+            choice = uw.uw_get_choice(hs[0], M)
+            call = lambda i: uw.uw_gemm(hs[i % LARGE_M_SETS], X, Y, M, uw.UW_PIPE_AUTO)
+            for i in range(3):
+                call(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(reps):
+                call(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            auto_us = 1e3 * e0.elapsed_time(e1) / reps
+            rec["autotuned"] = {"total_us": auto_us, "choice": choice,
+                                "tflops_whole_pipeline": flops / (auto_us * 1e-6) / 1e12}
             ts = []
             for i in range(3 + reps):
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
