@@ -121,6 +121,7 @@ struct GemmParams {
   uint32_t palette[4];
   uint32_t stage_bytes, x_bytes;
   uint64_t wait_ns;
+  int32_t withhold;  // failure-detection tests: contributors never publish (see launch)
 };
 
 // Per-stage shared-memory layout, offsets from the stage base.
@@ -778,7 +779,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       if (split && !owner) {  // hand the partial sum over
         __threadfence();
         epi_sync();
-        if (leader) st_release(p.sync + 2 + slot_of(pid), tag);
+        if (leader && !p.withhold) st_release(p.sync + 2 + slot_of(pid), tag);
       }
       tc_fence_before();
       __syncwarp();
@@ -1411,6 +1412,12 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, const LaunchHooks* ho
   p.x_bytes = (uint32_t)(pair ? a.tile_n / 2 : a.tile_n) * kBK * 2;
   p.stage_bytes = stage_layout(a.mode, a.tile_n, p.halves, KS).bytes;
   p.wait_ns = wait_limit_ns();
+  // Failure-detection tests (UW_TEST_WITHHOLD_HANDOFF set in the environment,
+  // read once per process): split-tile contributors keep their ready flags
+  // back, so every owner's bounded wait runs out and the launch reports a
+  // timeout through the status word instead of hanging.
+  static const int withhold = std::getenv("UW_TEST_WITHHOLD_HANDOFF") ? 1 : 0;
+  p.withhold = withhold;
   const size_t smem =
       smem_bytes(a.mode, a.tile_n, a.stages, a.wslots, p.halves, tw, KS, a.xstages, a.y_tma != 0,
                  a.pair != 0);
