@@ -75,12 +75,13 @@ def _args():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-large-m", action="store_true",
-                    help="skip the large-M matmul block (gate M = 1024, down M = 256, 1024)")
+                    help="skip the large-M matmul block (gate M = 1024, down M = 256, 1024) "
+                         "and the Huffman-direct block (pipeline 5, M = 1, 2, 8)")
     # single-kernel runs for profilers: three launches of one kernel, nothing timed
     ap.add_argument("--only", choices=("decode_full", "decode_exp", "transcode", "gemm_bf16",
                                        "gemm_exp", "gemm_palette", "gemv_bf16", "gemv_exp",
-                                       "gemv_palette"))
-    ap.add_argument("--m", type=int, default=1, help="tokens for --only gemm_*")
+                                       "gemv_palette", "decode_dot"))
+    ap.add_argument("--m", type=int, default=1, help="tokens for --only gemm_*, gemv_*, decode_dot")
     # the Llama-3.1-8B-shaped MLP stack end to end (prints its own JSON line)
     ap.add_argument("--mlp-layers", type=int, default=0,
                     help="time uw_mlp_forward over this many gate/up/down layers")
@@ -118,6 +119,7 @@ def _alg_bytes(kind, st, M, N, K, x_frac=1.0):
         "gemm_bf16": 2 * T + xy,
         "gemm_exp": 2 * T + xy,
         "gemm_palette": T + T // 2 + esc + xy,
+        "decode_dot": stream + T + xy,
     }
     return b[kind.replace("gemv_", "gemm_")]
 
@@ -283,6 +285,78 @@ def _large_m_block(uw, torch, stream, peaks, reps=8):
                 raise RuntimeError("device status")
             h.free()
         del wbf, ws
+    return out
+
+
+# Huffman-direct product block of the bench line: shapes, token counts, and
+# the weight sets rotated per call.
+HDOT = (("gate_14336x4096", (1, 2, 8)), ("down_4096x14336", (1, 2, 8)))
+HDOT_SETS = 2
+
+
+def _hdot_block(uw, torch, stream, peaks, reps=10):
+    """Pipeline 5 (the stream decoded inside the matmul, no preprocessing
+    pass) at small M on the gate and down shapes: whole-call time back to back
+    (weight sets rotated), the kernel's traced time, its algorithmic bytes
+    (stream, offsets, S, X, Y) and fraction of HBM; beside it the whole
+    pipelines 2, 3 and 4 at the same M, timed the same way."""
+    import numpy as np
+    import synthdata
+    out = {}
+    for wl, Ms in HDOT:
+        spec = synthdata.WORKLOADS[wl]
+        N, K = spec["N"], spec["K"]
+        hs = []
+        for i in range(HDOT_SETS):
+            w = synthdata.normal(N, K, spec["std"], spec["seed_w"] + 2 * i)
+            hs.append(uw.uw_encode(w, stream=stream))
+            del w
+        st = hs[0].stats()
+        need = max(uw.uw_workspace_bytes(hs[0], p, m) for p in (2, 3, 5) for m in Ms)
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        for h in hs:
+            uw.uw_set_workspace(h, ws)
+        for M in Ms:
+            X = torch.from_numpy(synthdata.activations(M, K, spec["seed_x"] + M).view(np.int16)).cuda()
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+
+            def chain(p):
+                call = lambda i: uw.uw_gemm(hs[i % HDOT_SETS], X, Y, M, p)
+                for i in range(3):
+                    call(i)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for i in range(reps):
+                    call(i)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                return 1e3 * e0.elapsed_time(e1) / reps
+
+            rec = {"total_us": chain(uw.UW_PIPE_HUFFMAN_DIRECT)}
+            for h in hs:
+                uw.uw_trace_read(h)
+                uw.uw_trace_enable(h, True)
+            for i in range(reps):
+                uw.uw_gemm(hs[i % HDOT_SETS], X, Y, M, uw.UW_PIPE_HUFFMAN_DIRECT)
+            torch.cuda.synchronize()
+            tr = [ms for h in hs for kind, ms in uw.uw_trace_read(h) if kind == "decode_dot"]
+            for h in hs:
+                uw.uw_trace_enable(h, False)
+            k_us = 1e3 * statistics.median(tr)
+            alg = _alg_bytes("decode_dot", st, M, N, K)
+            rec.update({"kernel_us_traced": k_us, "alg_bytes": alg,
+                        "bytes_per_weight": (st["bytes_stream"] + st["bytes_offsets"] + N * K) / (N * K),
+                        "frac_hbm_b2b": alg / (rec["total_us"] * 1e-6) / (peaks["hbm_gbs"] * 1e9),
+                        "frac_hbm_traced": alg / (k_us * 1e-6) / (peaks["hbm_gbs"] * 1e9)})
+            for p in ("exp", "palette_rt", "palette_direct"):
+                rec[f"{p}_total_us"] = chain(uw.PIPELINES[p])
+            out[f"{wl}/M{M}"] = rec
+        for h in hs:
+            if uw.uw_last_device_status(h) != uw.UW_OK:
+                raise RuntimeError("device status")
+            h.free()
+        del ws
     return out
 
 
@@ -791,6 +865,8 @@ def run_ours(args):
 
     # ---- the metric's large-M matmuls (gate and down shapes)
     gemm_large = None if args.no_large_m else _large_m_block(uw, torch, stream, peaks)
+    # ---- the Huffman-direct product (pipeline 5) at small M
+    hdot = None if args.no_large_m else _hdot_block(uw, torch, stream, peaks)
 
     # ---- end to end through the public call with host buffers: every step
     # copies its X in from pinned host memory and its Y out to pinned host
@@ -894,6 +970,7 @@ def run_ours(args):
         "torch_matmul_bf16_us": tm,
         "back_to_back_us": b2b,
         "gemm_large_m": gemm_large,
+        "huffman_direct": hdot,
         "gpu_launches": launches,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -913,8 +990,9 @@ def run_ours(args):
 def run_only(args):
     """Three launches of one kernel on the bench workload (first set of weights),
     for a profiler to capture (select by kernel name: decode_kernel<0|1|2> is
-    exponent / full / transcode, gemm_kernel<0|1|2> bf16 / exponent / palette,
-    gemv_kernel<0|1|2, tokens> the matrix-vector kernels).
+    exponent / full / transcode, decode_kernel<3> the Huffman-direct product,
+    gemm_kernel<0|1|2> bf16 / exponent / palette, gemv_kernel<0|1|2, tokens>
+    the matrix-vector kernels).
     The handle is uploaded without the load-time transcode unless the palette
     GEMM needs it (that launch comes first)."""
     import numpy as np
@@ -928,7 +1006,7 @@ def run_only(args):
     h = uw.uw_encode(w, uw.default_opts(prepare_direct=1 if direct else 0))
     out = torch.empty(2 * N * K, dtype=torch.uint8, device="cuda")
     pipe = {"gemm_bf16": 1, "gemm_exp": 2, "gemm_palette": 4,
-            "gemv_bf16": 1, "gemv_exp": 2, "gemv_palette": 4}.get(args.only)
+            "gemv_bf16": 1, "gemv_exp": 2, "gemv_palette": 4, "decode_dot": 5}.get(args.only)
     gemv = args.only.startswith("gemv")
     if pipe:
         M = args.m

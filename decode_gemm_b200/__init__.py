@@ -32,6 +32,8 @@ UW_OK, UW_ERR_ARG, UW_ERR_SHAPE, UW_ERR_FORMAT, UW_ERR_UNSUPPORTED = 0, 1, 2, 3,
 UW_ERR_OOM, UW_ERR_CUDA, UW_ERR_DEVICE, UW_ERR_TIMEOUT, UW_ERR_WORKSPACE = 5, 6, 7, 8, 9
 UW_ERR_IO = 10
 UW_PIPE_AUTO, UW_PIPE_FULL, UW_PIPE_EXP, UW_PIPE_PALETTE_RT, UW_PIPE_PALETTE_DIRECT = 0, 1, 2, 3, 4
+UW_PIPE_HUFFMAN_DIRECT = 5   # the Huffman-direct product (M <= DOT_MAX_M)
+DOT_MAX_M = 4
 PIPELINES = {"full": UW_PIPE_FULL, "exp": UW_PIPE_EXP, "palette_rt": UW_PIPE_PALETTE_RT,
              "palette_direct": UW_PIPE_PALETTE_DIRECT}
 
@@ -519,7 +521,8 @@ def uw_get_choice(h: Handle, M: int) -> dict:
 
 
 KERNEL_KINDS = ("decode_full", "decode_exp", "transcode", "gemm_bf16", "gemm_exp",
-                "gemm_palette", "splitk_fixup", "gemv_bf16", "gemv_exp", "gemv_palette")
+                "gemm_palette", "splitk_fixup", "gemv_bf16", "gemv_exp", "gemv_palette",
+                "decode_dot")
 
 
 def uw_trace_enable(h: Handle, enable: bool = True) -> None:

@@ -1,5 +1,6 @@
 // C ABI, device side: upload, preprocessing entry points, GEMM dispatch over
-// the four pipelines, workspace and status handling.
+// the four pipelines and the Huffman-direct product, workspace and status
+// handling.
 //
 // *Unweight*, "Four ways to use compressed weights": pipeline 1 decodes to
 // BF16 in HBM and runs a plain GEMM; pipeline 2 decodes exponent bytes only,
@@ -69,7 +70,12 @@ GemmArgs base_gemm_args(const uw_handle_s* h) {
   return a;
 }
 
-bool valid_pipeline(int p) { return p >= UW_PIPE_FULL && p <= UW_PIPE_PALETTE_DIRECT; }
+bool valid_pipeline(int p) { return p >= UW_PIPE_FULL && p <= UW_PIPE_HUFFMAN_DIRECT; }
+
+// Workspace bytes of the Huffman-direct product's partial sums.
+size_t dot_part_bytes(const uw_handle_s* h) {
+  return align_up((size_t)dot_part_floats(h->n_chunks) * 4, 256);
+}
 
 }  // namespace
 
@@ -115,6 +121,13 @@ uw_gemm_config choose_variant(const uw_handle_s* h, int64_t M) {
     if (it == h->profile.end()) --it;
     c = it->second;
     if (c.pipeline == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) c.pipeline = UW_PIPE_PALETTE_RT;
+    // an entry tuned for fewer tokens may name a kernel that does not serve M:
+    // the tensor-core GEMM of its pipeline, or the default pipeline, instead
+    if (c.gemv > 0 && M > kGemvMaxM) c.gemv = 0;
+    if (c.pipeline == UW_PIPE_HUFFMAN_DIRECT && !dot_for(h, M)) {
+      std::memset(&c, 0, sizeof(c));
+      c.pipeline = h->d_pal_idx ? UW_PIPE_PALETTE_DIRECT : UW_PIPE_PALETTE_RT;
+    }
     return c;
   }
   c.pipeline = h->d_pal_idx ? UW_PIPE_PALETTE_DIRECT : UW_PIPE_PALETTE_RT;
@@ -143,6 +156,30 @@ void trace_end(uw_handle_s* h, int slot) {
 static int hook_begin(void* ctx, int kind) { return trace_begin(static_cast<uw_handle_s*>(ctx), kind); }
 static void hook_end(void* ctx, int slot) { trace_end(static_cast<uw_handle_s*>(ctx), slot); }
 
+bool dot_for(const uw_handle_s* h, int64_t M) {
+  return dot_supported(h->K, h->chunk_syms, M);
+}
+
+// The Huffman-direct product Y = X W^T (pipeline 5), partial sums in `part`.
+uw_status run_dot_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M, int out_f32,
+                     int ctas, float* part, size_t part_bytes, cudaStream_t s) {
+  if (!dot_for(h, M)) return UW_ERR_UNSUPPORTED;
+  if (!part || part_bytes < (size_t)dot_part_floats(h->n_chunks) * 4) return UW_ERR_WORKSPACE;
+  DecodeArgs a = decode_args(h);
+  a.cpr = (int32_t)(h->K / h->chunk_syms);
+  a.matrix_rows = h->N;
+  a.x = X;
+  a.y = Y;
+  a.m = (int32_t)M;
+  a.out_f32 = out_f32;
+  a.part = part;
+  a.row_cnt = h->d_row_cnt;
+  const int slot = trace_begin(h, UW_KERNEL_DECODE_DOT);
+  const cudaError_t e = launch_decode(kDecodeDot, a, nullptr, ctas, s);
+  trace_end(h, slot);
+  return map_cuda(e);
+}
+
 uw_status run_decode(uw_handle_s* h, int mode, void* out, int ctas, cudaStream_t s) {
   DecodeArgs a = decode_args(h);
   // kinds: 0 full, 1 exponent, 2 transcode
@@ -162,6 +199,14 @@ uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
   a.X = X;
   a.Y = Y;
   a.out_f32 = out_f32;
+  if (cfg.pipeline == UW_PIPE_HUFFMAN_DIRECT) {  // one kernel: partial sums only
+    if (!dot_for(h, M)) return UW_ERR_UNSUPPORTED;
+    a.partials_bytes = dot_part_bytes(h);
+    *pre_bytes = 0;
+    *ws_need = a.partials_bytes;
+    *ga = a;
+    return UW_OK;
+  }
   a.tile_n = cfg.tile_n;
   a.stages = cfg.stages;
   a.halves = cfg.halves;
@@ -193,6 +238,7 @@ uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg) {
   if (cfg.halves < 0 || cfg.halves > 2) return UW_ERR_ARG;
   if (cfg.pair < 0 || cfg.pair > 1 || (cfg.pair && cfg.halves == 2)) return UW_ERR_ARG;
   if (cfg.pair && cfg.pipeline != UW_PIPE_FULL) return UW_ERR_UNSUPPORTED;
+  if (cfg.gemv && cfg.pipeline == UW_PIPE_HUFFMAN_DIRECT) return UW_ERR_ARG;
   if (cfg.stages < 0 || cfg.stages > 16 || (cfg.halves != 2 && (cfg.stages & 1)))
     return UW_ERR_ARG;
   if (cfg.gemm_ctas < 0 || cfg.decode_ctas < 0) return UW_ERR_ARG;
@@ -260,6 +306,8 @@ bool gemv_for(const uw_handle_s* h, const uw_gemm_config& cfg, int64_t M) {
 uw_status run_gemm_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
                       const uw_gemm_config& cfg, int out_f32, const void* pre, float* partials,
                       size_t partials_bytes, cudaStream_t s) {
+  if (cfg.pipeline == UW_PIPE_HUFFMAN_DIRECT)
+    return run_dot_on(h, X, Y, M, out_f32, cfg.gemm_ctas, partials, partials_bytes, s);
   if (gemv_for(h, cfg, M)) return run_gemv_on(h, X, Y, M, cfg.pipeline, out_f32, pre, s);
   GemmArgs a;
   size_t need = 0, pre_b = 0;
@@ -293,6 +341,11 @@ uw_status run_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
   uw_status st = check_config(h, cfg);
   if (st != UW_OK) return st;
   if (cfg.gemv > 0 && M > kGemvMaxM) return UW_ERR_UNSUPPORTED;
+  if (cfg.pipeline == UW_PIPE_HUFFMAN_DIRECT) {
+    if (!dot_for(h, M)) return UW_ERR_UNSUPPORTED;
+    return run_dot_on(h, X, Y, M, out_f32, cfg.gemm_ctas, static_cast<float*>(h->ws),
+                      h->ws_bytes, h->stream);
+  }
   if (gemv_for(h, cfg, M)) {
     // preprocessed weights (pipelines 1-3) in the workspace; no partial sums
     const size_t pre_b = align_up(preprocess_bytes(h, cfg.pipeline), 256);
@@ -394,6 +447,7 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   const size_t o_stat = place(256);
   const size_t o_sync = place(kGemmSyncWords * 4);
   const size_t o_pidx = o.prepare_direct ? place(T / 2) : 0;
+  const size_t o_rcnt = place((size_t)f->N * 4);
   cudaError_t e = cudaMalloc(&h->d_block, off);
   if (e != cudaSuccess) {
     delete h;
@@ -424,6 +478,7 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
   h->d_status = reinterpret_cast<uint32_t*>(base + o_stat);
   h->d_sync = reinterpret_cast<uint32_t*>(base + o_sync);
   h->d_pal_idx = o.prepare_direct ? base + o_pidx : nullptr;
+  h->d_row_cnt = reinterpret_cast<uint32_t*>(base + o_rcnt);
   cudaStream_t s = h->stream;
   const Part parts[] = {
       {(void**)&h->d_words, f->words, (size_t)f->n_words * 4},
@@ -445,6 +500,7 @@ uw_status uw_upload(const uw_format* f, const uw_encode_opts* opts, void* stream
     e = cudaMemsetAsync(h->d_words + f->n_words, 0, (size_t)pad_words * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->d_status, 0, 256, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->d_sync, 0, kGemmSyncWords * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->d_row_cnt, 0, (size_t)f->N * 4, s);
   if (e == cudaSuccess && h->d_pal_idx) {
     // load-time transcode: the resident palette form of pipeline 4
     DecodeArgs a = decode_args(h);

@@ -48,6 +48,12 @@ std::vector<uw_gemm_config> candidates(const uw_handle_s* h, int64_t M) {
   for (int t : {16, 32, 64, 128, 256})
     if (t <= std::max(16, 2 * m16) && (M <= 256 || t >= 128)) tiles.push_back(t);
   std::vector<uw_gemm_config> out;
+  if (dot_for(h, M)) {  // the Huffman-direct product: one kernel, no preprocessing
+    uw_gemm_config c;
+    std::memset(&c, 0, sizeof(c));
+    c.pipeline = UW_PIPE_HUFFMAN_DIRECT;
+    out.push_back(c);
+  }
   for (int p = UW_PIPE_FULL; p <= UW_PIPE_PALETTE_DIRECT; ++p) {
     if (p == UW_PIPE_PALETTE_DIRECT && !h->d_pal_idx) continue;
     if (M <= kGemvMaxM) {  // the matrix-vector kernel on the CUDA cores, if it fits

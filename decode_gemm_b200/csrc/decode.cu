@@ -35,6 +35,7 @@
 //     128-symbol round the warp writes its 32 chunks' outputs with 128-bit
 //     stores, each warp-wide store covering contiguous, fully used lines.
 //     Shared memory stays small so L1 can hold every lane's stream lines.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -57,6 +58,8 @@ constexpr int kStageStride = kRoundWords + 1;   // 17: lanes spread over banks
 constexpr int kExcCap = 4;                      // exceptions held per lane
 constexpr int kFullPair = 2 * 4 * kPalCap;      // 4x symbols two whole lookups may yield
 constexpr int kFullOne = 4 * kPalCap;
+constexpr int kNoRound = 1 << 30;
+
 
 // Shared memory: the tables, then per warp its ranks stage (32 lanes x 17
 // words) and exception lists.  At most ~104 KB, so L1 keeps over 120 KB for the
@@ -66,10 +69,13 @@ struct __align__(16) SmemHead {
   uint32_t canon[kCanonWords];
 };
 constexpr int kWarpSmemWords = 32 * kStageStride + 32 * kExcCap;
+// The product's running sums between rounds: 8 per lane (see below).
+constexpr int kDotAccWords = 32 * 16;  // and its corrections: 8 more per lane
 
-size_t smem_bytes(int warps) {
-  return sizeof(SmemHead) + (size_t)warps * kWarpSmemWords * 4;
+size_t smem_bytes(int warps, int mode) {
+  return sizeof(SmemHead) + (size_t)warps * (kWarpSmemWords + (mode == kDecodeDot ? kDotAccWords : 0)) * 4;
 }
+
 
 // Four consecutive stream words; bit q (MSB first) of w0 is the next bit.
 struct Bits {
@@ -138,6 +144,58 @@ __device__ __forceinline__ uint32_t ld_u32_if(const uint32_t* p, bool pred) {
   return v;
 }
 
+// D += A B for one m16n8k16 tile (BF16 operands, FP32 accumulation).  Lane
+// (g, t) = (lane / 4, lane % 4) holds a0..a3 = A[g][2t..2t+1], A[g+8][2t..2t+1],
+// A[g][2t+8..2t+9], A[g+8][2t+8..2t+9], b0 / b1 = B[2t..2t+1][g] /
+// B[2t+8..2t+9][g], and d = D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1].
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The caller's X, read after the dependency wait with coherent loads (the
+// kernel ahead of this one may have written it).
+__device__ __forceinline__ uint4 ld_x4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+// Four X values (two pair words), or zeros where pred is false.
+__device__ __forceinline__ uint2 ldx_v2_if(const void* p, bool pred) {
+  uint2 v = make_uint2(0u, 0u);
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %3, 0;\n\t"
+               "@q ld.global.v2.u32 {%0, %1}, [%2];\n\t}"
+               : "+r"(v.x), "+r"(v.y)
+               : "l"(p), "r"((uint32_t)pred));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t ld_x1(const uint16_t* p) {
+  uint16_t v;
+  asm volatile("ld.global.u16 %0, [%1];" : "=h"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// 16 sign+mantissa bytes (the handle's own, never written by a kernel), or
+// zeros where pred is false.
+__device__ __forceinline__ uint4 ld_v4_if(const void* p, bool pred) {
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %5, 0;\n\t"
+      "@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+      : "l"(p), "r"((uint32_t)pred));
+  return v;
+}
+
+
 // Stream bit position of the next bit.
 __device__ __forceinline__ uint32_t bits_pos(const Bits& b) { return (b.nxt - 4u) * 32u + b.q; }
 
@@ -187,6 +245,9 @@ __device__ __forceinline__ void pack(Packer& pk, uint32_t e, uint32_t c4) {
 // GATHER (full decode only): the launch's chunks are the chunks of the rows
 // a.rows[] (see DecodeArgs); a lane reads its chunk's stream and S at the real
 // chunk and writes its output at the launch's (virtual) chunk.
+//
+// DOT (the Huffman-direct product): the write-out becomes a matrix product of
+// the rebuilt weights with X; nothing but Y leaves the chip.
 template <int MODE, bool GATHER>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     decode_kernel(const DecodeArgs a, void* __restrict__ out) {
@@ -210,8 +271,16 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
       reinterpret_cast<uint32_t*>(smem_raw + sizeof(SmemHead)) + warp * kWarpSmemWords;
   const uint32_t st_addr = (uint32_t)__cvta_generic_to_shared(stage + lane * kStageStride);
   uint32_t* const exc = stage + 32 * kStageStride + lane * kExcCap;
+  // (product) this lane's 8 running sums and 8 corrections (one per token),
+  // behind all warps' areas
+  float* const dsum_w = reinterpret_cast<float*>(smem_raw + sizeof(SmemHead)) +
+                        (size_t)n_warps * kWarpSmemWords + (size_t)warp * 32 * 16;
+  float* const dsum = dsum_w + lane * 16;
+  float* const dcorr = dsum + 8;
   const uint32_t* const lut = sm.lut;
-  const int64_t groups = (a.n_chunks + 31) / 32;
+  // the product's groups are 32 rows at one chunk position (one column range)
+  const int64_t groups =
+      MODE == kDecodeDot ? (a.matrix_rows + 31) / 32 * a.cpr : (a.n_chunks + 31) / 32;
   const uint32_t* const words = a.words;
   const uint32_t stream_bits = (uint32_t)(a.n_words * 32);
   const int64_t cs = a.chunk_syms;
@@ -224,11 +293,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   for (int64_t grp = (int64_t)blockIdx.x * n_warps + warp; grp < groups; grp += grid_warps) {
     const int64_t c0 = grp * 32;
     const int64_t c = c0 + lane;
-    const bool live = c < a.n_chunks;
+    // product: rows rb*32 .. rb*32+31 (lane = row), chunk position cc
+    const int64_t rb = MODE == kDecodeDot ? grp / a.cpr : 0;
+    const int cc = MODE == kDecodeDot ? (int)(grp - rb * a.cpr) : 0;
+    const bool live = MODE == kDecodeDot ? rb * 32 + lane < a.matrix_rows : c < a.n_chunks;
     uint32_t start = 0, end = 0;
     int nsyms = 0;
     bool bad = false;
-    int64_t cr = c;  // the chunk of the matrix this lane decodes
+    // the chunk of the matrix this lane decodes
+    int64_t cr = MODE == kDecodeDot ? (rb * 32 + lane) * a.cpr + cc : c;
     if (GATHER && !waited) {  // the row ids are the caller's: after the kernel before
       pdl_wait();
       waited = true;
@@ -246,7 +319,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     if (live && cr >= 0) {
       start = __ldg(a.chunk_off + cr);
       end = __ldg(a.chunk_off + cr + 1);
-      const int64_t left = GATHER ? cs : a.total_syms - c * cs;
+      const int64_t left = (GATHER || MODE == kDecodeDot) ? cs : a.total_syms - c * cs;
       nsyms = (int)(left < cs ? left : cs);
       if (start > stream_bits) {  // corrupt offset: nothing is read
         bad = true;
@@ -254,11 +327,18 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         nsyms = 0;
       }
     }
-    if (cr < 0) cr = 0;  // (a rejected row reads nothing; S accesses stay in bounds)
+    if (cr < 0 || (MODE == kDecodeDot && !live)) cr = 0;  // (a rejected row or a row
+                                                          // past N reads nothing)
     // the stream of this warp's next group: into L2 while this one decodes
     if (!GATHER) {
-      const int64_t cn = c + grid_warps * 32;
-      if (cn < a.n_chunks) {
+      int64_t cn = c + grid_warps * 32;
+      bool next = cn < a.n_chunks;
+      if (MODE == kDecodeDot) {
+        const int64_t g2 = grp + grid_warps, rb2 = g2 / a.cpr;
+        cn = (rb2 * 32 + lane) * a.cpr + (g2 - rb2 * a.cpr);
+        next = g2 < groups && rb2 * 32 + lane < a.matrix_rows;
+      }
+      if (next) {
         const uint32_t nb = __ldg(a.chunk_off + cn) >> 3;
         if (nb < stream_bits / 8) {
           const char* p = reinterpret_cast<const char*>(words) + nb;
@@ -286,6 +366,27 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     int left4 = 4 * nsyms;  // 4 x symbols of the chunk not yet decoded
     int nx = 0;
     bool overflow = false;
+
+    // Product state: the first round after which this lane's chunk is left to
+    // the replay (its exception list overflowed).  The running sums (dsum)
+    // and the lane's corrections (dcorr: the true weights' products at its
+    // chunk's exceptions, per token) live in shared memory.
+    int dirty_from = kNoRound;
+    bool fixed = false;  // a correction was made
+    if (MODE == kDecodeDot) {
+#pragma unroll
+      for (int q = 0; q < kExcCap; ++q) exc[q] = 0xFFFFFFFFu;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) reinterpret_cast<float4*>(dsum)[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // BF16 weight w times X[t, column col] into this lane's correction
+    // (the product of two BF16 is exact in FP32)
+    auto add_corr = [&](uint32_t w, int64_t col) {
+      const int64_t K = (int64_t)a.kb_per_row * kRow;
+      fixed = true;
+      for (int t = 0; t < a.m; ++t)
+        dcorr[t] += __uint_as_float(w << 16) * __uint_as_float((uint32_t)ld_x1(a.x + t * K + col) << 16);
+    };
 
     // A flagged entry: record the exception (position = symbols decoded so far).
     auto special = [&](uint32_t e, uint32_t win, int left4_before) {
@@ -339,10 +440,14 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 
     for (int r = 0; r < warp_rounds; ++r) {
       pk.sp = st_addr;
-      if (MODE == kDecodeFull && r < my_rounds) {
-        // this round's sign+mantissa bytes into L2 while the round decodes
+      if ((MODE == kDecodeFull || MODE == kDecodeDot) && r < my_rounds) {
+        // this round's sign+mantissa bytes into L2 (the product: into L1, its
+        // reads follow this lane's own chunk) while the round decodes
         const uint8_t* sp8 = a.sm + cr * cs + (int64_t)r * kRoundSyms;
-        asm volatile("prefetch.global.L2 [%0];" :: "l"(sp8));
+        if (MODE == kDecodeDot)
+          asm volatile("prefetch.global.L1 [%0];" :: "l"(sp8));
+        else
+          asm volatile("prefetch.global.L2 [%0];" :: "l"(sp8));
       }
       if (r < my_rounds - 1) {
         // a round that ends inside the chunk: fill exactly kRoundWords words,
@@ -424,6 +529,93 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
           write([&](uint32_t v) { return run8(v, b4); });
         else
           write([&](uint32_t v) { return palette8(v, p0, p1, p2, p3); });
+      } else if (MODE == kDecodeDot) {
+        // The group's 32 chunks hold the same columns of 32 rows, so the
+        // round's product is a small matrix product: for each block of 16
+        // rows and each 16 of the round's 128 columns, one mma.sync m16n8k16
+        // with A = the rebuilt BF16 weights, straight from the field merge,
+        // and B = X transposed (tokens as columns, zero past M), FP32
+        // accumulation.  The 16 k slots of MMA q are columns 32t + 4q + {0..3}
+        // of lane group t = lane % 4 (any column order works when A and B
+        // share it), so lane (g, t) = (lane / 4, lane % 4) rebuilds rows g and
+        // g + 8 of each block at columns 32t .. 32t+31 and holds X[g] at the
+        // same columns.  A lane whose exception list overflowed leaves its
+        // chunk to the replay from this round on; at recorded exceptions the
+        // weight is zeroed here and the owner lane adds the true product to
+        // its correction.
+        if (overflow && dirty_from == kNoRound) dirty_from = r;
+        const uint32_t dirty = __ballot_sync(0xffffffffu, dirty_from <= r);
+        const uint32_t excm = __ballot_sync(0xffffffffu, nx > 0);
+        const int g = lane >> 2, tq = lane & 3;
+        const int p32 = (int)rel0 + 32 * tq;  // this lane's first symbol in each chunk
+        const bool in_chunk = p32 < cs;
+        const int64_t K = (int64_t)a.kb_per_row * kRow;
+        const int64_t col0 = (int64_t)cc * cs + p32;  // its first column
+        // X[g] at this lane's columns (zero past M or past the chunk), read
+        // four columns per MMA
+        const bool have_x = in_chunk && g < a.m;
+        const uint16_t* xp = a.x + (have_x ? g * K + col0 : 0);
+        // this lane's rows j (g, then g + 8, of block bk): rebuild rule and
+        // exceptions to zero (bit i: symbol p32 + i)
+        auto row_setup = [&](int j, bool& valid, uint32_t& kill) {
+          valid = in_chunk && rb * 32 + j < a.matrix_rows && !((dirty >> j) & 1u);
+          kill = 0;
+          if ((excm >> j) & 1u) {
+            const uint32_t* ej = stage + 32 * kStageStride + j * kExcCap;
+#pragma unroll
+            for (int qq = 0; qq < kExcCap; ++qq) {
+              const uint32_t d = (ej[qq] >> 8) - (uint32_t)p32;
+              if (d < 32u) kill |= 1u << d;
+            }
+          }
+        };
+        auto killed = [&](uint2 b, uint32_t kill, int q) {
+          const uint32_t k4 = kill >> (4 * q);
+          b.x &= ((k4 & 1u) ? 0u : 0xFFFFu) | ((k4 & 2u) ? 0u : 0xFFFF0000u);
+          b.y &= ((k4 & 4u) ? 0u : 0xFFFFu) | ((k4 & 8u) ? 0u : 0xFFFF0000u);
+          return b;
+        };
+        auto dot = [&](auto expo) {
+#pragma unroll 1
+          for (int bk = 0; bk < 2; ++bk) {
+            const int ja = 16 * bk + g, jb = ja + 8;
+            bool va, vb;
+            uint32_t ka, kb;
+            row_setup(ja, va, ka);
+            row_setup(jb, vb, kb);
+            const bool any_kill = __any_sync(0xffffffffu, (ka | kb) != 0u);
+            float4 d4 = reinterpret_cast<const float4*>(dsum)[bk];  // the block's sums
+            float dacc[4] = {d4.x, d4.y, d4.z, d4.w};
+            __syncwarp();  // converged for the warp-wide MMAs below
+            const uint8_t* spa = a.sm + (rb * 32 + ja) * K + col0;
+            const uint8_t* spb = a.sm + (rb * 32 + jb) * K + col0;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {  // symbols 8u .. 8u+7 of the lane's 32
+              const uint2 sa = ld_v2_if(spa + 8 * u, va), sb = ld_v2_if(spb + 8 * u, vb);
+              uint2 ea = expo(stage[ja * kStageStride + 4 * tq + u]);
+              uint2 eb = expo(stage[jb * kStageStride + 4 * tq + u]);
+              ea = va ? ea : make_uint2(0u, 0u);  // (S reads as zero there too: +0)
+              eb = vb ? eb : make_uint2(0u, 0u);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int q = 2 * u + h;
+                uint2 wa = merge4(h ? sa.y : sa.x, h ? ea.y : ea.x);
+                uint2 wb = merge4(h ? sb.y : sb.x, h ? eb.y : eb.x);
+                if (any_kill) {  // (uniform; lanes without exceptions keep all)
+                  wa = killed(wa, ka, q);
+                  wb = killed(wb, kb, q);
+                }
+                const uint2 xq = ldx_v2_if(xp + 4 * q, have_x);
+                mma_16816(dacc, wa.x, wb.x, wa.y, wb.y, xq.x, xq.y);
+              }
+            }
+            reinterpret_cast<float4*>(dsum)[bk] = make_float4(dacc[0], dacc[1], dacc[2], dacc[3]);
+          }
+        };
+        if (pal_run)
+          dot([&](uint32_t v) { return run8(v, b4); });
+        else
+          dot([&](uint32_t v) { return palette8(v, p0, p1, p2, p3); });
       } else {
         // 4 lanes per chunk, 32 symbols (four rank words, half a 64-weight
         // row) per lane; escape rows are written as zeros
@@ -474,22 +666,42 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             const int64_t o = base + pos;
             if (MODE == kDecodeExp) {
               static_cast<uint8_t*>(out)[o] = (uint8_t)(x & 0xFFu);
-            } else {
+            } else if (MODE == kDecodeFull) {
               const uint32_t s = a.sm[cr * cs + pos];
               static_cast<uint16_t*>(out)[o] =
                   (uint16_t)(((s & 0x80u) << 8) | ((x & 0xFFu) << 7) | (s & 0x7Fu));
+            } else if (dirty_from > r) {  // the product: the true weight's terms
+              const uint32_t s = a.sm[cr * cs + pos];
+              add_corr(((s & 0x80u) << 8) | ((x & 0xFFu) << 7) | (s & 0x7Fu),
+                       (int64_t)cc * cs + pos);
             }
           } else {
             exc[keep++] = x;
           }
         }
+        if (MODE == kDecodeDot)  // freed entries match no position
+          for (int q = keep; q < nx; ++q) exc[q] = 0xFFFFFFFFu;
         nx = keep;
       }
       __syncwarp();
     }
 
     // a lane whose exception list overflowed replays its chunk symbol by symbol
-    if (MODE != kDecodePalette && overflow) {
+    if (MODE == kDecodeDot && overflow) {  // the product: from its first dirty round on
+      Bits sb;
+      bits_init(sb, words, start);
+      for (int i = 0; i < nsyms; ++i) {
+        uint32_t len;
+        const uint32_t ex = canon_symbol(sm.canon, bits_peek(sb) >> 20, &len);
+        sb.q += len;
+        bits_slide(sb, words);
+        if (i >= dirty_from * kRoundSyms) {
+          const uint32_t s = a.sm[cr * cs + i];
+          add_corr(((s & 0x80u) << 8) | (ex << 7) | (s & 0x7Fu), (int64_t)cc * cs + i);
+        }
+      }
+    }
+    if (MODE != kDecodePalette && MODE != kDecodeDot && overflow) {
       Bits sb;
       bits_init(sb, words, start);
       const int64_t base = c * cs;
@@ -509,6 +721,51 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     }
     if (live && (bad || bits_pos(b) != end)) atomicOr(a.status, kStatusBadChunk);
     __syncwarp();
+
+    if (MODE == kDecodeDot) {
+      // Lane (g, t) holds the sums of rows 16 bk + g + 8 h (dsum[4 bk + 2 h +
+      // e]) for tokens 2t + e; with the owners' corrections added they are
+      // the group's partial sums, stored at part[(row * kDotMaxM + token) *
+      // cpr + cc].  The group that brings a row's cpr-th partial adds them in
+      // chunk order and writes Y.
+      const int g = lane >> 2, tq = lane & 3;
+      const bool any_corr = __any_sync(0xffffffffu, fixed);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int bk = k >> 2, h = (k >> 1) & 1, e = k & 1;
+        const int j = 16 * bk + g + 8 * h, t = 2 * tq + e;
+        float v = dsum[k];
+        if (any_corr && t < a.m) v += dsum_w[j * 16 + 8 + t];  // row j's owner's correction
+        const int64_t row = rb * 32 + j;
+        if (t < a.m && row < a.matrix_rows) a.part[(row * kDotMaxM + t) * a.cpr + cc] = v;
+      }
+      __threadfence();
+      __syncwarp();
+      const int64_t row = rb * 32 + lane;  // lane l: row l of the group
+      if (row < a.matrix_rows && atomicAdd(a.row_cnt + row, 1u) == (uint32_t)(a.cpr - 1)) {
+        __threadfence();
+        for (int t = 0; t < a.m; ++t) {
+          // the row's partials for token t are contiguous: loaded four at a
+          // time when they can be, added in chunk order
+          const float* pt = a.part + (row * kDotMaxM + t) * a.cpr;
+          float y = 0.f;
+          int q = 0;
+          if ((a.cpr & 3) == 0)
+            for (; q < a.cpr; q += 4) {
+              const float4 v = __ldcg(reinterpret_cast<const float4*>(pt + q));
+              y = y + v.x + v.y + v.z + v.w;
+            }
+          for (; q < a.cpr; ++q) y += __ldcg(pt + q);
+          const int64_t o = (int64_t)t * a.matrix_rows + row;
+          if (a.out_f32)
+            static_cast<float*>(a.y)[o] = y;
+          else
+            static_cast<uint16_t*>(a.y)[o] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+        }
+        a.row_cnt[row] = 0u;
+      }
+      __syncwarp();
+    }
   }
 }
 
@@ -523,6 +780,10 @@ cudaError_t set_attrs(F* f, size_t smem) {
 }
 
 }  // namespace
+
+bool dot_supported(int64_t K, int64_t chunk_syms, int64_t M) {
+  return chunk_syms > 0 && K % chunk_syms == 0 && M >= 1 && M <= kDotMaxM;
+}
 
 // Launch shape: one CTA per SM (capped at `sms`) with W warps, a warp decoding
 // 32 chunks per pass.  A pass takes about as long as the SM's warps share its
@@ -570,9 +831,17 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cu
   if (ctas > 0 && ctas < sms) sms = ctas;  // an SM budget (decoder/GEMM split)
   int grid = 0, warps = 0;
   decode_launch_shape(a.n_chunks, sms, &grid, &warps);
-  const size_t smem = smem_bytes(warps);
+  const size_t smem = smem_bytes(warps, mode);
   const dim3 block(32 * warps);
   switch (mode) {
+    case kDecodeDot: {
+      if (a.rows || !a.x || !a.y || !a.part || !a.row_cnt || a.m < 1 || a.m > kDotMaxM)
+        return cudaErrorInvalidValue;
+      e = set_attrs(decode_kernel<kDecodeDot, false>, smem);
+      if (e == cudaSuccess)
+        e = launch_pdl(decode_kernel<kDecodeDot, false>, grid, block, smem, s, a, out);
+      break;
+    }
     case kDecodeExp:
       if (a.rows) return cudaErrorInvalidValue;
       e = set_attrs(decode_kernel<kDecodeExp, false>, smem);

@@ -38,6 +38,7 @@ struct uw_handle_s {
   uint32_t* d_status = nullptr;
   uint32_t* d_sync = nullptr;    // GEMM split-K hand-off (kGemmSyncWords, zeroed at upload)
   uint8_t* d_pal_idx = nullptr;  // resident palette indices (pipeline 4), may be null
+  uint32_t* d_row_cnt = nullptr; // Huffman-direct product: N row arrival counters (zeroed)
 
   // workspace for pipelines 1-3 and split-K partial sums
   void* ws = nullptr;
@@ -60,6 +61,10 @@ uw_gemm_config choose_variant(const uw_handle_s* h, int64_t M);
 uw_status check_config(const uw_handle_s* h, const uw_gemm_config& cfg);
 bool use_gemv(const uw_gemm_config& c, int64_t M);
 bool gemv_for(const uw_handle_s* h, const uw_gemm_config& cfg, int64_t M);
+// The Huffman-direct product (pipeline 5) serves (handle, M).
+bool dot_for(const uw_handle_s* h, int64_t M);
+// Does the pipeline need a preprocessing pass (pipelines 1-3)?
+inline bool needs_preprocess(int pipeline) { return pipeline >= 1 && pipeline <= 3; }
 size_t preprocessed_bytes(const uw_handle_s* h, int pipeline);
 uw_status plan_gemm(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M,
                     const uw_gemm_config& cfg, int out_f32, GemmArgs* ga, size_t* ws_need,

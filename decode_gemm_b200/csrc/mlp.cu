@@ -109,7 +109,7 @@ uw_status make_plan(const uw_mlp_layer* layers, int32_t n, int64_t M, const uw_m
       if (o.gemm_ctas > 0 && pr.cfg.gemm_ctas == 0) pr.cfg.gemm_ctas = o.gemm_ctas;
       const uw_status st = check_config(hh[j], pr.cfg);
       if (st != UW_OK) return st;
-      pr.hard = pr.cfg.pipeline != UW_PIPE_PALETTE_DIRECT;
+      pr.hard = needs_preprocess(pr.cfg.pipeline);
       GemmArgs a;
       size_t need = 0, pre = 0;
       const uw_status ps = plan_gemm(hh[j], nullptr, nullptr, M, pr.cfg, 0, &a, &need, &pre);

@@ -19,7 +19,9 @@ inline uint64_t wait_limit_ns() {
   return ns;
 }
 
-enum DecodeMode { kDecodeExp = 0, kDecodeFull = 1, kDecodePalette = 2 };
+// kDecodeDot: the Huffman-direct matrix-vector product (no decoded weights
+// leave the chip; see DecodeArgs' product fields).
+enum DecodeMode { kDecodeExp = 0, kDecodeFull = 1, kDecodePalette = 2, kDecodeDot = 3 };
 
 // Zero words that follow the Huffman stream in device memory: a lane decoding
 // a chunk reads at most 12 bits per symbol past the chunk's start plus a
@@ -36,7 +38,7 @@ struct DecodeArgs {
   const uint32_t* canon;      // canonical-code tables (kCanonWords words)
   uint32_t palette[4];        // the 16 palette exponents, byte i = rank i
   uint32_t pal_run_b4;        // palette = the run b..b+15: b in every byte, else 0xFFFFFFFF
-  const uint8_t* sm;          // sign+mantissa bytes (full decode only)
+  const uint8_t* sm;          // sign+mantissa bytes (full decode and product)
   const uint32_t* esc_bits;   // escape bitmap (palette transcode only)
   uint32_t* status;           // device status word (bit 0: bad chunk)
   int64_t n_words;
@@ -53,7 +55,27 @@ struct DecodeArgs {
   int64_t gather_rows = 0;
   int64_t matrix_rows = 0;    // N
   int32_t cpr = 0;
+  // Huffman-direct product (kDecodeDot): Y[t, n] = sum_k X[t, k] W[n, k] for
+  // t < m, computed while the stream decodes; needs K % chunk_syms == 0 and
+  // cpr = K / chunk_syms.  A warp's group is 32 rows at one chunk position
+  // (one column range); each (row, position) leaves m FP32 partial sums at
+  // part[(row * kDotMaxM + t) * cpr + position], and the group that brings a
+  // row's last partial (row_cnt, zero between launches) adds them in position
+  // order and writes Y (BF16 or FP32, [m, N]).
+  const uint16_t* x = nullptr;  // X [m, K] BF16, rows 16-byte aligned
+  void* y = nullptr;
+  int32_t m = 0;
+  int32_t out_f32 = 0;
+  float* part = nullptr;
+  uint32_t* row_cnt = nullptr;
 };
+
+constexpr int kDotMaxM = 8;
+// Whether the product serves (K, chunk_syms, M): rows are whole chunks and
+// 1 <= M <= kDotMaxM.
+bool dot_supported(int64_t K, int64_t chunk_syms, int64_t M);
+// Partial-sum floats of a Huffman-direct launch over n_chunks chunks.
+inline int64_t dot_part_floats(int64_t n_chunks) { return n_chunks * kDotMaxM; }
 
 // Decode/transcode every chunk into `out` (layout per mode: BF16 [N*K],
 // exponent bytes [N*K], packed nibbles [N*K/2]).  ctas > 0 caps the SMs the

@@ -82,7 +82,17 @@ typedef enum uw_pipeline {
   UW_PIPE_FULL = 1,            /* Huffman decode to BF16 in HBM, then plain GEMM         */
   UW_PIPE_EXP = 2,             /* decode exponent bytes to HBM, reconstructive GEMM      */
   UW_PIPE_PALETTE_RT = 3,      /* transcode to 4-bit palette indices, reconstructive GEMM */
-  UW_PIPE_PALETTE_DIRECT = 4   /* palette indices prepared at load, reconstructive GEMM  */
+  UW_PIPE_PALETTE_DIRECT = 4,  /* palette indices prepared at load, reconstructive GEMM  */
+  /* Beyond the four: the Huffman-direct product (*Unweight*, "How the
+   * reconstructive matmul works": decoding inside the matmul moves about 30 %
+   * fewer weight bytes than the palette form).  One kernel decodes the stream
+   * and multiplies the rebuilt BF16 weights with X in warp-level MMAs (FP32
+   * accumulation) as they decode; it reads the stream and the sign+mantissa
+   * bytes (about 1.33 bytes per weight) and writes only Y.  M <= 8; K a
+   * multiple of chunk_syms (UW_ERR_UNSUPPORTED otherwise).  Partial sums live
+   * in the workspace (uw_workspace_bytes); no preprocessing pass.  Calls on
+   * one handle must not overlap on the GPU (row counters in the handle).    */
+  UW_PIPE_HUFFMAN_DIRECT = 5
 } uw_pipeline;
 
 /* Encoder options.  uw_default_encode_opts fills the defaults. */
@@ -144,7 +154,8 @@ typedef struct uw_gemm_config {
   int32_t tile_n;        /* tokens per MMA tile: 16..256, multiple of 16 (0=auto)  */
   int32_t stages;        /* weight load-ring depth, 2..16, even unless halves=2
                             (0 = auto; X tiles have their own, automatic ring)      */
-  int32_t gemm_ctas;     /* persistent GEMM CTAs (0 = one per SM)                   */
+  int32_t gemm_ctas;     /* persistent GEMM CTAs (0 = one per SM); pipeline 5: the
+                            SMs (one CTA each) of its single kernel                 */
   int32_t decode_ctas;   /* SMs (one CTA each) of the preprocessing kernel (0 = all) */
   int32_t halves;        /* W rows per GEMM unit / 128: 1, or 2 (the wide shape: X
                             is read once per 256 rows); 0 = 1                       */
@@ -156,7 +167,9 @@ typedef struct uw_gemm_config {
   int32_t gemv;          /* 1: the matrix-vector kernel on the CUDA cores, M <= 2 only
                             (each weight rebuilt in registers and multiplied in FP32,
                             no tensor cores; UW_ERR_UNSUPPORTED above M = 2); 0: the
-                            tensor-core GEMM.  The autotuner tries 1 at M <= 2      */
+                            tensor-core GEMM.  The autotuner tries 1 at M <= 2.
+                            Pipeline 5 (always on the CUDA cores): must be 0.
+                            Pipeline 5 ignores tile_n, stages, halves, decode_ctas */
 } uw_gemm_config;
 
 typedef struct uw_host_s* uw_host_t;       /* host-side encoded matrix         */
@@ -337,7 +350,8 @@ typedef enum uw_kernel_kind {
   UW_KERNEL_DECODE_FULL = 0, UW_KERNEL_DECODE_EXP = 1, UW_KERNEL_TRANSCODE = 2,
   UW_KERNEL_GEMM_BF16 = 3, UW_KERNEL_GEMM_EXP = 4, UW_KERNEL_GEMM_PALETTE = 5,
   UW_KERNEL_SPLITK_FIXUP = 6,  /* reserved: split tiles are summed inside the GEMM */
-  UW_KERNEL_GEMV_BF16 = 7, UW_KERNEL_GEMV_EXP = 8, UW_KERNEL_GEMV_PALETTE = 9
+  UW_KERNEL_GEMV_BF16 = 7, UW_KERNEL_GEMV_EXP = 8, UW_KERNEL_GEMV_PALETTE = 9,
+  UW_KERNEL_DECODE_DOT = 10  /* the Huffman-direct product (UW_PIPE_HUFFMAN_DIRECT) */
 } uw_kernel_kind;
 UW_API uw_status uw_trace_enable(uw_handle_t h, int32_t enable);
 UW_API uw_status uw_trace_read(uw_handle_t h, int32_t* kinds, float* ms, int32_t capacity,
