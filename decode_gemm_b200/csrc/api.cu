@@ -174,6 +174,9 @@ uw_status run_dot_on(uw_handle_s* h, const uint16_t* X, void* Y, int64_t M, int 
   a.out_f32 = out_f32;
   a.part = part;
   a.row_cnt = h->d_row_cnt;
+  // (from the device's SM count, not the launch's: the summation order, and so
+  // the result, does not depend on an SM budget)
+  a.run = dot_run_length(h->N, a.cpr, h->sm_count);
   const int slot = trace_begin(h, UW_KERNEL_DECODE_DOT);
   const cudaError_t e = launch_decode(kDecodeDot, a, nullptr, ctas, s);
   trace_end(h, slot);

@@ -290,7 +290,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   const uint32_t b4 = a.pal_run_b4;
   const int64_t grid_warps = (int64_t)gridDim.x * n_warps;
 
-  for (int64_t grp = (int64_t)blockIdx.x * n_warps + warp; grp < groups; grp += grid_warps) {
+  // A warp takes runs of G consecutive groups (the product: G chunk positions
+  // of the same 32 rows, whose sums carry over; every other mode: G = 1).
+  const int G = MODE == kDecodeDot ? a.run : 1;
+  const int64_t n_runs = (groups + G - 1) / G;
+  bool fixed = false;  // (product) a correction was made in this run
+  for (int64_t run = (int64_t)blockIdx.x * n_warps + warp; run < n_runs; run += grid_warps)
+  for (int64_t grp = run * G; grp < (run + 1) * G && grp < groups; ++grp) {
+    const bool run_first = grp == run * G;
+    const bool run_last = grp + 1 == (run + 1) * G || grp + 1 == groups;
     const int64_t c0 = grp * 32;
     const int64_t c = c0 + lane;
     // product: rows rb*32 .. rb*32+31 (lane = row), chunk position cc
@@ -334,7 +342,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
       int64_t cn = c + grid_warps * 32;
       bool next = cn < a.n_chunks;
       if (MODE == kDecodeDot) {
-        const int64_t g2 = grp + grid_warps, rb2 = g2 / a.cpr;
+        const int64_t g2 = run_last ? (run + grid_warps) * G : grp + 1, rb2 = g2 / a.cpr;
         cn = (rb2 * 32 + lane) * a.cpr + (g2 - rb2 * a.cpr);
         next = g2 < groups && rb2 * 32 + lane < a.matrix_rows;
       }
@@ -372,12 +380,14 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     // and the lane's corrections (dcorr: the true weights' products at its
     // chunk's exceptions, per token) live in shared memory.
     int dirty_from = kNoRound;
-    bool fixed = false;  // a correction was made
     if (MODE == kDecodeDot) {
 #pragma unroll
       for (int q = 0; q < kExcCap; ++q) exc[q] = 0xFFFFFFFFu;
+      if (run_first) {
 #pragma unroll
-      for (int v = 0; v < 4; ++v) reinterpret_cast<float4*>(dsum)[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = 0; v < 4; ++v) reinterpret_cast<float4*>(dsum)[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        fixed = false;
+      }
     }
     // BF16 weight w times X[t, column col] into this lane's correction
     // (the product of two BF16 is exact in FP32)
@@ -722,13 +732,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     if (live && (bad || bits_pos(b) != end)) atomicOr(a.status, kStatusBadChunk);
     __syncwarp();
 
-    if (MODE == kDecodeDot) {
+    if (MODE == kDecodeDot && run_last) {
       // Lane (g, t) holds the sums of rows 16 bk + g + 8 h (dsum[4 bk + 2 h +
       // e]) for tokens 2t + e; with the owners' corrections added they are
-      // the group's partial sums, stored at part[(row * kDotMaxM + token) *
-      // cpr + cc].  The group that brings a row's cpr-th partial adds them in
-      // chunk order and writes Y.
+      // the run's partial sums, stored at part[(row * kDotMaxM + token) * S +
+      // segment] (S = cpr / G segments per row, this run's is cc / G).  The
+      // run that brings a row's S-th partial adds them in segment order and
+      // writes Y.
       const int g = lane >> 2, tq = lane & 3;
+      const int nseg = a.cpr / G;
       const bool any_corr = __any_sync(0xffffffffu, fixed);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -737,25 +749,25 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         float v = dsum[k];
         if (any_corr && t < a.m) v += dsum_w[j * 16 + 8 + t];  // row j's owner's correction
         const int64_t row = rb * 32 + j;
-        if (t < a.m && row < a.matrix_rows) a.part[(row * kDotMaxM + t) * a.cpr + cc] = v;
+        if (t < a.m && row < a.matrix_rows) a.part[(row * kDotMaxM + t) * nseg + cc / G] = v;
       }
       __threadfence();
       __syncwarp();
       const int64_t row = rb * 32 + lane;  // lane l: row l of the group
-      if (row < a.matrix_rows && atomicAdd(a.row_cnt + row, 1u) == (uint32_t)(a.cpr - 1)) {
+      if (row < a.matrix_rows && atomicAdd(a.row_cnt + row, 1u) == (uint32_t)(nseg - 1)) {
         __threadfence();
         for (int t = 0; t < a.m; ++t) {
           // the row's partials for token t are contiguous: loaded four at a
           // time when they can be, added in chunk order
-          const float* pt = a.part + (row * kDotMaxM + t) * a.cpr;
+          const float* pt = a.part + (row * kDotMaxM + t) * nseg;
           float y = 0.f;
           int q = 0;
-          if ((a.cpr & 3) == 0)
-            for (; q < a.cpr; q += 4) {
+          if ((nseg & 3) == 0)
+            for (; q < nseg; q += 4) {
               const float4 v = __ldcg(reinterpret_cast<const float4*>(pt + q));
               y = y + v.x + v.y + v.z + v.w;
             }
-          for (; q < a.cpr; ++q) y += __ldcg(pt + q);
+          for (; q < nseg; ++q) y += __ldcg(pt + q);
           const int64_t o = (int64_t)t * a.matrix_rows + row;
           if (a.out_f32)
             static_cast<float*>(a.y)[o] = y;
@@ -780,6 +792,16 @@ cudaError_t set_attrs(F* f, size_t smem) {
 }
 
 }  // namespace
+
+// The longest run (a divisor of cpr) that still leaves about 24 runs per SM,
+// so a launch keeps its warps busy in one pass.
+int dot_run_length(int64_t N, int64_t cpr, int sms) {
+  const int64_t groups = (N + 31) / 32 * cpr;
+  int best = 1;
+  for (int G = 2; G <= 8 && G <= cpr; ++G)
+    if (cpr % G == 0 && groups / G >= (int64_t)sms * 24) best = G;
+  return best;
+}
 
 bool dot_supported(int64_t K, int64_t chunk_syms, int64_t M) {
   return chunk_syms > 0 && K % chunk_syms == 0 && M >= 1 && M <= kDotMaxM;
@@ -830,12 +852,15 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cu
   if (e != cudaSuccess) return e;
   if (ctas > 0 && ctas < sms) sms = ctas;  // an SM budget (decoder/GEMM split)
   int grid = 0, warps = 0;
-  decode_launch_shape(a.n_chunks, sms, &grid, &warps);
+  // (the product's work items are its runs)
+  decode_launch_shape(mode == kDecodeDot ? (a.matrix_rows + 31) / 32 * a.cpr / a.run * 32 : a.n_chunks,
+                      sms, &grid, &warps);
   const size_t smem = smem_bytes(warps, mode);
   const dim3 block(32 * warps);
   switch (mode) {
     case kDecodeDot: {
-      if (a.rows || !a.x || !a.y || !a.part || !a.row_cnt || a.m < 1 || a.m > kDotMaxM)
+      if (a.rows || !a.x || !a.y || !a.part || !a.row_cnt || a.m < 1 || a.m > kDotMaxM ||
+          a.run < 1 || a.cpr % a.run)
         return cudaErrorInvalidValue;
       e = set_attrs(decode_kernel<kDecodeDot, false>, smem);
       if (e == cudaSuccess)

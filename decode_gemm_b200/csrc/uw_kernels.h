@@ -58,22 +58,27 @@ struct DecodeArgs {
   // Huffman-direct product (kDecodeDot): Y[t, n] = sum_k X[t, k] W[n, k] for
   // t < m, computed while the stream decodes; needs K % chunk_syms == 0 and
   // cpr = K / chunk_syms.  A warp's group is 32 rows at one chunk position
-  // (one column range); each (row, position) leaves m FP32 partial sums at
-  // part[(row * kDotMaxM + t) * cpr + position], and the group that brings a
-  // row's last partial (row_cnt, zero between launches) adds them in position
-  // order and writes Y (BF16 or FP32, [m, N]).
+  // (one column range); a warp takes runs of `run` groups (consecutive
+  // positions of the same rows, run divides cpr), and each (row, run) leaves
+  // m FP32 partial sums at part[(row * kDotMaxM + t) * (cpr / run) + segment];
+  // the run that brings a row's last partial (row_cnt, zero between
+  // launches) adds them in segment order and writes Y (BF16 or FP32, [m, N]).
   const uint16_t* x = nullptr;  // X [m, K] BF16, rows 16-byte aligned
   void* y = nullptr;
   int32_t m = 0;
   int32_t out_f32 = 0;
   float* part = nullptr;
   uint32_t* row_cnt = nullptr;
+  int32_t run = 1;
 };
 
 constexpr int kDotMaxM = 8;
 // Whether the product serves (K, chunk_syms, M): rows are whole chunks and
 // 1 <= M <= kDotMaxM.
 bool dot_supported(int64_t K, int64_t chunk_syms, int64_t M);
+// Chunk positions per run of the product for an N x (cpr chunks) matrix on
+// `sms` SMs (decode.cu).
+int dot_run_length(int64_t N, int64_t cpr, int sms);
 // Partial-sum floats of a Huffman-direct launch over n_chunks chunks.
 inline int64_t dot_part_floats(int64_t n_chunks) { return n_chunks * kDotMaxM; }
 

@@ -169,13 +169,27 @@ def test_hdot_deterministic_over_grid_sizes(uw):
 
 
 def test_hdot_full_size(uw):
-    """The 8B gate and down shapes at M = 1 and 8 against FP64."""
+    """The 8B gate and down shapes (where a warp carries its sums over runs of
+    chunk positions) at M = 1 and 8 against FP64, one-hot columns exactly, and
+    bitwise equal over SM budgets."""
     for name in ("gate_14336x4096", "down_4096x14336"):
         w = synthdata.workload(name)
+        K = w.shape[1]
         h, ws = _setup(uw, w, 256)
         for M in (1, 8):
             x = synthdata.activation_for(name, M)
-            _check(_run(uw, h, x), x, w)
+            y = _run(uw, h, x)
+            _check(y, x, w)
+            if M == 1:
+                for ctas in (37, 148):
+                    assert np.array_equal(_run(uw, h, x, gemm_ctas=ctas), y)
+        ks = [0, 255, 256, 257, 4095, K - 257, K - 256, K - 1]
+        xo = np.zeros((8, K), np.uint16)
+        for t, k in enumerate(ks):
+            xo[t, k] = 0x3F80
+        yo = _run(uw, h, xo)
+        for t, k in enumerate(ks):
+            assert np.array_equal(yo[t], oracle.to_float64(w[:, k])), f"{name} column {k}"
         h.free()
 
 
