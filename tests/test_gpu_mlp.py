@@ -143,7 +143,10 @@ SPLITS = {
     "overlap_decode4_gemm100": dict(overlap=True, decode_ctas=4, gemm_ctas=100),
     "serial_gemm60": dict(overlap=False, gemm_ctas=60),
     "overlap_matvec": dict(overlap=True),  # every projection on the matrix-vector kernel
+    "overlap_hdot": dict(overlap=True),  # pipeline 5 mixed in (HDOT_PIPES)
 }
+# the Huffman-direct product (pipeline 5, no preprocessing) among hard and easy projections
+HDOT_PIPES = [(5, 4, 2), (3, 5, 5), (5, 5, 4)]
 
 
 @pytest.mark.parametrize("M", [1, 2, 24])
@@ -158,8 +161,9 @@ def test_mlp_stack_projections_against_fp64(uw, M, split):
     gemv = 1 if split == "overlap_matvec" else 0
     if gemv and M > 2:
         pytest.skip("the matrix-vector kernel serves M <= 2")
-    layers, weights = _layers(uw, 3, PIPES)
-    _load_pipelines(uw, layers, PIPES, M, gemv=gemv)
+    pipes = HDOT_PIPES if split == "overlap_hdot" else PIPES
+    layers, weights = _layers(uw, 3, pipes)
+    _load_pipelines(uw, layers, pipes, M, gemv=gemv)
     x = synthdata.activations(M, D, seed=160 + M)
     X = torch.from_numpy(x.view(np.int16)).cuda()
     side = torch.cuda.Stream()
@@ -180,7 +184,7 @@ def test_mlp_stack_projections_against_fp64(uw, M, split):
         for name, out, inp, w in (("gate", g, cur, wg), ("up", u, cur, wu), ("down", nxt, hh, wd)):
             ok, worst = oracle.within_tolerance(oracle.to_float64(out), oracle.gemm_fp64(inp, w),
                                                 oracle.abs_product_sum(inp, w), bf16_output=True)
-            assert ok, (split, l, name, PIPES[l], worst)
+            assert ok, (split, l, name, pipes[l], worst)
         ref = oracle.swiglu(g, u)
         assert np.all(np.abs(oracle.to_float64(hh) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
         cur = nxt
