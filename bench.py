@@ -60,9 +60,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum of one launch), valid only while the kernel source
 # (src_sha, see _kernel_src_sha) is unchanged.
 TRAFFIC = {
-    "gemm_palette": {"bytes_per_launch": 89.758976e6 + 2.869504e6, "src_sha": "0bd3631b51fba772",
+    "gemm_palette": {"bytes_per_launch": 89.683968e6 + 2.589440e6, "src_sha": "0bd3631b51fba772",
                      "capture": "palette GEMM, 14336x4096, M = 1 launch"},
-    "decode_full": {"bytes_per_launch": 87.158272e6 + 64.990720e6, "src_sha": "97266aa6e257b3ca",
+    "decode_full": {"bytes_per_launch": 87.146496e6 + 65.034496e6, "src_sha": "ee028cbb4583e97d",
                     "capture": "full decode, 14336x4096 (output partly still in L2)"},
 }
 
