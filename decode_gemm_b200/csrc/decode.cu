@@ -35,6 +35,12 @@
 //     128-symbol round the warp writes its 32 chunks' outputs with 128-bit
 //     stores, each warp-wide store covering contiguous, fully used lines.
 //     Shared memory stays small so L1 can hold every lane's stream lines.
+//   * The Huffman-direct product (kDecodeDot; *Unweight*, "How the
+//     reconstructive matmul works": decoding inside the matmul) keeps the
+//     decode and replaces the write-out: a warp's 32 chunks are one chunk
+//     position of 32 rows, and each decoded round is multiplied with X in
+//     warp-level BF16 MMAs (FP32 accumulation) while the weights are still
+//     in registers; only Y leaves the chip.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
