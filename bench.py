@@ -87,8 +87,9 @@ def _args():
                     help="time uw_mlp_forward over this many gate/up/down layers")
     ap.add_argument("--mlp-ms", default="1,64,256,1024")
     ap.add_argument("--mlp-force-down", default="",
-                    help="comma list of pipelines (2, 3, or 5 at M <= 8) to force on every down_proj, gate/up "
-                         "on pipeline 4: times the stack with the preprocessing overlap off, "
+                    help="comma list of pipelines (2, 3, or 5 at M <= 8) to force on every "
+                         "down_proj, gate/up on pipeline 4: times the stack with the preprocessing "
+                         "overlap off, "
                          "on, and with the tuned decoder/GEMM SM split")
     return ap.parse_args()
 
