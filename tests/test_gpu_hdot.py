@@ -254,3 +254,32 @@ def test_hdot_autotune_candidate(uw):
         assert uw.uw_last_device_status(h) == uw.UW_OK
         _check(Y.cpu().numpy().astype(np.float64), x, w)
     h.free()
+
+
+def test_hdot_corrupt_stream_reports_device_status(uw):
+    """Flipped stream bits (the format still valid) run through the product
+    without faulting and are reported like the decoders report them; the row
+    counters are left clean, so the next call on a sound handle is exact."""
+    import torch
+    N, K = 64, 1024
+    w = synthdata.normal(N, K, 0.02, seed=360)
+    a = uw.uw_encode_host(w, uw.default_opts(chunk_syms=64)).arrays()
+    words = a["words"].copy()
+    words[7] ^= 0x00F0F000
+    words[90] ^= 0x12345678
+    b = uw.FormatBuffers(N, K, 12, 64, a["code_len"], a["palette"], words, a["chunk_off"],
+                         a["sm"], a["esc_bits"], a["esc_off"], a["esc_exp"])
+    assert uw.uw_validate_format(b.fmt) == uw.UW_OK
+    h = uw.uw_upload(b.fmt, uw.default_opts(chunk_syms=64, prepare_direct=0))
+    ws = torch.empty(uw.uw_workspace_bytes(h, uw.UW_PIPE_HUFFMAN_DIRECT, 1), dtype=torch.uint8,
+                     device="cuda")
+    uw.uw_set_workspace(h, ws)
+    x = synthdata.activations(2, K, seed=361)
+    X = torch.from_numpy(x.view(np.int16)).cuda()
+    Y = torch.empty((2, N), dtype=torch.float32, device="cuda")
+    uw.uw_gemm_ex(h, X, Y, 2, uw.gemm_config(uw.UW_PIPE_HUFFMAN_DIRECT), True)
+    assert uw.uw_last_device_status(h) == uw.UW_ERR_DEVICE
+    h.free()
+    h2, ws2 = _setup(uw, w, 64)
+    _check(_run(uw, h2, x), x, w)
+    h2.free()
