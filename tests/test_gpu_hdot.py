@@ -258,8 +258,8 @@ def test_hdot_autotune_candidate(uw):
 
 def test_hdot_corrupt_stream_reports_device_status(uw):
     """Flipped stream bits (the format still valid) run through the product
-    without faulting and are reported like the decoders report them; the row
-    counters are left clean, so the next call on a sound handle is exact."""
+    without faulting and are reported like the decoders report them; the
+    process goes on to an exact product on a sound handle."""
     import torch
     N, K = 64, 1024
     w = synthdata.normal(N, K, 0.02, seed=360)
