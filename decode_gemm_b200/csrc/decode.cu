@@ -65,6 +65,9 @@ constexpr int kExcCap = 4;                      // exceptions held per lane
 constexpr int kFullPair = 2 * 4 * kPalCap;      // 4x symbols two whole lookups may yield
 constexpr int kFullOne = 4 * kPalCap;
 constexpr int kNoRound = 1 << 30;
+// The product runs at most 25 warps per CTA: 72 registers a thread instead of
+// 64 (fewer spills; measured 3 % faster than a 32-warp bound).
+constexpr int kDotMaxWarps = 25;
 
 
 // Shared memory: the tables, then per warp its ranks stage (32 lanes x 17
@@ -255,7 +258,7 @@ __device__ __forceinline__ void pack(Packer& pk, uint32_t e, uint32_t c4) {
 // DOT (the Huffman-direct product): the write-out becomes a matrix product of
 // the rebuilt weights with X; nothing but Y leaves the chip.
 template <int MODE, bool GATHER>
-__global__ void __launch_bounds__(32 * kMaxWarps, 1)
+__global__ void __launch_bounds__(32 * (MODE == kDecodeDot ? kDotMaxWarps : kMaxWarps), 1)
     decode_kernel(const DecodeArgs a, void* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SmemHead& sm = *reinterpret_cast<SmemHead*>(smem_raw);
@@ -818,7 +821,7 @@ bool dot_supported(int64_t K, int64_t chunk_syms, int64_t M) {
 // issue slots, so W is chosen in [16, 32] to minimise passes x W (the last
 // pass nearly full); a problem too small to give every SM 16 warps spreads
 // over more SMs with fewer warps instead.
-void decode_launch_shape(int64_t n_chunks, int sms, int* ctas, int* warps) {
+void decode_launch_shape(int64_t n_chunks, int sms, int* ctas, int* warps, int max_w) {
   const int64_t groups = (n_chunks + 31) / 32;
   if (sms < 1) sms = 1;
   if (groups <= (int64_t)sms * kMinWarps) {
@@ -827,9 +830,9 @@ void decode_launch_shape(int64_t n_chunks, int sms, int* ctas, int* warps) {
     *ctas = (int)((groups + w - 1) / w);
     return;
   }
-  int best_w = kMaxWarps;
+  int best_w = max_w;
   int64_t best_cost = -1;
-  for (int w = kMaxWarps; w >= kMinWarps; --w) {
+  for (int w = max_w; w >= kMinWarps; --w) {
     const int64_t per = (int64_t)sms * w;
     const int64_t cost = (groups + per - 1) / per * w;
     if (best_cost < 0 || cost < best_cost) {
@@ -860,7 +863,7 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cu
   int grid = 0, warps = 0;
   // (the product's work items are its runs)
   decode_launch_shape(mode == kDecodeDot ? (a.matrix_rows + 31) / 32 * a.cpr / a.run * 32 : a.n_chunks,
-                      sms, &grid, &warps);
+                      sms, &grid, &warps, mode == kDecodeDot ? kDotMaxWarps : kMaxWarps);
   const size_t smem = smem_bytes(warps, mode);
   const dim3 block(32 * warps);
   switch (mode) {

@@ -88,8 +88,9 @@ inline int64_t dot_part_floats(int64_t n_chunks) { return n_chunks * kDotMaxM; }
 // launch error.
 cudaError_t launch_decode(int mode, const DecodeArgs& a, void* out, int ctas, cudaStream_t s);
 int decode_ctas_needed(int64_t n_chunks);
-// CTAs and warps per CTA of a decode over n_chunks chunks on `sms` SMs.
-void decode_launch_shape(int64_t n_chunks, int sms, int* ctas, int* warps);
+// CTAs and warps per CTA (at most max_w) of a decode over n_chunks chunks on
+// `sms` SMs.
+void decode_launch_shape(int64_t n_chunks, int sms, int* ctas, int* warps, int max_w = 32);
 
 // Device status bits.
 constexpr uint32_t kStatusBadChunk = 1u;
