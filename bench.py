@@ -60,9 +60,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum of one launch), valid only while the kernel source
 # (src_sha, see _kernel_src_sha) is unchanged.
 TRAFFIC = {
-    "gemm_palette": {"bytes_per_launch": 89.683968e6 + 2.589440e6, "src_sha": "0bd3631b51fba772",
+    "gemm_palette": {"bytes_per_launch": 89.744128e6 + 2.605312e6, "src_sha": "0bd3631b51fba772",
                      "capture": "palette GEMM, 14336x4096, M = 1 launch"},
-    "decode_full": {"bytes_per_launch": 87.146496e6 + 65.034496e6, "src_sha": "ee028cbb4583e97d",
+    "decode_full": {"bytes_per_launch": 87.244288e6 + 64.507392e6, "src_sha": "d12398d63b87327d",
                     "capture": "full decode, 14336x4096 (output partly still in L2)"},
 }
 
