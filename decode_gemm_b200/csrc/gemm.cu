@@ -1171,9 +1171,10 @@ int tmem_cols_for(int tile_n, int w_cols) {
 // then reads A from there, and the shared-memory W ring becomes load stages);
 // 0 when W goes through shared memory.  Needs one half per unit and the slots
 // (32 columns per K block) beside the accumulators.  Two K blocks per unit
-// when K allows: the load time is set by the number of TMA boxes more than by
-// their bytes (pure load streams of the 14336x4096 palette form: 35 us with
-// one K block per stage, 26 us with two).
+// when K allows: the ring then holds twice the bytes in flight in the same
+// number of stages (pure load streams of the 14336x4096 palette form: 35 us
+// with one K block per stage, 26 us with two; with 64 KB or more in flight per
+// SM every box shape and layout measured the same).
 int tmem_ks_for(const GemmArgs& a) {
   if (a.mode == kGemmBf16 || a.halves != 1) return 0;
   const int acc = 2 * mma_warps_for(a.tile_n) * a.tile_n;
