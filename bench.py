@@ -62,7 +62,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     "gemm_palette": {"bytes_per_launch": 89.744128e6 + 2.605312e6, "src_sha": "0bd3631b51fba772",
                      "capture": "palette GEMM, 14336x4096, M = 1 launch"},
-    "decode_full": {"bytes_per_launch": 87.244288e6 + 64.507392e6, "src_sha": "d12398d63b87327d",
+    "decode_full": {"bytes_per_launch": 87.415040e6 + 64.024064e6, "src_sha": "2a78f2d845afbc82",
                     "capture": "full decode, 14336x4096 (output partly still in L2)"},
 }
 
