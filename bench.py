@@ -55,6 +55,7 @@ N_SETS = 4
 REF_ROWS = 48             # oracle rows per reference-arm step (~2 s of CPU work)
 CPU_BASELINE_ROWS = 300   # oracle rows for the cpu_baseline leg (~12 s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e, nominal (HGX)
 
 # DRAM traffic per launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum of one launch), valid only while the kernel source
@@ -795,7 +796,9 @@ def run_ours(args):
                 # no overlap with its neighbours; includes each launch's own
                 # start-up): the isolated figure beside the back-to-back one
                 "frac_traced": (d["bytes"] / (d["ms"] * 1e-3) / 1e9) / peaks["hbm_gbs"],
-                "peak_source": peak_src}
+                "peak_source": peak_src,
+                # against the nominal HBM3e figure (HGX), for context beside the measured peak
+                "frac_nominal": achieved / NOMINAL_HBM_GBS}
     kernels = {k: {"launches": v["n"], "total_ms": v["ms"], "share": v["ms"] / traced_ms,
                    "GBps": v["bytes"] / (v["ms"] * 1e-3) / 1e9 if v["ms"] > 0 else None,
                    "frac_hbm": (v["bytes"] / (v["ms"] * 1e-3) / 1e9) / peaks["hbm_gbs"]
