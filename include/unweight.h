@@ -237,8 +237,10 @@ UW_API uw_status uw_stats(uw_handle_t h, uw_stats_t* out);
 
 /* Workspace: pipelines FULL, EXP and PALETTE_RT write their preprocessed
  * weights (2*N*K, N*K, N*K/2 bytes) and the GEMM its split-K partial sums to a
- * device workspace.  uw_workspace_bytes gives a size that serves (pipeline, M)
- * with any variant (token tile up to 256, up to one CTA per SM);
+ * device workspace; HUFFMAN_DIRECT keeps its per-row partial sums there
+ * (32 bytes per chunk of the stream).  uw_workspace_bytes gives a size that
+ * serves (pipeline, M) with any variant (token tile up to 256, up to one CTA
+ * per SM), or UW_ERR_UNSUPPORTED where the pipeline does not serve M;
  * uw_set_workspace registers caller-owned device memory (kept by pointer until
  * replaced or the handle is freed; ptr NULL unregisters); uw_alloc_workspace
  * makes the handle allocate and own one of `bytes` bytes.  Calls that need
