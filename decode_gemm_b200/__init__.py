@@ -33,7 +33,7 @@ UW_ERR_OOM, UW_ERR_CUDA, UW_ERR_DEVICE, UW_ERR_TIMEOUT, UW_ERR_WORKSPACE = 5, 6,
 UW_ERR_IO = 10
 UW_PIPE_AUTO, UW_PIPE_FULL, UW_PIPE_EXP, UW_PIPE_PALETTE_RT, UW_PIPE_PALETTE_DIRECT = 0, 1, 2, 3, 4
 UW_PIPE_HUFFMAN_DIRECT = 5   # the Huffman-direct product (M <= DOT_MAX_M)
-DOT_MAX_M = 4
+DOT_MAX_M = 8     # tokens the Huffman-direct product serves per call
 PIPELINES = {"full": UW_PIPE_FULL, "exp": UW_PIPE_EXP, "palette_rt": UW_PIPE_PALETTE_RT,
              "palette_direct": UW_PIPE_PALETTE_DIRECT}
 
