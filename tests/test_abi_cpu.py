@@ -25,10 +25,13 @@ def uw():
     return decode_gemm_b200
 
 
-def _declared_functions():
+def _header_text():
     text = open(os.path.join(ROOT, "include", "unweight.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(uw_[a-z0-9_]+)\s*\(", text)))
+    return re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+
+
+def _declared_functions():
+    return sorted(set(re.findall(r"\b(uw_[a-z0-9_]+)\s*\(", _header_text())))
 
 
 def test_library_exports_every_declared_symbol(uw):
@@ -43,6 +46,48 @@ def test_library_exports_every_declared_symbol(uw):
     assert exported <= set(declared), sorted(exported - set(declared))
     for name in declared:
         assert hasattr(uw.lib, name)
+
+
+def test_binding_constants_match_header(uw):
+    """Status codes, pipeline ids and trace kinds in the binding are the header's values."""
+    vals = {n: int(v) for n, v in re.findall(r"\b(UW_[A-Z0-9_]+)\s*=\s*(\d+)", _header_text())}
+    status = [n for n in vals if n == "UW_OK" or n.startswith("UW_ERR_")]
+    pipes = [n for n in vals if n.startswith("UW_PIPE_")]
+    kinds = [n for n in vals if n.startswith("UW_KERNEL_")]
+    assert len(status) == 11 and len(pipes) == 6 and len(kinds) == 11
+    for n in status + pipes:
+        assert getattr(uw, n) == vals[n], n
+    assert len(uw.KERNEL_KINDS) == len(kinds)
+    for n in kinds:
+        assert uw.KERNEL_KINDS[vals[n]] == n[len("UW_KERNEL_"):].lower(), n
+
+
+_STRUCTS = ("uw_encode_opts", "uw_format", "uw_stats_t", "uw_gemm_config", "uw_mlp_layer",
+            "uw_mlp_opts")
+
+
+def test_binding_structs_match_header(uw, tmp_path):
+    """Each ctypes mirror has the C compiler's size and field offsets for the header's struct."""
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "unweight.h"', "int main(void) {"]
+    for s in _STRUCTS:
+        lines.append(f'  printf("{s} %zu\\n", sizeof({s}));')
+        for f, _ in getattr(uw, s)._fields_:
+            lines.append(f'  printf("{s}.{f} %zu %zu\\n", offsetof({s}, {f}), '
+                         f"sizeof((({s}*)0)->{f}));")
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe)], check=True)
+    got = dict(l.split(" ", 1) for l in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                      check=True).stdout.splitlines())
+    for s in _STRUCTS:
+        cls = getattr(uw, s)
+        assert int(got[s]) == C.sizeof(cls), s
+        for f, t in cls._fields_:
+            off, size = map(int, got[f"{s}.{f}"].split())
+            assert (off, size) == (getattr(cls, f).offset, C.sizeof(t)), (s, f)
 
 
 def test_status_strings(uw):
