@@ -197,6 +197,17 @@ uw_status uw_host_load(const char* path, uw_host_t* out) {
   uw_host_view(h, &v);
   st = uw_validate_format(&v);
   if (st == UW_OK && (int64_t)e.sm.size() != e.N * e.K) st = UW_ERR_FORMAT;
+  // the stored histogram (statistics only) must count the N*K exponents, every
+  // counted exponent having a code
+  if (st == UW_OK) {
+    int64_t total = 0;
+    for (int s = 0; s < 256 && st == UW_OK; ++s) {
+      const int64_t c = e.hist[s];
+      if (c < 0 || c > e.N * e.K || (c > 0 && e.code_len[s] == 0)) st = UW_ERR_FORMAT;
+      total += c;
+    }
+    if (st == UW_OK && total != e.N * e.K) st = UW_ERR_FORMAT;
+  }
   if (st != UW_OK) {
     delete h;
     return st;

@@ -208,7 +208,8 @@ UW_API uw_status uw_host_stats(uw_host_t h, uw_stats_t* out);
  * histogram, array sizes), the arrays of uw_format in their order, then a 64-bit
  * FNV-1a checksum of all preceding bytes and an end tag.  uw_host_load reads such
  * a file into a new host encoding (owned by the caller: uw_host_free) after
- * checking the tag, the checksum, the header and uw_validate_format.  Errors:
+ * checking the tag, the checksum, the header, uw_validate_format, and that the
+ * histogram counts the N*K exponents with a code for every counted one.  Errors:
  * UW_ERR_ARG (null), UW_ERR_IO (open, read or write failed), UW_ERR_FORMAT
  * (truncated, corrupted or not a bundle), UW_ERR_SHAPE, UW_ERR_OOM. */
 UW_API uw_status uw_host_save(uw_host_t h, const char* path);

@@ -124,6 +124,46 @@ def test_valid_checksum_invalid_content_refused(uw, tmp_path):
     assert e.value.status in (uw.UW_ERR_FORMAT, uw.UW_ERR_SHAPE)
 
 
+def _rechecksum(bad):
+    body = len(bad) - 16
+    h = 14695981039346656037
+    for byte in bad[:body]:
+        h = ((h ^ byte) * 1099511628211) & (2**64 - 1)
+    bad[body:body + 8] = h.to_bytes(8, "little")
+    return bytes(bad)
+
+
+HIST_AT = 320  # the header's int64 exponent histogram: 8 magic + 8 + 16 + 8 + 256 + 16 + 8 bytes in
+
+
+@pytest.mark.parametrize("how", ["negative", "moved", "uncoded", "over"])
+def test_histogram_must_match_the_matrix(uw, tmp_path, how):
+    """The stored histogram only feeds the statistics, but a file whose histogram
+    does not count the matrix's N*K exponents (each with a code) is refused."""
+    path, raw = _saved(uw, tmp_path)
+    he = uw.uw_host_load(path)
+    code_len = he.arrays()["code_len"]
+    hist = np.frombuffer(raw, dtype="<i8", count=256, offset=HIST_AT).copy()
+    assert hist.sum() == 200 * 320 and np.all((hist > 0) <= (code_len > 0))
+    a, b = [int(s) for s in np.flatnonzero(hist)[:2]]
+    if how == "negative":
+        hist[a], hist[b] = -1, hist[b] + hist[a] + 1      # total kept
+    elif how == "moved":
+        hist[a] -= 1                                       # total one short
+    elif how == "uncoded":
+        z = int(np.flatnonzero(code_len == 0)[0])
+        hist[a] -= 1
+        hist[z] += 1                                       # total kept, uncoded exponent
+    else:
+        hist[a] += 2**62                                   # above N*K
+    bad = bytearray(raw)
+    bad[HIST_AT:HIST_AT + 2048] = hist.astype("<i8").tobytes()
+    open(path, "wb").write(_rechecksum(bad))
+    with pytest.raises(uw.UwError) as e:
+        uw.uw_host_load(path)
+    assert e.value.status == uw.UW_ERR_FORMAT
+
+
 def test_io_errors(uw, tmp_path):
     w = synthdata.normal(64, 64, 0.02, seed=66)
     he = uw.uw_encode_host(w)
