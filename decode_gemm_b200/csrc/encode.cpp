@@ -271,7 +271,7 @@ uw_status encode_host(const uint16_t* w, int64_t N, int64_t K, const uw_encode_o
     for (int64_t c = 0; c < C; ++c) {
       e.chunk_off[c] = (uint32_t)acc;
       acc += cbits[c];
-      if (acc >= (uint64_t(1) << 32)) return UW_ERR_UNSUPPORTED;
+      if (acc > (uint64_t)kMaxStreamWords * 32) return UW_ERR_UNSUPPORTED;
     }
     e.chunk_off[C] = (uint32_t)acc;
     e.total_bits = acc;
@@ -516,6 +516,7 @@ uw_status uw_validate_format(const uw_format* f) {
   const int64_t C = (T + f->chunk_syms - 1) / f->chunk_syms;
   if (f->n_chunks != C) return UW_ERR_FORMAT;
   if (f->n_words < 0 || f->n_words % 4) return UW_ERR_FORMAT;
+  if (f->n_words > kMaxStreamWords) return UW_ERR_UNSUPPORTED;
   if (f->chunk_off[0] != 0) return UW_ERR_FORMAT;
   if ((uint64_t)f->chunk_off[C] > (uint64_t)f->n_words * 32) return UW_ERR_FORMAT;
   for (int64_t c = 0; c < C; ++c) {

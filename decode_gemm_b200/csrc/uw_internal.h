@@ -13,6 +13,8 @@ constexpr int kRow = 64;            // weights per escape row
 constexpr int kEscGroupRows = 128;  // rows per escape-row group (one GEMM row tile)
 constexpr int kLutBits = 12;        // decode-table index width (= largest code length)
 constexpr int kLutSize = 1 << kLutBits;
+// Largest stream: the kernels count the stream's bits, padding words included, in 32 bits
+constexpr int64_t kMaxStreamWords = (int64_t(1) << 27) - 4;
 
 // Decode-table entry (one u32 per 12-bit window of the stream).  The table
 // decodes to 4-bit palette ranks; all three preprocessing outputs derive from

@@ -187,7 +187,8 @@ UW_API void uw_default_encode_opts(uw_encode_opts* opts);
  * optimal length-limited code lengths (package-merge, cap max_code_len),
  * canonical codes, chunked bitstream with bit offsets, S stream.
  * Errors: UW_ERR_ARG (null), UW_ERR_SHAPE (N<1, K<64, K%64), UW_ERR_UNSUPPORTED
- * (stream >= 2^32 bits), UW_ERR_OOM.  *out is owned by the caller: uw_host_free. */
+ * (stream above 2^32 - 128 bits), UW_ERR_OOM.  *out is owned by the caller:
+ * uw_host_free. */
 UW_API uw_status uw_encode_host(const uint16_t* w_host, int64_t N, int64_t K,
                          const uw_encode_opts* opts, uw_host_t* out);
 /* Fill *view with pointers into h (valid until uw_host_free(h)). */
@@ -196,7 +197,8 @@ UW_API void uw_host_free(uw_host_t h);
 /* Structural validation of an encoded matrix: shapes, Kraft inequality, length
  * cap, monotone chunk offsets within the stream, per-chunk bit counts between
  * min and max code length, distinct palette, escape bitmap consistent with
- * the group offsets.  UW_OK or UW_ERR_FORMAT / UW_ERR_SHAPE / UW_ERR_ARG. */
+ * the group offsets.  UW_OK or UW_ERR_FORMAT / UW_ERR_SHAPE / UW_ERR_ARG, or
+ * UW_ERR_UNSUPPORTED for a stream longer than 2^27 - 4 words. */
 UW_API uw_status uw_validate_format(const uw_format* f);
 /* Statistics of a host-side encoding (no GPU). */
 UW_API uw_status uw_host_stats(uw_host_t h, uw_stats_t* out);

@@ -191,6 +191,17 @@ def test_validation_accepts_encoder_output(uw, good_arrays):
     assert uw.uw_validate_format(b.fmt) == uw.UW_OK
 
 
+def test_validation_bounds_the_stream_length(uw, good_arrays):
+    """The kernels count a stream's bits (padding included) in 32 bits: a stream
+    of more than 2^27 - 4 words is refused as unsupported.  (The validator does
+    not read the words, so the small buffer behind the view is safe.)"""
+    b = _buffers(uw, good_arrays)
+    b.fmt.n_words = 2**27
+    assert uw.uw_validate_format(b.fmt) == uw.UW_ERR_UNSUPPORTED
+    b.fmt.n_words = 2**27 - 4
+    assert uw.uw_validate_format(b.fmt) == uw.UW_OK
+
+
 def _mutations(a):
     cl = a["code_len"].copy()
     nz = np.nonzero(cl)[0]
