@@ -7,8 +7,11 @@ library is missing; there is no Python or CPU fallback.
 
 The functions carry the names of the C ABI in ``include/unweight.h``.  Tensors
 are ``torch`` tensors on the GPU (device memory and streams come from torch);
-host arrays are ``numpy`` arrays.  Every call raises :class:`UwError` when the
-library returns a status other than ``UW_OK``.
+host arrays are ``numpy`` arrays.  A device tensor goes to the library as its
+data pointer, as in the C ABI: it must be contiguous, on the handle's device
+and at least as large as the header states for that argument (nothing here
+checks its size).  Every call raises :class:`UwError` when the library returns
+a status other than ``UW_OK``.
 """
 from __future__ import annotations
 
