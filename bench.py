@@ -824,7 +824,11 @@ def run_ours(args):
                              rounds=max(args.steps // 2, 3))
             gbs = bt[2] / (bt[0] * 1e-3) / 1e9
             kernels[kind].update({"b2b_launches": bt[1], "b2b_us": 1e3 * bt[0] / bt[1],
-                                  "b2b_GBps": gbs, "b2b_frac_hbm": gbs / peaks["hbm_gbs"]})
+                                  "b2b_GBps": gbs, "b2b_frac_hbm": gbs / peaks["hbm_gbs"],
+                                  "b2b_frac_nominal": gbs / NOMINAL_HBM_GBS,
+                                  # BF16 weights the launch decodes (N*K*2 bytes) per second
+                                  "b2b_decoded_weight_GBps":
+                                      2 * N * K / (bt[0] / bt[1] * 1e-3) / 1e9})
 
     # ---- BF16 torch.matmul on the same box (context only)
     wbf = []
