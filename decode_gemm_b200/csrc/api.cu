@@ -738,7 +738,10 @@ uw_status uw_last_device_status(uw_handle_t h) {
   UW_CK(cudaStreamSynchronize(h->stream));
   uint32_t st = 0;
   UW_CK(cudaMemcpy(&st, h->d_status, 4, cudaMemcpyDeviceToHost));
-  UW_CK(cudaMemset(h->d_status, 0, 4));
+  // cleared on the handle's own stream (which need not synchronise with the
+  // legacy default stream) and waited for, so no later launch can race it
+  UW_CK(cudaMemsetAsync(h->d_status, 0, 4, h->stream));
+  UW_CK(cudaStreamSynchronize(h->stream));
   if (st & kStatusTimeout) return UW_ERR_TIMEOUT;
   if (st & kStatusBadChunk) return UW_ERR_DEVICE;
   return UW_OK;
