@@ -347,7 +347,9 @@ UW_API uw_status uw_get_choice(uw_handle_t h, int64_t M, uw_gemm_config* cfg);
 
 /* Kernel tracing.  While enabled, every kernel the handle launches is
  * bracketed by two CUDA events recorded on the handle's stream (no extra
- * synchronisation).  uw_trace_read synchronises the stream and returns, in
+ * synchronisation); the times are meaningful for calls that launch on that
+ * stream (uw_gemm*, the decode calls), not for the MLP calls, which launch on
+ * the streams they are given.  uw_trace_read synchronises the stream and returns, in
  * launch order, each recorded launch's kind (uw_kernel_kind) and device time
  * in milliseconds, then clears the record.  At most 16384 launches are kept;
  * *count gets the number recorded, of which min(count, capacity) are copied. */
