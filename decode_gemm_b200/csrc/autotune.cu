@@ -17,6 +17,7 @@
 #include <algorithm>
 #include <map>
 #include <cctype>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -238,7 +239,8 @@ struct JParser {
 
 bool num_field(const JVal& o, const char* k, int64_t* out) {
   const JVal* v = o.get(k);
-  if (!v || v->kind != JVal::Num) return false;
+  // (a number outside the int64 range, or not finite, is not a field value)
+  if (!v || v->kind != JVal::Num || !(std::fabs(v->num) < 9.0e18)) return false;
   *out = (int64_t)v->num;
   return true;
 }
