@@ -1,12 +1,17 @@
-"""The bench's roofline numerators on CPU: the algorithmic bytes each kernel
-must move, per weight, on weights drawn like the gate_proj workload
-(N(0, 0.02) BF16, about 2.6 bits per Huffman-coded exponent).
+"""The bench's host logic on CPU.
+
+The roofline numerators: the algorithmic bytes each kernel must move, per
+weight, on weights drawn like the gate_proj workload (N(0, 0.02) BF16, about
+2.6 bits per Huffman-coded exponent).
 
 The pages' accounting: a full decode reads the stream and the sign+mantissa
 bytes and writes BF16 (about 3.33 B per weight), an exponent decode writes one
 byte (1.33), a transcode half a byte (0.83); the palette GEMM reads 1.5 B per
 weight plus the escape rows, the BF16 and exponent GEMMs 2 B, and the
 Huffman-direct product the stream and the sign+mantissa bytes (about 1.34).
+
+The clock record: the median SM clock under load and every throttle reason
+seen active during the timed region, from nvidia-smi's CSV samples.
 """
 import os
 import sys
@@ -55,3 +60,24 @@ def test_algorithmic_bytes_per_weight(stats, kind, lo, hi):
     M = 16
     assert bench._alg_bytes(kind, st, M, N, K) - b == (0 if kind.startswith(("decode_full",
            "decode_exp", "transcode")) else 2 * M * K + 2 * M * N)
+
+
+def _sample(sm, mx=1965, reasons=("Not Active",) * 4):
+    return ", ".join(["0", str(sm), str(mx), "700.00", "0x0000000000000000"] + list(reasons))
+
+
+def test_clock_record():
+    sys.path.insert(0, ROOT)
+    import bench
+    cs = bench.ClockSampler(0)
+    cs.lines = [_sample(345), _sample(1965), _sample(1965), _sample(1950),
+                _sample(1965, reasons=("Not Active", "Not Active", "Not Active", "Active")),
+                "garbage line", _sample("[N/A]")]
+    rec = cs.summary()
+    # the idle sample before the load starts is left out of the median
+    assert rec["sm_mhz"] == 1965 and rec["sm_max_mhz"] == 1965 and rec["samples"] == 5
+    assert rec["reasons"] == ["sw_power_cap"]
+    cs.lines = [_sample(1200, reasons=("Active", "Not Active", "Active", "Not Active"))]
+    assert cs.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    cs.lines = []
+    assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
