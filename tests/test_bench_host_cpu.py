@@ -81,3 +81,14 @@ def test_clock_record():
     assert cs.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     cs.lines = []
     assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+
+def test_traffic_figures_are_for_the_current_sources():
+    """The DRAM traffic the bench reports beside its roofline was captured on
+    the kernel sources as they are (else the bench reports none)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    fam = {"gemm_palette": "gemm", "decode_full": "decode"}
+    assert set(bench.TRAFFIC) == set(fam)
+    for kind, rec in bench.TRAFFIC.items():
+        assert rec["src_sha"] == bench._kernel_src_sha(fam[kind]), kind
