@@ -12,6 +12,7 @@ import oracle.huffman as H
 import oracle.bf16 as B
 import oracle.palette as P
 import oracle.gemm as G
+import oracle.container as Cn
 import tests.test_oracle_pins as pins
 
 
@@ -100,6 +101,55 @@ def _tolerance_full_step(bound, y_ref, bf16_output):
     return tol
 
 
+def _escape_only_if_all_outside(e, palette):
+    # a row escapes only when none of its exponents is in the palette
+    e = np.asarray(e, np.uint8)
+    n, k = e.shape
+    inpal = np.isin(e, np.asarray(palette)).reshape(n, k // 64, 64)
+    return ~inpal.any(axis=2)
+
+
+def _transcode_keeps_escape_ranks(e, palette, esc):
+    # the escape rows keep whatever rank their in-palette exponents have
+    rank = np.zeros(256, np.uint8)
+    rank[np.asarray(palette, np.int64)] = np.arange(16, dtype=np.uint8)
+    return rank[np.asarray(e, np.uint8)]
+
+
+def _silu_wrong_sign(g_bits, u_bits):
+    g, u = B.to_float64(g_bits), B.to_float64(u_bits)
+    return g / (1.0 + np.exp(g)) * u
+
+
+def _offsets_at_chunk_end(starts, total_bits, chunk_syms):
+    # each chunk's offset taken at its last symbol instead of its first
+    n = starts.size
+    c = (n + chunk_syms - 1) // chunk_syms
+    last = np.minimum(np.arange(c) * chunk_syms + chunk_syms - 1, n - 1)
+    return np.concatenate([starts[last], [total_bits]]).astype(np.uint32)
+
+
+def _decode_first_code_off_by_one(words, start_bit, n_syms, lengths):
+    # the first code of each length advanced one too far
+    max_bits, count, syms = H._decode_tables(lengths)
+    w = [int(x) for x in np.asarray(words, np.uint32)] if not isinstance(words, list) else words
+    pos, out = int(start_bit), np.empty(n_syms, np.uint8)
+    for i in range(n_syms):
+        code = first = index = 0
+        for length in range(1, max_bits + 1):
+            code |= (w[pos >> 5] >> (31 - (pos & 31))) & 1
+            pos += 1
+            if 0 <= code - first < count[length]:
+                out[i] = syms[index + code - first]
+                break
+            index += count[length]
+            first = (first + count[length] + 1) << 1
+            code <<= 1
+        else:
+            raise ValueError("not a code word")
+    return out, pos
+
+
 CASES = [
     ("canonical order", oracle, "canonical_codes", _canonical_desc_within_length,
      pins.test_canonical_codes_rfc1951_example),
@@ -121,6 +171,15 @@ CASES = [
      pins.test_transcode_and_nibble_order),
     ("BF16 allowance a full step", G, "tolerance", _tolerance_full_step,
      pins.test_bf16_output_tolerance_branch),
+    ("escape only if all outside", Cn, "escape_rows", _escape_only_if_all_outside,
+     pins.test_planted_rare_exponent_escapes_only_its_row),
+    ("escape rows keep ranks", P, "transcode", _transcode_keeps_escape_ranks,
+     pins.test_transcode_and_nibble_order),
+    ("SiLU sign", G, "swiglu", _silu_wrong_sign, pins.test_swiglu_closed_forms),
+    ("offsets at chunk end", Cn, "chunk_offsets", _offsets_at_chunk_end,
+     lambda: pins.test_chunk_offsets_delimit_chunks(64)),
+    ("decoder first code off by one", H, "decode_chunk", _decode_first_code_off_by_one,
+     lambda: pins.test_roundtrip_lossless("normal")),
 ]
 
 
