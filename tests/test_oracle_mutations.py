@@ -150,6 +150,21 @@ def _decode_first_code_off_by_one(words, start_bit, n_syms, lengths):
     return out, pos
 
 
+def _escape_groups_column_major(e, esc):
+    # groups taken K block first, then row block
+    n, k = e.shape
+    kbs, nbs = k // 64, (n + 127) // 128
+    off, rows = [0], []
+    for kb in range(kbs):
+        for nb in range(nbs):
+            for r in range(nb * 128, min(n, (nb + 1) * 128)):
+                if esc[r, kb]:
+                    rows.append(e[r, kb * 64:(kb + 1) * 64])
+            off.append(len(rows))
+    exp = np.array(rows, np.uint8).reshape(-1, 64) if rows else np.zeros((0, 64), np.uint8)
+    return np.array(off, np.uint32), exp
+
+
 CASES = [
     ("canonical order", oracle, "canonical_codes", _canonical_desc_within_length,
      pins.test_canonical_codes_rfc1951_example),
@@ -180,6 +195,8 @@ CASES = [
      lambda: pins.test_chunk_offsets_delimit_chunks(64)),
     ("decoder first code off by one", H, "decode_chunk", _decode_first_code_off_by_one,
      lambda: pins.test_roundtrip_lossless("normal")),
+    ("escape groups column-major", Cn, "escape_storage", _escape_groups_column_major,
+     pins.test_escape_group_order_hand_example),
 ]
 
 

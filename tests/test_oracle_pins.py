@@ -268,6 +268,23 @@ def test_planted_rare_exponent_escapes_only_its_row():
     assert enc.esc_bits.sum() == (1 << (r % 32))
 
 
+def test_escape_group_order_hand_example():
+    """Escape rows planted at known places; the storage order written out by hand:
+    groups (n // 128, kb) in row-major order, rows ascending inside a group."""
+    w = synthdata.exponent_pattern(256, 128, list(range(110, 126)), seed=19)
+    planted = [(200, 0), (5, 1), (130, 0), (7, 1), (3, 0)]  # (row n, K block kb)
+    for n, kb in planted:
+        k = kb * 64 + 17
+        w[n, k] = (w[n, k] & 0x807F) | (200 << 7)
+    enc = oracle.encode(w, chunk_syms=64)
+    # groups: (0, 0) holds row 3; (0, 1) rows 5, 7; (1, 0) rows 130, 200; (1, 1) none
+    assert [int(v) for v in enc.esc_off] == [0, 1, 3, 5, 5]
+    e = oracle.exponent_bytes(w)
+    order = [(3, 0), (5, 1), (7, 1), (130, 0), (200, 0)]
+    for i, (n, kb) in enumerate(order):
+        assert np.array_equal(enc.esc_exp[i], e[n, kb * 64:(kb + 1) * 64]), (n, kb)
+
+
 def test_escape_invariants_on_heavy_tails():
     w = synthdata.student_t(256, 1024, 3.0, 0.015, seed=13)
     enc = oracle.encode(w, chunk_syms=1024)
