@@ -165,6 +165,27 @@ def _escape_groups_column_major(e, esc):
     return np.array(off, np.uint32), exp
 
 
+def _join_mantissa_low_bits_dropped(s, e):
+    # the mantissa's lowest bit lost when the fields are joined
+    s32 = np.asarray(s, np.uint8).astype(np.uint32)
+    e32 = np.asarray(e, np.uint8).astype(np.uint32)
+    return (((s32 >> 7) << 15) | (e32 << 7) | (s32 & 0x7E)).astype(np.uint16)
+
+
+def _abs_sum_without_abs(x_bits, w_bits):
+    return np.abs(B.to_float64(x_bits) @ B.to_float64(w_bits).T)
+
+
+def _bitmap_bits_reversed(esc):
+    # row n at bit 31 - n % 32 instead of bit n % 32
+    n, kb = esc.shape
+    nw = 4 * ((n + 127) // 128)
+    out = np.zeros((kb, nw), np.uint64)
+    for r in range(n):
+        out[:, r // 32] |= esc[r, :].astype(np.uint64) << np.uint64(31 - r % 32)
+    return out.astype(np.uint32)
+
+
 CASES = [
     ("canonical order", oracle, "canonical_codes", _canonical_desc_within_length,
      pins.test_canonical_codes_rfc1951_example),
@@ -197,6 +218,12 @@ CASES = [
      lambda: pins.test_roundtrip_lossless("normal")),
     ("escape groups column-major", Cn, "escape_storage", _escape_groups_column_major,
      pins.test_escape_group_order_hand_example),
+    ("mantissa bit dropped on join", oracle, "join_fields", _join_mantissa_low_bits_dropped,
+     pins.test_field_split_roundtrip_all_patterns),
+    ("bound without the absolute values", G, "abs_product_sum", _abs_sum_without_abs,
+     pins.test_gemm_matches_fsum_triple_loop),
+    ("escape bitmap bit order", Cn, "escape_bitmap", _bitmap_bits_reversed,
+     pins.test_planted_rare_exponent_escapes_only_its_row),
 ]
 
 
